@@ -1,0 +1,159 @@
+"""Plausible mistakes planted in the oracle must each fail at least one pin.
+
+Every mutant replaces one oracle function (on the CPU, through monkeypatch)
+with a version carrying a typical slip: an off-by-one in the successive rule,
+a dropped modulo, interleaved instead of half-split RoPE pairing, a flipped
+sign, a wrong frequency exponent, a missing softmax scale, a log2 LSE, a
+causal off-by-one, a wrong GQA mapping, a shifted chunk origin, a broken
+partial merge, or a decode that reads one key too few.  The pins of
+``test_oracle_pins`` must reject each one.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import dca_oracle as orc
+from tests import test_oracle_pins as pins
+
+_orig_query_position = orc.query_position
+_orig_rotate = orc.rotate
+_orig_piece = orc.piece
+_orig_softmax_row = orc.softmax_row
+
+
+def _qpos_succ_le(i, j, s, c):
+    i = np.asarray(i, np.int64)
+    j = np.asarray(j, np.int64)
+    im = i % s
+    p = orc.piece(i, j, s)
+    succ = np.where(im <= c - s, s + im, c - 1)
+    out = np.where(p == 0, im, np.where(p == 1, succ, c - 1))
+    return np.where(p < 0, -1, out)
+
+
+def _qpos_succ_c(i, j, s, c):
+    out = _orig_query_position(i, j, s, c)
+    i = np.asarray(i, np.int64)
+    p = orc.piece(i, j, s)
+    return np.where((p == 1) & (i % s >= c - s), c, out)
+
+
+def _qpos_inter_succ(i, j, s, c):
+    # inter piece wrongly treated like the successive piece
+    i = np.asarray(i, np.int64)
+    j = np.asarray(j, np.int64)
+    im = i % s
+    p = orc.piece(i, j, s)
+    succ = np.where(im < c - s, s + im, c - 1)
+    out = np.where(p == 0, im, succ)
+    return np.where(p < 0, -1, out)
+
+
+def _qpos_succ_as_intra(i, j, s, c):
+    out = _orig_query_position(i, j, s, c)
+    p = orc.piece(i, j, s)
+    return np.where(p == 1, np.asarray(i) % s, out)
+
+
+def _key_abs(j, s):
+    return np.asarray(j, np.int64)
+
+
+def _rotate_interleaved(x, pos, base):
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    ang = np.asarray(pos, np.float64)[..., None] * orc.inv_freq(D, base)
+    cos, sin = np.cos(ang), np.sin(ang)
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * cos - b * sin
+    out[..., 1::2] = b * cos + a * sin
+    return out
+
+
+def _rotate_sign(x, pos, base):
+    return _orig_rotate(x, -np.asarray(pos), base)
+
+
+def _inv_freq_half(D, base):
+    k = np.arange(D // 2, dtype=np.float64)
+    return np.power(np.float64(base), -k / D)
+
+
+def _scale_one(D, scale):
+    return 1.0
+
+
+def _softmax_log2(z, v):
+    o, lse = _orig_softmax_row(z, v)
+    return o, lse / np.log(2.0)
+
+
+def _softmax_drop_last(z, v):
+    # causal off-by-one: the diagonal key is left out of the row
+    if len(z) == 1:
+        return _orig_softmax_row(z, v)
+    return _orig_softmax_row(z[:-1], v[:-1])
+
+
+def _kv_head_mod(h, Hq, Hkv):
+    return h % Hkv
+
+
+def _piece_shift(i, j, s):
+    i = np.asarray(i, np.int64)
+    j = np.asarray(j, np.int64)
+    diff = (i + 1) // s - (j + 1) // s
+    out = np.where(diff == 0, 0, np.where(diff == 1, 1, 2))
+    return np.where(j > i, -1, out).astype(np.int8)
+
+
+def _merge_mean(o_parts, lse_parts):
+    return np.mean(np.asarray(o_parts), axis=0), np.max(lse_parts)
+
+
+def _decode_short(q, k_cache_rot, v_cache, t, s, c, base=10000.0, scale=0.0,
+                  batches=None, heads=None):
+    return _ORIG_DECODE(q, k_cache_rot, v_cache, np.asarray(t) - 1, s, c, base,
+                        scale, batches, heads)
+
+
+_ORIG_DECODE = orc.dca_decode
+
+MUTANTS = {
+    "succ_rule_le": ("query_position", _qpos_succ_le),
+    "succ_far_pos_c": ("query_position", _qpos_succ_c),
+    "inter_as_succ": ("query_position", _qpos_inter_succ),
+    "succ_as_intra": ("query_position", _qpos_succ_as_intra),
+    "key_not_mod_s": ("key_position", _key_abs),
+    "rope_interleaved": ("rotate", _rotate_interleaved),
+    "rope_sign": ("rotate", _rotate_sign),
+    "theta_exponent": ("inv_freq", _inv_freq_half),
+    "no_softmax_scale": ("_scale", _scale_one),
+    "lse_log2": ("softmax_row", _softmax_log2),
+    "causal_off_by_one": ("softmax_row", _softmax_drop_last),
+    "gqa_modulo": ("kv_head", _kv_head_mod),
+    "chunk_origin_shift": ("piece", _piece_shift),
+    "merge_mean": ("merge_partials", _merge_mean),
+    "decode_short": ("dca_decode", _decode_short),
+}
+
+
+def _some_pin_fails():
+    for pin in pins.PINS:
+        try:
+            pin()
+        except AssertionError:
+            return True
+    return False
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert not _some_pin_fails()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    assert _some_pin_fails(), f"mutant {name} passed every pin"

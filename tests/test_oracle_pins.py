@@ -1,0 +1,290 @@
+"""Pins that hold the fp64 oracle to facts fixed outside itself.
+
+Each pin is a module-level function ``pin_*`` so that the mutation tests can
+re-run them against a deliberately broken oracle; the ``test_*`` wrappers run
+them against the oracle as committed.  Sources of each fact:
+
+* hand-worked index tables under ``tests/golden/`` (the DCA rule applied by
+  hand; no code wrote them);
+* the bound "effective distance never exceeds the pretrained window" and
+  "intra-chunk distance is the exact, unscaled i - j" (Dual-Chunk Attention:
+  Training-Free 100k+ Context Guide, "Architectural Taxonomy" and
+  "Intra-Chunk Attention");
+* closed-form piece counts (pure counting over chunk sizes);
+* reduction to ordinary causal RoPE attention when the whole sequence fits
+  in one chunk, checked against torch's scaled_dot_product_attention with the
+  rotation done by complex multiplication;
+* closed forms for Q = 0 and constant V, RoPE relativity (Guide, "The
+  Problem": the score depends only on the position difference), literal
+  rotation values, and the split-softmax identity.
+"""
+
+import math
+import pathlib
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dca_oracle as orc
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+TABLES = [("dca_index_s4_c6_L12.txt", 4, 6), ("dca_index_s3_c5_L9.txt", 3, 5),
+          ("dca_index_s3_c3_L7.txt", 3, 3), ("dca_index_s2_c5_L7.txt", 2, 5)]
+
+
+def parse_table(name):
+    lines = [ln for ln in (GOLDEN / name).read_text().splitlines()
+             if ln.strip() and not ln.startswith("#")]
+    rows = lines[1:]
+    L = len(rows)
+    pc = np.full((L, L), -1, np.int8)
+    dist = np.full((L, L), -1, np.int64)
+    for r, line in enumerate(rows):
+        toks = line.split()
+        assert int(toks[0]) == r
+        assert len(toks) == L + 1
+        for j, tok in enumerate(toks[1:]):
+            if tok == ".":
+                continue
+            pc[r, j] = {"A": 0, "S": 1, "I": 2}[tok[0]]
+            dist[r, j] = int(tok[1:])
+    return pc, dist
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _complex_rotate(x, pos, base):
+    """RoPE as complex multiplication: (x_k + i x_{k+D/2}) * e^{i pos theta_k}."""
+    D = x.shape[-1]
+    half = D // 2
+    theta = np.array([base ** (-(2.0 * k) / D) for k in range(half)])
+    z = (x[..., :half] + 1j * x[..., half:]) * np.exp(1j * np.asarray(pos)[..., None] * theta)
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+# --------------------------------------------------------------------------
+# pins
+# --------------------------------------------------------------------------
+
+def pin_worked_tables():
+    for name, s, c in TABLES:
+        want_pc, want_d = parse_table(name)
+        L = want_pc.shape[0]
+        qpos, kpos, pc = orc.index_map(L, s, c)
+        assert (pc == want_pc).all(), name
+        d = np.where(pc >= 0, qpos - kpos, -1)
+        assert (d == want_d).all(), name
+        jj = np.broadcast_to(np.arange(L), (L, L))
+        assert (kpos[pc >= 0] == (jj % s)[pc >= 0]).all(), name
+
+
+def pin_distance_bounds():
+    for s, c in [(4, 6), (3, 5), (5, 8), (8, 8), (2, 5), (7, 9), (192, 256), (1, 1)]:
+        for L in list(range(1, 41)) + [3 * c + 7]:
+            qpos, kpos, pc = orc.index_map(L, s, c)
+            i = np.arange(L)[:, None] + 0 * np.arange(L)[None, :]
+            j = np.arange(L)[None, :] + 0 * np.arange(L)[:, None]
+            causal = j <= i
+            assert ((pc >= 0) == causal).all()
+            d = qpos - kpos
+            assert d[causal].min() >= 0 and d[causal].max() <= c - 1
+            intra = pc == orc.PIECE_INTRA
+            assert (d[intra] == (i - j)[intra]).all()
+            near = (pc == orc.PIECE_SUCC) & ((i % s) < c - s)
+            assert (d[near] == (i - j)[near]).all()
+            far = ((pc == orc.PIECE_SUCC) & ((i % s) >= c - s)) | (pc == orc.PIECE_INTER)
+            assert (d[far] >= c - s).all() and (d[far] <= c - 1).all()
+
+
+def closed_form_counts(L, s):
+    n = [min(s, L - k * s) for k in range(-(-L // s))]
+    intra = sum(nk * (nk + 1) // 2 for nk in n)
+    succ = sum(nk * s for nk in n[1:])
+    inter = sum(nk * (k - 1) * s for k, nk in enumerate(n) if k >= 2)
+    return intra, succ, inter
+
+
+def pin_piece_counts():
+    # tiny prefill workload: L=1024, s=192 (c=256); sums to L(L+1)/2
+    qpos, kpos, pc = orc.index_map(1024, 192, 256)
+    got = tuple(int((pc == p).sum()) for p in (0, 1, 2))
+    assert got == (94720, 159744, 270336)
+    assert sum(got) == 1024 * 1025 // 2
+    for L, s, c in [(1, 3, 5), (17, 4, 6), (40, 5, 8), (100, 7, 9), (64, 16, 16)]:
+        qpos, kpos, pc = orc.index_map(L, s, c)
+        got = tuple(int((pc == p).sum()) for p in (0, 1, 2))
+        assert got == closed_form_counts(L, s)
+
+
+def pin_rotation_literals():
+    # D=4, base 10000: theta = (1, 0.01); half-split pairs (0,2) and (1,3)
+    e0, e1 = np.array([1.0, 0, 0, 0]), np.array([0, 1.0, 0, 0])
+    e2 = np.array([0, 0, 1.0, 0])
+    np.testing.assert_allclose(orc.rotate(e0, 1, 10000.0),
+                               [math.cos(1), 0, math.sin(1), 0], atol=1e-15)
+    np.testing.assert_allclose(orc.rotate(e1, 1, 10000.0),
+                               [0, math.cos(0.01), 0, math.sin(0.01)], atol=1e-15)
+    np.testing.assert_allclose(orc.rotate(e2, 3, 10000.0),
+                               [-math.sin(3), 0, math.cos(3), 0], atol=1e-15)
+    x = _rand((5, 7, 3, 16), 1)
+    pos = np.arange(7)[None, :, None] * 37
+    np.testing.assert_allclose(orc.rotate(x, pos, 500.0),
+                               _complex_rotate(x, pos, 500.0), atol=1e-12)
+
+
+def pin_rope_relativity():
+    q, k = _rand(16, 2), _rand(16, 3)
+    for p, r in [(0, 0), (5, 2), (255, 0), (4095, 3071)]:
+        ref = orc.rotate(q, p, 10000.0) @ orc.rotate(k, r, 10000.0)
+        for delta in (1, 17, 1000):
+            got = orc.rotate(q, p + delta, 10000.0) @ orc.rotate(k, r + delta, 10000.0)
+            assert abs(got - ref) < 1e-12
+
+
+def _sdpa_reference(Q, K, V, base):
+    """Causal RoPE attention via torch SDPA (fp64 CPU), complex-rotated inputs."""
+    B, L, Hq, D = Q.shape
+    G = Hq // K.shape[2]
+    pos = np.arange(L)[None, :, None]
+    qr = torch.from_numpy(_complex_rotate(Q, pos, base)).permute(0, 2, 1, 3)
+    kr = torch.from_numpy(_complex_rotate(K, pos, base)).permute(0, 2, 1, 3)
+    v = torch.from_numpy(np.asarray(V, np.float64)).permute(0, 2, 1, 3)
+    kr, v = kr.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1)
+    O = torch.nn.functional.scaled_dot_product_attention(qr, kr, v, is_causal=True)
+    z = (qr @ kr.transpose(-1, -2)) / math.sqrt(D)
+    z = z.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), -math.inf)
+    lse = torch.logsumexp(z, dim=-1)
+    return O.permute(0, 2, 1, 3).numpy(), lse.numpy()
+
+
+def pin_plain_rope_matches_sdpa():
+    Q, K, V = _rand((2, 13, 4, 8), 4), _rand((2, 13, 2, 8), 5), _rand((2, 13, 2, 8), 6)
+    O, LSE = orc.plain_rope_attention(Q, K, V, base=100.0)
+    O_ref, LSE_ref = _sdpa_reference(Q, K, V, 100.0)
+    np.testing.assert_allclose(O, O_ref, atol=1e-12)
+    np.testing.assert_allclose(LSE, LSE_ref, atol=1e-12)
+
+
+def pin_single_chunk_is_plain_rope():
+    # L <= s: every pair is intra and both positions are absolute
+    Q, K, V = _rand((1, 11, 4, 8), 7), _rand((1, 11, 2, 8), 8), _rand((1, 11, 2, 8), 9)
+    O, LSE = orc.dca_prefill(Q, K, V, s=12, c=16, base=100.0)
+    O_ref, LSE_ref = _sdpa_reference(Q, K, V, 100.0)
+    np.testing.assert_allclose(O, O_ref, atol=1e-12)
+    np.testing.assert_allclose(LSE, LSE_ref, atol=1e-12)
+    # L <= c with w <= s: chunk-1 queries all have i mod s < w, so the
+    # successive piece sees i - j and DCA is again plain RoPE attention
+    Q, K, V = _rand((1, 16, 2, 8), 10), _rand((1, 16, 2, 8), 11), _rand((1, 16, 2, 8), 12)
+    O, LSE = orc.dca_prefill(Q, K, V, s=10, c=16, base=100.0)
+    O_ref, LSE_ref = _sdpa_reference(Q, K, V, 100.0)
+    np.testing.assert_allclose(O, O_ref, atol=1e-10)
+    np.testing.assert_allclose(LSE, LSE_ref, atol=1e-10)
+
+
+def pin_long_sequence_differs_from_plain():
+    # beyond c the remapping must change the result (guards a no-op oracle)
+    Q, K, V = _rand((1, 24, 1, 8), 13), _rand((1, 24, 1, 8), 14), _rand((1, 24, 1, 8), 15)
+    O, _ = orc.dca_prefill(Q, K, V, s=4, c=6, base=2.0)
+    O_ref, _ = _sdpa_reference(Q, K, V, 2.0)
+    assert np.abs(O - O_ref)[0, 6:].max() > 1e-3
+    np.testing.assert_allclose(O[0, :4], O_ref[0, :4], atol=1e-12)
+
+
+def pin_q_zero_closed_form():
+    L = 40
+    K, V = _rand((1, L, 2, 8), 16), _rand((1, L, 2, 8), 17)
+    Q = np.zeros((1, L, 4, 8))
+    O, LSE = orc.dca_prefill(Q, K, V, s=6, c=10)
+    for i in range(L):
+        for h in range(4):
+            np.testing.assert_allclose(LSE[0, h, i], math.log(i + 1), atol=1e-13)
+            np.testing.assert_allclose(O[0, i, h], V[0, :i + 1, h // 2].mean(0), atol=1e-13)
+
+
+def pin_constant_v():
+    L = 30
+    Q, K = _rand((1, L, 2, 8), 18), _rand((1, L, 1, 8), 19)
+    v = _rand(8, 20)
+    V = np.broadcast_to(v, (1, L, 1, 8)).copy()
+    O, _ = orc.dca_prefill(Q, K, V, s=5, c=8)
+    np.testing.assert_allclose(O[0], np.broadcast_to(v, (L, 2, 8)), atol=1e-13)
+
+
+def pin_gqa_mapping():
+    # q head h reads kv head h // G: same as expanding K, V by repeat_interleave
+    Q, K, V = _rand((1, 20, 6, 8), 21), _rand((1, 20, 2, 8), 22), _rand((1, 20, 2, 8), 23)
+    O, LSE = orc.dca_prefill(Q, K, V, s=4, c=7)
+    Ke, Ve = np.repeat(K, 3, axis=2), np.repeat(V, 3, axis=2)
+    O2, LSE2 = orc.dca_prefill(Q, Ke, Ve, s=4, c=7)
+    np.testing.assert_allclose(O, O2, atol=1e-14)
+    np.testing.assert_allclose(LSE, LSE2, atol=1e-14)
+
+
+def pin_decode_equals_prefill_row():
+    B, L, s, c = 2, 30, 6, 10
+    Q, K, V = _rand((B, L, 4, 8), 24), _rand((B, L, 2, 8), 25), _rand((B, L, 2, 8), 26)
+    k_rot = _complex_rotate(K, (np.arange(L) % s)[None, :, None], 10000.0)
+    t = np.array([29, 17])
+    q = np.stack([Q[b, t[b]] for b in range(B)])
+    O, LSE = orc.dca_decode(q, k_rot, V, t, s, c)
+    for b in range(B):
+        ref = orc.dca_prefill_rows(Q[b:b + 1], K[b:b + 1], V[b:b + 1], s, c,
+                                   rows=[int(t[b])])
+        for h in range(4):
+            o, lse = ref[(0, h, int(t[b]))]
+            np.testing.assert_allclose(O[b, h], o, atol=1e-12)
+            np.testing.assert_allclose(LSE[b, h], lse, atol=1e-12)
+
+
+def pin_merge_partials():
+    z, v = _rand(50, 27) * 3, _rand((50, 8), 28)
+    o_full, lse_full = orc.softmax_row(z, v)
+    cuts = [0, 7, 31, 50]
+    parts = [orc.softmax_row(z[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+    o, lse = orc.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    np.testing.assert_allclose(o, o_full, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_full, atol=1e-13)
+    # LSE is the natural-log normaliser of the scaled scores
+    np.testing.assert_allclose(lse_full, math.log(np.exp(z).sum()), atol=1e-12)
+
+
+def pin_rule_positions():
+    s, c = 5, 8
+    n = 23
+    i = np.arange(n)
+    assert (orc.rule_positions(n, orc.POS_KEY, s, c) == i % s).all()
+    assert (orc.rule_positions(n, orc.POS_Q_INTRA, s, c) == i % s).all()
+    assert (orc.rule_positions(n, orc.POS_Q_INTER, s, c) == c - 1).all()
+    assert (orc.rule_positions(n, orc.POS_ABSOLUTE, s, c, 9) == i + 9).all()
+    # derived closed form of the successive rule: min(s + i mod s, c - 1)
+    for s2, c2 in [(5, 8), (3, 3), (2, 5), (3072, 4096)]:
+        m = 3 * s2 + 1
+        got = orc.rule_positions(m, orc.POS_Q_SUCC, s2, c2)
+        assert (got == np.minimum(s2 + np.arange(m) % s2, c2 - 1)).all()
+    # the successive rule agrees with the index map's previous-chunk column
+    qpos, _, pc = orc.index_map(n, s, c)
+    succ = orc.rule_positions(n, orc.POS_Q_SUCC, s, c)
+    for r in range(s, n):
+        assert qpos[r, (r // s - 1) * s] == succ[r]
+
+
+PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
+        pin_rotation_literals, pin_rope_relativity, pin_plain_rope_matches_sdpa,
+        pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
+        pin_q_zero_closed_form, pin_constant_v, pin_gqa_mapping,
+        pin_decode_equals_prefill_row, pin_merge_partials, pin_rule_positions]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin()
+
+
+def test_rejects_bad_chunking():
+    with pytest.raises(ValueError):
+        orc.index_map(8, 5, 4)
+    with pytest.raises(ValueError):
+        orc.index_map(8, 0, 4)
