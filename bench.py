@@ -1,0 +1,442 @@
+"""Benchmark of the DCA hot path on B200.
+
+One step = one pass of the whole path on synthetic data:
+  prefill  (Llama-2-7B attention shape, L=16384, 32/32 heads, D=128,
+            c=4096, s=3072): fused RoPE, then DCA attention;
+  decode   (16 sequences, 64/8 heads, D=128, t ~ U[32768, 65536), cache
+            pre-rotated at j mod s): split-KV kernel, then LSE merge.
+`value` is prefill TFLOP/s (algorithmic causal FLOPs 4*D*Hq*B*L(L+1)/2 over
+the device time of RoPE + attention); decode KV GB/s is reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
+(the path has no exchange step), times are max-reduced over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_attention_dca_b200 import workloads as W  # noqa: E402
+
+PREFILL = "llama2_7b_16k"
+DECODE = "decode_b16"
+METRIC = "DCA prefill TFLOP/s (bf16, % of TC peak); decode KV GB/s (% of HBM peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the dominant kernels from the committed ncu
+    summary (profiles/traffic.json), or {} when none was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f)
+    return {}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the prefill workload
+# ---------------------------------------------------------------------------
+class _F64:
+    """float64 numpy view of a CPU torch tensor, converted per index."""
+
+    def __init__(self, t):
+        self.t, self.shape = t, tuple(t.shape)
+
+    def __getitem__(self, idx):
+        return self.t[idx].to(torch.float64).numpy()
+
+
+_CPU_INPUTS = {}
+
+
+def oracle_sample(budget_s: float, seed: int = 0):
+    """Time the oracle on random (row, head) outputs of the prefill workload
+    until `budget_s` seconds have passed; returns (TFLOP/s, rows, heads, s)."""
+    import numpy as np
+    from oracle import dca_oracle as orc
+    cfg = W.CONFIGS[PREFILL]
+    if PREFILL not in _CPU_INPUTS:
+        _CPU_INPUTS[PREFILL] = W.make_prefill_inputs(cfg)
+    Q, K, V = _CPU_INPUTS[PREFILL]
+    rng = np.random.default_rng(seed)
+    flops = 0.0
+    n_rows = 0
+    heads = [0]
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        rows = sorted(int(x) for x in rng.integers(0, cfg["L"], size=8))
+        orc.dca_prefill_rows(_F64(Q), _F64(K), _F64(V), cfg["s"], cfg["c"],
+                             cfg["base"], rows=rows, heads=heads)
+        flops += sum(4.0 * cfg["D"] * (i + 1) for i in rows) * len(heads)
+        n_rows += len(rows)
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, n_rows, len(heads), dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    per_step = []
+    rows_total = 0
+    budget = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for k in range(args.warmup + args.steps):
+        tf, n_rows, _, dt = oracle_sample(budget, seed=k)
+        if k >= args.warmup:
+            per_step.append((tf, dt))
+            rows_total += n_rows
+    value = statistics.mean(x[0] for x in per_step)
+    ms = statistics.mean(x[1] for x in per_step) * 1e3
+    cores = blas_threads()
+    sample = (f"{rows_total} random query rows x 1 head of the {PREFILL} prefill workload, "
+              f"fp64 oracle, ~{budget:.0f} s per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL, **_cfg_summary(W.CONFIGS[PREFILL])},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _cfg_summary(cfg):
+    keys = ("B", "L", "Hq", "Hkv", "D", "c", "s", "Tcap")
+    return {k: cfg[k] for k in keys if k in cfg}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, dev):
+    import long_context_attention_dca_b200 as dca
+    from long_context_attention_dca_b200 import build
+    build.build()
+    lib = dca.lib()
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    import ctypes
+    P = ctypes.c_void_p
+
+    pc = W.CONFIGS[PREFILL]
+    dc = W.CONFIGS[DECODE]
+    Q, K, V = W.make_prefill_inputs(pc, device=dev)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    s, c, base = pc["s"], pc["c"], pc["base"]
+    ws_bytes = dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    path = dca.dca_prefill_path(L, D, s, c)
+
+    t_dec, q_dec, Kc, Vc = W.make_decode_inputs(dc, device=dev)
+    Bd, Hqd, Dd = q_dec.shape
+    Tcap, Hkvd = Kc.shape[1], Kc.shape[2]
+    dws_bytes = dca.dca_attn_decode_workspace(Bd, Hqd, Dd, Tcap)
+    dws = torch.empty(dws_bytes, dtype=torch.uint8, device=dev)
+    Od = torch.empty_like(q_dec)
+    LSEd = torch.empty(Bd, Hqd, dtype=torch.float32, device=dev)
+    t_host = t_dec.cpu()
+
+    def chk(st):
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+
+    def rope():
+        chk(lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s, c,
+                                 base, P(ws.data_ptr()), ws_bytes, P(sptr)))
+
+    def attn():
+        chk(lib.dca_prefill_attention(P(V.data_ptr()), P(O.data_ptr()), P(LSE.data_ptr()), B, L,
+                                      Hq, Hkv, D, s, c, 0.0, 0, P(ws.data_ptr()), ws_bytes,
+                                      P(sptr)))
+
+    def decode():
+        chk(lib.dca_attn_decode(P(q_dec.data_ptr()), P(Kc.data_ptr()), P(Vc.data_ptr()),
+                                P(t_dec.data_ptr()), P(Od.data_ptr()), P(LSEd.data_ptr()), Bd,
+                                Hqd, Hkvd, Dd, Tcap, dc["s"], dc["c"], dc["base"], 0.0,
+                                P(dws.data_ptr()), dws_bytes, P(sptr)))
+
+    for _ in range(args.warmup):
+        rope(); attn(); decode()
+    torch.cuda.synchronize(dev)
+    dca.dca_sync_status(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.15)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        e = ev[k]
+        e[0].record(stream); rope()
+        e[1].record(stream); attn()
+        e[2].record(stream); decode()
+        e[3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    _barrier(world)
+    dca.dca_sync_status(dev)
+
+    total_ms = t_start.elapsed_time(t_end)
+    rope_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = _max_over_ranks(total_ms, world, dev)
+    prefill_ms = _max_over_ranks(sum(rope_ms) + sum(attn_ms), world, dev)
+    attn_sum = _max_over_ranks(sum(attn_ms), world, dev)
+    rope_sum = _max_over_ranks(sum(rope_ms), world, dev)
+    dec_sum = _max_over_ranks(sum(dec_ms), world, dev)
+
+    flops = W.prefill_flops(pc)
+    dec_bytes = W.decode_bytes(dc, t_host.tolist())
+    rope_bytes = float(B * L * (Hq + Hkv) * D * 2 + B * L * (3 * Hq + Hkv) * D * 2)
+    value = world * flops * args.steps / (prefill_ms * 1e-3) / 1e12
+    attn_tflops = flops * args.steps / (attn_sum * 1e-3) / 1e12
+    dec_gbs = world * dec_bytes * args.steps / (dec_sum * 1e-3) / 1e9
+    rope_gbs = rope_bytes * args.steps / (rope_sum * 1e-3) / 1e9
+
+    peaks, peak_kind = load_peaks()
+    traffic = load_traffic()
+    tpk = peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+
+    # ---- e2e through the public API with host buffers ----
+    e2e = run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc)
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tf, n_rows, n_heads, dt = oracle_sample(args.cpu_seconds)
+            cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"{n_rows} random query rows x {n_heads} head of the {PREFILL} "
+                             f"prefill workload, fp64 oracle, {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16, Llama-2 attention shapes)",
+            "config": {"workload": PREFILL, **_cfg_summary(pc),
+                       "decode_workload": DECODE, "decode": _cfg_summary(dc),
+                       "prefill_path": {1: "general (warp MMA)",
+                                        2: "tcgen05/TMEM/TMA"}.get(path, str(path)),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (Q,K,V 402 MB; decode KV 3.2 GB)"},
+            "prefill": {"tflops_rope_plus_attn": value / world, "attn_tflops": attn_tflops,
+                        "attn_ms": attn_sum / args.steps, "rope_ms": rope_sum / args.steps,
+                        "rope_gbs": rope_gbs, "frac_of_peak": attn_tflops / tpk},
+            "decode": {"value": dec_gbs, "unit": "GB/s", "ms": dec_sum / args.steps,
+                       "bytes_per_step": dec_bytes, "frac_of_hbm_peak": dec_gbs / world / hbm},
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpk,
+                         "unit": "TFLOP/s", "frac": attn_tflops / tpk,
+                         "traffic": traffic.get("prefill_attn"),
+                         "kernel": "prefill attention", "peak_source": f"{peak_kind} burst"},
+            "rooflines": {
+                "decode_split_kv+merge": {"bound": "hbm", "achieved": dec_gbs / world,
+                                          "peak": hbm, "unit": "GB/s",
+                                          "frac": dec_gbs / world / hbm,
+                                          "traffic": traffic.get("decode")},
+                "prefill_rope": {"bound": "hbm", "achieved": rope_gbs, "peak": hbm,
+                                 "unit": "GB/s", "frac": rope_gbs / hbm,
+                                 "traffic": traffic.get("prefill_rope")}},
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    return line
+
+
+def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
+    """Prefill through dca_attn_prefill with pinned host inputs: each step
+    copies Q, K, V host->device, runs the path and reads O and LSE back.
+    Decode through dca_attn_decode with q and t copied in and O, LSE read back
+    (the KV cache is device-resident state, as in serving)."""
+    hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    hO = torch.empty(Q.shape, dtype=torch.bfloat16).pin_memory()
+    hL = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], dtype=torch.float32).pin_memory()
+    hq, ht = q_dec.cpu().pin_memory(), t_dec.cpu().pin_memory()
+    dq, dt_ = torch.empty_like(q_dec), torch.empty_like(t_dec)
+    hOd = torch.empty(q_dec.shape, dtype=torch.bfloat16).pin_memory()
+    hLd = torch.empty(q_dec.shape[:2], dtype=torch.float32).pin_memory()
+    s, c = pc["s"], pc["c"]
+    ws = torch.empty(dca.dca_attn_prefill_workspace(*Q.shape[:3], K.shape[2], Q.shape[3]),
+                     dtype=torch.uint8, device=dev)
+    dws = torch.empty(dca.dca_attn_decode_workspace(*q_dec.shape[:2], q_dec.shape[2],
+                                                    Kc.shape[1]), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dQ.copy_(hQ, non_blocking=True); dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        O, LSE = dca.dca_attn_prefill(dQ, dK, dV, s, c, pc["base"], workspace=ws)
+        hO.copy_(O, non_blocking=True); hL.copy_(LSE, non_blocking=True)
+        dq.copy_(hq, non_blocking=True); dt_.copy_(ht, non_blocking=True)
+        Od, LSEd = dca.dca_attn_decode(dq, Kc, Vc, dt_, dc["s"], dc["c"], dc["base"],
+                                       workspace=dws)
+        hOd.copy_(Od, non_blocking=True); hLd.copy_(LSEd, non_blocking=True)
+
+    n = max(1, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = _max_over_ranks(a.elapsed_time(b), world, dev) / n
+    flops = W.prefill_flops(pc)
+    h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hq, ht))
+    d2h = sum(x.numel() * x.element_size() for x in (hO, hL, hOd, hLd))
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "api": "dca_attn_prefill + dca_attn_decode (decode KV cache device-resident)"}
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, rank, world)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    try:
+        line = run_ours(args, rank, world, dev)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

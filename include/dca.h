@@ -1,0 +1,165 @@
+/*
+ * dca.h -- C ABI of the B200 (sm_100a) Dual Chunk Attention library.
+ *
+ * Dual Chunk Attention (DCA) extends a RoPE model past its pretraining length
+ * c without training by cutting the sequence into chunks of s tokens and
+ * remapping rotary positions so that every query-key distance stays inside
+ * [0, c-1] (Training-Free Long-Context Scaling of Large Language Models,
+ * Abstract: intra-chunk and inter-chunk attention pieces that fit Flash
+ * Attention; Dual-Chunk Attention: Training-Free 100k+ Context Guide,
+ * "Architectural Taxonomy").  With w = c - s and im = i mod s:
+ *
+ *   key j                        rotated once at j mod s
+ *   query i vs key in same chunk rotated at im                    (intra)
+ *   query i vs previous chunk    rotated at s + im if im < w,
+ *                                else c - 1                       (successive)
+ *   query i vs earlier chunks    rotated at c - 1                 (inter)
+ *
+ * and all causal keys j <= i share ONE softmax.  Scores are
+ * scale * <R(q_pos) q_i, R(k_pos) k_j> with half-split RoPE pairing
+ * (element k with k + D/2, angle pos * base^(-2k/D)); scale = 1/sqrt(D) when
+ * 0 is passed.  LSE is the natural-log normaliser of the scaled scores.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated; the caller owns all memory
+ *     and the library allocates none.  Scratch comes from the caller's
+ *     workspace (size from the *_workspace query; 256-byte alignment is
+ *     recommended, 16-byte alignment is required of every pointer).
+ *   - Tensors are contiguous.  bf16 unless stated; LSE is fp32.
+ *       Q, O      [B][L][Hq][D]        K, V          [B][L][Hkv][D]
+ *       LSE       [B][Hq][L]           q (decode)    [B][Hq][D]
+ *       Kcache, Vcache [B][Tcap][Hkv][D]   t (decode) int32 [B] on device
+ *   - GQA: query head h reads kv head h / (Hq / Hkv).
+ *   - Supported: D in {64, 128}; Hq % Hkv == 0; 1 <= s <= c; base > 0.
+ *     Sizes of 0 (B, L) are accepted and do nothing.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous: they enqueue kernels and return.  A kernel-side failure
+ *     (a pipeline wait that ran past its deadline, a decode position outside
+ *     the cache) is recorded in a per-device error word and reported by
+ *     dca_sync_status().  Nothing is thrown across the ABI and no kernel traps.
+ *   - On a non-DCA_OK return nothing was enqueued; dca_last_error_string()
+ *     (per host thread) says why.
+ */
+#ifndef DCA_B200_H
+#define DCA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DCA_ABI_VERSION 1
+
+typedef enum dca_status {
+  DCA_OK = 0,
+  DCA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, ... */
+  DCA_ERR_UNSUPPORTED = 2, /* D not 64/128, Hq % Hkv != 0, s > c, ...     */
+  DCA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed            */
+  DCA_ERR_TIMEOUT = 4,     /* a kernel wait passed its deadline (device)   */
+  DCA_ERR_WORKSPACE = 5    /* workspace missing or smaller than required   */
+} dca_status_t;
+
+typedef enum dca_pos_rule {
+  DCA_POS_KEY = 0,      /* (pos_offset + row) mod s                          */
+  DCA_POS_Q_INTRA = 1,  /* (pos_offset + row) mod s                          */
+  DCA_POS_Q_SUCC = 2,   /* s + im if im < c - s else c - 1, im = (..) mod s   */
+  DCA_POS_Q_INTER = 3,  /* c - 1                                             */
+  DCA_POS_ABSOLUTE = 4  /* pos_offset + row: plain RoPE                      */
+} dca_pos_rule_t;
+
+typedef enum dca_prefill_path {
+  DCA_PATH_AUTO = 0,    /* tcgen05 path when D == 128 and s % 128 == 0      */
+  DCA_PATH_GENERAL = 1, /* warp-MMA path: any s, D 64 or 128                */
+  DCA_PATH_TCGEN05 = 2  /* tcgen05/TMEM/TMA path: D == 128, s % 128 == 0     */
+} dca_prefill_path_t;
+
+/* Rotate x [B][L][H][D] (bf16) into out (same shape; may equal x) with
+ * half-split RoPE at the position a DCA rule assigns to each row; row r of a
+ * sequence has absolute index i = pos_offset + r.  Builds a decode cache
+ * pre-rotated at j mod s (DCA_POS_KEY), or the query rotations of one piece.
+ * Source: RoPE relative form (Guide, "The Problem"); the DCA rule above.
+ * Angles in fp64, rotation in fp32, result rounded to bf16 (nearest even).
+ * Errors: INVALID_ARG (null/misaligned pointer, negative size or offset),
+ * UNSUPPORTED (D, rule, or s/c for a DCA rule), CUDA. */
+dca_status_t dca_rope_rotate(const void* x, void* out, int B, int L, int H, int D,
+                             int pos_offset, int s, int c, float base, dca_pos_rule_t rule,
+                             void* stream);
+
+/* Workspace bytes needed by dca_attn_prefill / dca_prefill_rope /
+ * dca_prefill_attention: the rotated keys Krot [B][L][Hkv][D] and the three
+ * query rotations Qrot [3][B][L][Hq][D] (intra, successive, inter), bf16.
+ * Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_workspace(int B, int L, int Hq, int Hkv, int D);
+
+/* Step 1 of prefill alone: fused RoPE.  Reads unrotated Q and K once and
+ * writes Krot (keys at j mod s) and the three Qrot planes into the workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_prefill_rope(const void* Q, const void* K, int B, int L, int Hq, int Hkv,
+                              int D, int s, int c, float base, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* Step 2 of prefill alone: DCA attention over a workspace filled by
+ * dca_prefill_rope with the same sizes, s and c.  Writes O (bf16) and LSE
+ * (fp32).  `path` is a dca_prefill_path_t; DCA_PATH_TCGEN05 on a shape it
+ * does not cover returns UNSUPPORTED.  Tiling follows the Flash-DCA idea
+ * (Guide, "Flash-DCA: Fusing DCA into FlashAttention Tiling Loops"): the
+ * query rotation is chosen per key tile by chunk relation; one online
+ * softmax (fp32 running max and sum) spans all three pieces.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, int L, int Hq,
+                                   int Hkv, int D, int s, int c, float scale, int path,
+                                   const void* workspace, size_t ws_bytes, void* stream);
+
+/* DCA prefill: Q, K unrotated, V as given -> O [B][L][Hq][D] bf16 and
+ * LSE [B][Hq][L] fp32.  Equivalent to dca_prefill_rope followed by
+ * dca_prefill_attention with DCA_PATH_AUTO.  Source: arXiv Abstract (chunked
+ * intra/inter attention in one Flash-style pass); Guide, "Flash-DCA".
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              int B, int L, int Hq, int Hkv, int D, int s, int c, float base,
+                              float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/* Which prefill path DCA_PATH_AUTO takes for these sizes (1 general,
+ * 2 tcgen05), or 0 for unsupported arguments. */
+int dca_prefill_path(int L, int D, int s, int c);
+
+/* Workspace bytes needed by dca_attn_decode: per (sequence, query head,
+ * split of 1024 keys) an unnormalised fp32 output row plus running max and
+ * sum.  Returns 0 for unsupported arguments. */
+size_t dca_attn_decode_workspace(int B, int Hq, int D, int Tcap);
+
+/* DCA decode of one new token per sequence.  q [B][Hq][D] is the UNROTATED
+ * query at absolute index t[b]; Kcache holds keys ALREADY rotated at j mod s
+ * (e.g. by dca_rope_rotate with DCA_POS_KEY); keys and values 0 .. t[b] are
+ * valid (the new token's own K/V included).  Writes O [B][Hq][D] bf16 and
+ * LSE [B][Hq] fp32.  Split-KV across SMs then an LSE merge (Guide,
+ * "Strategic Recommendations", item 3: pair DCA with FlashDecoding).
+ * t lives on the device; a t[b] outside [0, Tcap) is reported by
+ * dca_sync_status (INVALID_ARG) and that sequence's outputs are NaN.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_decode(const void* q, const void* Kcache, const void* Vcache,
+                             const int* t, void* O, float* LSE, int B, int Hq, int Hkv, int D,
+                             int Tcap, int s, int c, float base, float scale, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/* Dense L x L tables of the index rule for small L (L <= 8192): qpos and
+ * kpos (int32, -1 where masked) and piece (int8: 0 intra, 1 successive,
+ * 2 inter, -1 masked, i.e. j > i), row-major [i][j].
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+dca_status_t dca_debug_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
+                                 void* stream);
+
+/* Synchronise `stream`, then read and clear the current device's kernel error
+ * word: DCA_OK, DCA_ERR_TIMEOUT (a pipeline wait gave up), DCA_ERR_INVALID_ARG
+ * (a device-side argument check failed) or DCA_ERR_CUDA. */
+dca_status_t dca_sync_status(void* stream);
+
+/* Message for the last non-OK status returned on this host thread. */
+const char* dca_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCA_B200_H */

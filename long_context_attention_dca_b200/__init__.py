@@ -1,1 +1,215 @@
-"""Placeholder; replaced by the ctypes binding once the library exists."""
+"""Dual Chunk Attention (DCA) for NVIDIA B200 -- thin Python binding.
+
+Every function here marshals torch tensors into the C ABI declared in
+``include/dca.h`` (data pointers, sizes, the current CUDA stream) and calls
+the in-tree shared library ``libdca_b200.so``.  All arithmetic runs in the
+library's sm_100a kernels; there is no CPU or PyTorch fallback: if the library
+is missing or a call fails, a ``DcaError`` is raised.  PyTorch is used only
+for device memory (outputs and the workspace the C ABI asks for) and streams.
+
+Build the library with ``python -m long_context_attention_dca_b200.build``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "DcaError", "lib", "lib_path",
+    "DCA_POS_KEY", "DCA_POS_Q_INTRA", "DCA_POS_Q_SUCC", "DCA_POS_Q_INTER", "DCA_POS_ABSOLUTE",
+    "DCA_PATH_AUTO", "DCA_PATH_GENERAL", "DCA_PATH_TCGEN05",
+    "dca_rope_rotate", "dca_attn_prefill_workspace", "dca_prefill_rope",
+    "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
+    "dca_attn_decode_workspace", "dca_attn_decode", "dca_debug_index_map",
+    "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
+]
+
+DCA_POS_KEY, DCA_POS_Q_INTRA, DCA_POS_Q_SUCC, DCA_POS_Q_INTER, DCA_POS_ABSOLUTE = range(5)
+DCA_PATH_AUTO, DCA_PATH_GENERAL, DCA_PATH_TCGEN05 = range(3)
+_STATUS = {0: "DCA_OK", 1: "DCA_ERR_INVALID_ARG", 2: "DCA_ERR_UNSUPPORTED",
+           3: "DCA_ERR_CUDA", 4: "DCA_ERR_TIMEOUT", 5: "DCA_ERR_WORKSPACE"}
+
+lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdca_b200.so")
+
+_I, _F, _P, _Z = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+# name -> (restype, argtypes); mirrors include/dca.h
+_SIGS = {
+    "dca_rope_rotate": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "dca_attn_prefill_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_prefill_rope": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "dca_prefill_attention": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _Z, _P]),
+    "dca_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _Z,
+                              _P]),
+    "dca_prefill_path": (_I, [_I, _I, _I, _I]),
+    "dca_attn_decode_workspace": (_Z, [_I, _I, _I, _I]),
+    "dca_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
+                             _Z, _P]),
+    "dca_debug_index_map": (_I, [_I, _I, _I, _P, _P, _P, _P]),
+    "dca_sync_status": (_I, [_P]),
+    "dca_last_error_string": (ctypes.c_char_p, []),
+}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+
+class DcaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise DcaError(3, f"{lib_path} not built; run "
+                              "python -m long_context_attention_dca_b200.build")
+        handle = ctypes.CDLL(lib_path)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(handle, name)
+            f.restype, f.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise DcaError(status, lib().dca_last_error_string().decode())
+
+
+def _stream(t: torch.Tensor | None = None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise DcaError(1, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous():
+        raise DcaError(1, f"{name} must be a contiguous {ndim}-d {dtype} tensor, "
+                          f"got {t.dtype} {tuple(t.shape)}")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def dca_last_error_string() -> str:
+    return lib().dca_last_error_string().decode()
+
+
+def dca_sync_status(device=None) -> None:
+    """Synchronise the current stream and raise if a kernel reported an error."""
+    dev = torch.device(device) if device is not None else torch.device("cuda")
+    _check(lib().dca_sync_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+def dca_rope_rotate(x: torch.Tensor, rule: int, s: int, c: int, base: float = 10000.0,
+                    pos_offset: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Rotate x [B, L, H, D] bf16 at the positions of a DCA rule (see dca.h)."""
+    _need(x, "x", torch.bfloat16, 4)
+    out = torch.empty_like(x) if out is None else out
+    _need(out, "out", torch.bfloat16, 4)
+    B, L, H, D = x.shape
+    _check(lib().dca_rope_rotate(_ptr(x), _ptr(out), B, L, H, D, pos_offset, s, c, base, rule,
+                                 _stream(x)))
+    return out
+
+
+def dca_attn_prefill_workspace(B: int, L: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().dca_attn_prefill_workspace(B, L, Hq, Hkv, D))
+
+
+def dca_prefill_path(L: int, D: int, s: int, c: int) -> int:
+    return int(lib().dca_prefill_path(L, D, s, c))
+
+
+def dca_prefill_rope(Q, K, s, c, base=10000.0, workspace=None):
+    """Fused RoPE step alone; returns the filled workspace (uint8 tensor)."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    nbytes = dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    _check(lib().dca_prefill_rope(_ptr(Q), _ptr(K), B, L, Hq, Hkv, D, s, c, base, _ptr(ws),
+                                  ws.numel(), _stream(Q)))
+    return ws
+
+
+def dca_prefill_attention(V, workspace, Hq, s, c, scale=0.0, path=DCA_PATH_AUTO, O=None,
+                          LSE=None):
+    """Attention step alone over a workspace from dca_prefill_rope."""
+    _need(V, "V", torch.bfloat16, 4)
+    B, L, Hkv, D = V.shape
+    O = torch.empty((B, L, Hq, D), dtype=torch.bfloat16, device=V.device) if O is None else O
+    LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=V.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 4)
+    _need(LSE, "LSE", torch.float32, 3)
+    _check(lib().dca_prefill_attention(_ptr(V), _ptr(O), _ptr(LSE), B, L, Hq, Hkv, D, s, c,
+                                       scale, path, _ptr(workspace), workspace.numel(),
+                                       _stream(V)))
+    return O, LSE
+
+
+def dca_attn_prefill(Q, K, V, s, c, base=10000.0, scale=0.0, workspace=None, O=None,
+                     LSE=None):
+    """DCA prefill: returns (O [B, L, Hq, D] bf16, LSE [B, Hq, L] fp32)."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    nbytes = dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    O = torch.empty_like(Q) if O is None else O
+    LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 4)
+    _need(LSE, "LSE", torch.float32, 3)
+    _check(lib().dca_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L, Hq, Hkv,
+                                  D, s, c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_decode_workspace(B: int, Hq: int, D: int, Tcap: int) -> int:
+    return int(lib().dca_attn_decode_workspace(B, Hq, D, Tcap))
+
+
+def dca_attn_decode(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, workspace=None,
+                    O=None, LSE=None):
+    """DCA decode: q [B, Hq, D] unrotated; caches [B, Tcap, Hkv, D] with keys
+    pre-rotated at j mod s; t int32 [B] on device.  Returns (O, LSE)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    _need(t, "t", torch.int32, 1)
+    B, Hq, D = q.shape
+    Tcap, Hkv = Kcache.shape[1], Kcache.shape[2]
+    nbytes = dca_attn_decode_workspace(B, Hq, D, Tcap)
+    ws = _workspace(nbytes, q.device) if workspace is None else workspace
+    O = torch.empty_like(q) if O is None else O
+    LSE = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if LSE is None else LSE
+    _check(lib().dca_attn_decode(_ptr(q), _ptr(Kcache), _ptr(Vcache), _ptr(t), _ptr(O),
+                                 _ptr(LSE), B, Hq, Hkv, D, Tcap, s, c, base, scale, _ptr(ws),
+                                 ws.numel(), _stream(q)))
+    return O, LSE
+
+
+def dca_debug_index_map(L: int, s: int, c: int, device="cuda"):
+    """Dense (qpos, kpos, piece) tables [L, L] computed on the GPU."""
+    qpos = torch.empty((L, L), dtype=torch.int32, device=device)
+    kpos = torch.empty((L, L), dtype=torch.int32, device=device)
+    piece = torch.empty((L, L), dtype=torch.int8, device=device)
+    _check(lib().dca_debug_index_map(L, s, c, _ptr(qpos), _ptr(kpos), _ptr(piece),
+                                     _stream(qpos)))
+    return qpos, kpos, piece

@@ -1,0 +1,271 @@
+// General DCA prefill attention: warp-level MMA (m16n8k16, bf16 -> fp32).
+//
+// Serves every chunking the tensor-core path does not (s not a multiple of
+// 128, D = 64) and doubles as an independent GPU cross-check of it.  Inputs
+// are the outputs of the fused RoPE kernel: Qrot [3][B][L][Hq][D] (the query
+// rotated for the intra, successive and inter pieces) and Krot [B][L][Hkv][D]
+// (keys at j mod s); V [B][L][Hkv][D] as given.
+//
+// Flash-style tiling (Dual-Chunk Attention: Training-Free 100k+ Context
+// Guide, "Flash-DCA: Fusing DCA into FlashAttention Tiling Loops"): a CTA owns
+// 64 query rows of one head, walks key tiles of 64 up to the diagonal and
+// keeps one online softmax (running max and sum in fp32) across the three
+// pieces.  Each warp (16 rows) derives from its rows' and the tile's chunk
+// ranges which pieces the tile touches; it computes S once per present piece
+// with that piece's query rotation and, when more than one is present
+// (tiles straddling a chunk boundary), selects per element by chunk relation.
+#include "dca_common.cuh"
+#include "dca_index.cuh"
+#include "dca_kernels.cuh"
+
+namespace dca {
+namespace {
+
+constexpr int kBM = 64;
+constexpr int kBN = 64;
+constexpr int kThreads = 128;
+
+// Row-major tile of `D` bf16 per row with 16-byte chunks XOR-swizzled by row,
+// so ldmatrix row addresses of one 8x8 matrix hit distinct banks.
+template <int D>
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)(row * D * 2 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D>
+__device__ __forceinline__ void compute_s(float (&acc)[8][4], uint32_t q_base, uint32_t k_base,
+                                          int warp, int lane) {
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    uint32_t a[4];
+    ldsm_x4(a, q_base + swz<D>(warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3),
+                               ks * 2 + (lane >> 4)));
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      uint32_t bk[4];
+      ldsm_x4(bk, k_base + swz<D>(np * 16 + (lane & 7) + ((lane >> 4) << 3),
+                                  ks * 2 + ((lane >> 3) & 1)));
+      const uint32_t b0[2] = {bk[0], bk[1]};
+      const uint32_t b1[2] = {bk[2], bk[3]};
+      mma_bf16_16816(acc[2 * np], a, b0);
+      mma_bf16_16816(acc[2 * np + 1], a, b1);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
+    const __nv_bfloat16* __restrict__ Qrot, const __nv_bfloat16* __restrict__ Krot,
+    const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ O, float* __restrict__ LSE,
+    int B, int L, int Hq, int Hkv, int s, int c, float scale_log2) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + 3 * kBM * D * 2;
+  const uint32_t sV = sK + 2 * kBN * D * 2;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int num_qt = (L + kBM - 1) / kBM;
+  const int qt = num_qt - 1 - (int)blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (Hq / Hkv);
+  const int q0 = qt * kBM;
+  const size_t plane = (size_t)B * L * Hq * D;
+
+  // Query tile, all three rotations.
+  for (int idx = tid; idx < 3 * kBM * CH; idx += kThreads) {
+    const int v = idx / (kBM * CH), r = (idx / CH) % kBM, ch = idx % CH;
+    const int row = q0 + r;
+    const bool ok = row < L;
+    const __nv_bfloat16* src =
+        Qrot + v * plane + (((size_t)b * L + (ok ? row : 0)) * Hq + h) * D + ch * 8;
+    cp_async_16(sQ + v * kBM * D * 2 + swz<D>(r, ch), src, ok);
+  }
+  auto load_kv = [&](int stage, int kt) {
+    for (int idx = tid; idx < kBN * CH; idx += kThreads) {
+      const int r = idx / CH, ch = idx % CH;
+      const int row = kt * kBN + r;
+      const bool ok = row < L;
+      const size_t off = (((size_t)b * L + (ok ? row : 0)) * Hkv + hk) * D + ch * 8;
+      cp_async_16(sK + stage * kBN * D * 2 + swz<D>(r, ch), Krot + off, ok);
+      cp_async_16(sV + stage * kBN * D * 2 + swz<D>(r, ch), V + off, ok);
+    }
+  };
+  load_kv(0, 0);
+  cp_async_commit();
+
+  const int g = lane >> 2, t4 = lane & 3;
+  const int r0 = q0 + warp * 16;
+  const int row_a = r0 + g, row_b = r0 + g + 8;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  float o[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+
+  const int n_kt = qt + 1;  // key tiles 0 .. diagonal (kBM == kBN)
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int stage = kt & 1;
+    if (kt + 1 < n_kt) {
+      load_kv(stage ^ 1, kt + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+
+    const int k0 = kt * kBN;
+    const uint32_t kb = sK + stage * kBN * D * 2;
+    const uint32_t vb = sV + stage * kBN * D * 2;
+
+    // Pieces this warp's rows meet in this tile (chunk differences form an
+    // interval; causal pairs have difference >= 0).
+    const int ci_lo = r0 / s, ci_hi = (r0 + 15) / s;
+    const int cj_lo = k0 / s, cj_hi = (k0 + kBN - 1) / s;
+    const int dmin = max(ci_lo - cj_hi, 0), dmax = ci_hi - cj_lo;
+    const bool need[3] = {dmin == 0, dmin <= 1 && dmax >= 1, dmax >= 2};
+    const int npieces = (int)need[0] + (int)need[1] + (int)need[2];
+
+    float sacc[8][4];
+    if (npieces == 1) {
+      const int p = need[0] ? 0 : (need[1] ? 1 : 2);
+      compute_s<D>(sacc, sQ + p * kBM * D * 2, kb, warp, lane);
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+      const int ci_a = row_a / s, ci_b = row_b / s;
+#pragma unroll 1
+      for (int p = 0; p < 3; ++p) {
+        if (!need[p]) continue;
+        float tmp[8][4];
+        compute_s<D>(tmp, sQ + p * kBM * D * 2, kb, warp, lane);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = k0 + nt * 8 + 2 * t4 + (e & 1);
+            const int d = ((e >> 1) ? ci_b : ci_a) - j / s;
+            const int pe = d <= 0 ? 0 : (d == 1 ? 1 : 2);
+            if (pe == p) sacc[nt][e] = tmp[nt][e];
+          }
+      }
+    }
+
+    // scale, causal mask, row max
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = k0 + nt * 8 + 2 * t4 + (e & 1);
+        const int i = (e >> 1) ? row_b : row_a;
+        const float v = (j <= i) ? sacc[nt][e] * scale_log2 : -INFINITY;
+        sacc[nt][e] = v;
+        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+      }
+    float m_use[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+      const float m_new = fmaxf(m_run[r], mx[r]);
+      m_use[r] = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = fast_exp2(m_run[r] - m_use[r]);
+      m_run[r] = m_new;
+      l_run[r] *= alpha;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        o[i][2 * r] *= alpha;
+        o[i][2 * r + 1] *= alpha;
+      }
+    }
+    uint32_t pa[4][4];  // P as A fragments, one per 16-key step
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const float p0 = fast_exp2(sacc[nt][0] - m_use[0]);
+      const float p1 = fast_exp2(sacc[nt][1] - m_use[0]);
+      const float p2 = fast_exp2(sacc[nt][2] - m_use[1]);
+      const float p3 = fast_exp2(sacc[nt][3] - m_use[1]);
+      l_run[0] += p0 + p1;
+      l_run[1] += p2 + p3;
+      pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
+      pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
+    }
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+      for (int np = 0; np < D / 16; ++np) {
+        uint32_t bv[4];
+        ldsm_x4_t(bv, vb + swz<D>(kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3),
+                                  np * 2 + (lane >> 4)));
+        const uint32_t b0[2] = {bv[0], bv[1]};
+        const uint32_t b1[2] = {bv[2], bv[3]};
+        mma_bf16_16816(o[2 * np], pa[kk], b0);
+        mma_bf16_16816(o[2 * np + 1], pa[kk], b1);
+      }
+    }
+    __syncthreads();
+  }
+
+  // finalize
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+  }
+  const float inv_a = 1.f / l_run[0], inv_b = 1.f / l_run[1];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    const int col = i * 8 + 2 * t4;
+    if (row_a < L)
+      *reinterpret_cast<uint32_t*>(O + (((size_t)b * L + row_a) * Hq + h) * D + col) =
+          pack_bf16(o[i][0] * inv_a, o[i][1] * inv_a);
+    if (row_b < L)
+      *reinterpret_cast<uint32_t*>(O + (((size_t)b * L + row_b) * Hq + h) * D + col) =
+          pack_bf16(o[i][2] * inv_b, o[i][3] * inv_b);
+  }
+  if (t4 == 0) {
+    const float ln2 = 0.69314718055994530942f;
+    if (row_a < L) LSE[((size_t)b * Hq + h) * L + row_a] = (m_run[0] + log2f(l_run[0])) * ln2;
+    if (row_b < L) LSE[((size_t)b * Hq + h) * L + row_b] = (m_run[1] + log2f(l_run[1])) * ln2;
+  }
+}
+
+template <int D>
+cudaError_t launch_mma(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
+                       int B, int L, int Hq, int Hkv, int s, int c, float scale,
+                       cudaStream_t stream) {
+  const int smem = (3 * kBM + 4 * kBN) * D * 2;
+  auto kern = prefill_attn_mma_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((L + kBM - 1) / kBM, Hq, B);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  kern<<<grid, kThreads, smem, stream>>>(
+      static_cast<const __nv_bfloat16*>(Qrot), static_cast<const __nv_bfloat16*>(Krot),
+      static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(O), LSE, B, L, Hq, Hkv,
+      s, c, scale_log2);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const void* V, void* O,
+                                    float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
+                                    int c, float scale, cudaStream_t stream) {
+  if (L == 0 || B == 0 || Hq == 0) return cudaSuccess;
+  if (D == 64) return launch_mma<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, stream);
+  return launch_mma<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, stream);
+}
+
+}  // namespace dca

@@ -1,0 +1,289 @@
+// C ABI of the DCA library: argument checks, workspace carving, dispatch to
+// the kernels, TMA tensor-map encoding and the status / error-word plumbing.
+// No function here allocates device memory; no exception crosses the ABI.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "../../include/dca.h"
+#include "dca_common.cuh"
+#include "dca_kernels.cuh"
+
+namespace dca {
+
+namespace {
+
+thread_local std::string t_last_error = "no error";
+
+dca_status_t fail(dca_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+dca_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(DCA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr bool kHaveTcgen05 = false;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define DCA_CHECK_PTR(p)                                                              \
+  do {                                                                                \
+    if ((p) == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: %s is null", fn, #p);   \
+    if (!aligned16(p))                                                                \
+      return fail(DCA_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, #p);      \
+  } while (0)
+
+dca_status_t check_chunking(const char* fn, int s, int c, float base) {
+  if (s < 1 || c < 1) return fail(DCA_ERR_INVALID_ARG, "%s: need s >= 1 and c >= 1", fn);
+  if (s > c)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: chunk s=%d exceeds pretraining length c=%d", fn, s, c);
+  if (!(base > 0.f)) return fail(DCA_ERR_INVALID_ARG, "%s: RoPE base must be > 0", fn);
+  return DCA_OK;
+}
+
+dca_status_t check_heads(const char* fn, int B, int L, int Hq, int Hkv, int D) {
+  if (B < 0 || L < 0) return fail(DCA_ERR_INVALID_ARG, "%s: negative B or L", fn);
+  if (Hq < 1 || Hkv < 1) return fail(DCA_ERR_INVALID_ARG, "%s: need Hq >= 1, Hkv >= 1", fn);
+  if (Hq % Hkv != 0)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: Hq=%d is not a multiple of Hkv=%d", fn, Hq, Hkv);
+  if (D != 64 && D != 128) return fail(DCA_ERR_UNSUPPORTED, "%s: D=%d (need 64 or 128)", fn, D);
+  return DCA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct PrefillWs {
+  void* qrot;
+  void* krot;
+  size_t bytes;
+};
+
+PrefillWs prefill_ws_layout(void* base, int B, int L, int Hq, int Hkv, int D) {
+  const size_t qbytes = align256((size_t)3 * B * L * Hq * D * 2);
+  const size_t kbytes = align256((size_t)B * L * Hkv * D * 2);
+  char* p = static_cast<char*>(base);
+  return PrefillWs{p, p ? p + qbytes : nullptr, qbytes + kbytes};
+}
+
+int auto_path(int D, int s) { return (kHaveTcgen05 && D == 128 && s % 128 == 0) ? DCA_PATH_TCGEN05 : DCA_PATH_GENERAL; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+}  // namespace
+
+bool encode_tensor_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box,
+                            CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                  const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                  reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace dca
+
+using namespace dca;
+
+extern "C" {
+
+dca_status_t dca_rope_rotate(const void* x, void* out, int B, int L, int H, int D,
+                             int pos_offset, int s, int c, float base, dca_pos_rule_t rule,
+                             void* stream) {
+  const char* fn = "dca_rope_rotate";
+  if (B < 0 || L < 0 || H < 1 || pos_offset < 0)
+    return fail(DCA_ERR_INVALID_ARG, "%s: bad sizes B=%d L=%d H=%d offset=%d", fn, B, L, H,
+                pos_offset);
+  if (D != 64 && D != 128) return fail(DCA_ERR_UNSUPPORTED, "%s: D=%d (need 64 or 128)", fn, D);
+  if ((int)rule < 0 || (int)rule > 4) return fail(DCA_ERR_UNSUPPORTED, "%s: rule %d", fn, rule);
+  if (rule != DCA_POS_ABSOLUTE) {
+    dca_status_t st = check_chunking(fn, s, c, base);
+    if (st != DCA_OK) return st;
+  } else if (!(base > 0.f)) {
+    return fail(DCA_ERR_INVALID_ARG, "%s: RoPE base must be > 0", fn);
+  }
+  if ((long long)pos_offset + L > 2147483647LL)
+    return fail(DCA_ERR_INVALID_ARG, "%s: positions overflow int32", fn);
+  if ((long long)B * L == 0) return DCA_OK;
+  DCA_CHECK_PTR(x);
+  DCA_CHECK_PTR(out);
+  cudaError_t e = launch_rope_rotate(x, out, B, L, H, D, pos_offset, s, c, base, (int)rule,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+size_t dca_attn_prefill_workspace(int B, int L, int Hq, int Hkv, int D) {
+  if (B < 0 || L < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
+  return prefill_ws_layout(nullptr, B, L, Hq, Hkv, D).bytes;
+}
+
+dca_status_t dca_prefill_rope(const void* Q, const void* K, int B, int L, int Hq, int Hkv,
+                              int D, int s, int c, float base, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  const char* fn = "dca_prefill_rope";
+  dca_status_t st = check_heads(fn, B, L, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if ((long long)B * L == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(workspace);
+  PrefillWs ws = prefill_ws_layout(workspace, B, L, Hq, Hkv, D);
+  if (ws_bytes < ws.bytes)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes,
+                ws.bytes);
+  cudaError_t e = launch_prefill_rope(Q, K, ws.qrot, ws.krot, B, L, Hq, Hkv, D, s, c, base,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+int dca_prefill_path(int L, int D, int s, int c) {
+  if (L < 0 || (D != 64 && D != 128) || s < 1 || s > c) return 0;
+  return auto_path(D, s);
+}
+
+dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, int L, int Hq,
+                                   int Hkv, int D, int s, int c, float scale, int path,
+                                   const void* workspace, size_t ws_bytes, void* stream) {
+  const char* fn = "dca_prefill_attention";
+  dca_status_t st = check_heads(fn, B, L, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, 10000.f);
+  if (st != DCA_OK) return st;
+  if (path < DCA_PATH_AUTO || path > DCA_PATH_TCGEN05)
+    return fail(DCA_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
+  if (path == DCA_PATH_AUTO) path = auto_path(D, s);
+  if (path == DCA_PATH_TCGEN05 && auto_path(D, s) != DCA_PATH_TCGEN05)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: tcgen05 path needs D == 128 and s %% 128 == 0", fn);
+  if ((long long)B * L == 0) return DCA_OK;
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  PrefillWs ws = prefill_ws_layout(const_cast<void*>(workspace), B, L, Hq, Hkv, D);
+  if (ws_bytes < ws.bytes)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes,
+                ws.bytes);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (path == DCA_PATH_TCGEN05)
+    e = launch_prefill_attn_sm100(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, c, sc,
+                                  sm_count(), strm);
+  else
+    e = launch_prefill_attn_mma(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, c, sc, strm);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              int B, int L, int Hq, int Hkv, int D, int s, int c, float base,
+                              float scale, void* workspace, size_t ws_bytes, void* stream) {
+  dca_status_t st = dca_prefill_rope(Q, K, B, L, Hq, Hkv, D, s, c, base, workspace, ws_bytes,
+                                     stream);
+  if (st != DCA_OK) return st;
+  return dca_prefill_attention(V, O, LSE, B, L, Hq, Hkv, D, s, c, scale, DCA_PATH_AUTO,
+                               workspace, ws_bytes, stream);
+}
+
+size_t dca_attn_decode_workspace(int B, int Hq, int D, int Tcap) {
+  if (B < 0 || Hq < 1 || (D != 64 && D != 128) || Tcap < 1) return 0;
+  return decode_workspace_bytes(B, Hq, D, Tcap);
+}
+
+dca_status_t dca_attn_decode(const void* q, const void* Kcache, const void* Vcache,
+                             const int* t, void* O, float* LSE, int B, int Hq, int Hkv, int D,
+                             int Tcap, int s, int c, float base, float scale, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_decode";
+  dca_status_t st = check_heads(fn, B, 1, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (Tcap < 1) return fail(DCA_ERR_INVALID_ARG, "%s: Tcap=%d", fn, Tcap);
+  if (B == 0) return DCA_OK;
+  DCA_CHECK_PTR(q);
+  DCA_CHECK_PTR(Kcache);
+  DCA_CHECK_PTR(Vcache);
+  if (t == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: t is null", fn);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = decode_workspace_bytes(B, Hq, D, Tcap);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes,
+                need);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaError_t e = launch_decode(q, Kcache, Vcache, t, O, LSE, B, Hq, Hkv, D, Tcap, s, c, base,
+                                sc, workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+dca_status_t dca_debug_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
+                                 void* stream) {
+  const char* fn = "dca_debug_index_map";
+  if (L < 0 || L > 8192) return fail(DCA_ERR_INVALID_ARG, "%s: L=%d (0..8192)", fn, L);
+  dca_status_t st = check_chunking(fn, s, c, 1.f);
+  if (st != DCA_OK) return st;
+  if (L == 0) return DCA_OK;
+  if (!qpos || !kpos || !piece) return fail(DCA_ERR_INVALID_ARG, "%s: null output", fn);
+  cudaError_t e = launch_index_map(L, s, c, qpos, kpos, piece, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+dca_status_t dca_sync_status(void* stream) {
+  const char* fn = "dca_sync_status";
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  int code = 0, site = 0;
+  e = cudaMemcpyFromSymbol(&code, g_error_code, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&site, g_error_site, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (code == 0) return DCA_OK;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_error_code, &zero, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_error_site, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (code == kDevTimeout)
+    return fail(DCA_ERR_TIMEOUT, "%s: a kernel wait passed its deadline (site %d)", fn, site);
+  return fail(DCA_ERR_INVALID_ARG, "%s: device-side argument check failed (site %d)", fn, site);
+}
+
+const char* dca_last_error_string(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Host-side launchers of the DCA kernels (internal to the library; the public
+// C ABI lives in include/dca.h and dca_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dca {
+
+enum PosRule : int { kPosKey = 0, kPosQIntra = 1, kPosQSucc = 2, kPosQInter = 3, kPosAbsolute = 4 };
+
+cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, int D,
+                               int pos_offset, int s, int c, float base, int rule,
+                               cudaStream_t stream);
+
+// Writes Krot [B][L][Hkv][D] and Qrot [3][B][L][Hq][D] (intra, succ, inter).
+cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
+                                int L, int Hq, int Hkv, int D, int s, int c, float base,
+                                cudaStream_t stream);
+
+// General prefill attention (warp MMA; any s, D in {64, 128}).
+cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const void* V, void* O,
+                                    float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
+                                    int c, float scale, cudaStream_t stream);
+
+// tcgen05/TMEM/TMA prefill attention (D = 128, s % 128 == 0).
+cudaError_t launch_prefill_attn_sm100(const void* Qrot, const void* Krot, const void* V, void* O,
+                                      float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
+                                      int c, float scale, int num_sms, cudaStream_t stream);
+
+// Split-KV decode + LSE merge.
+size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap);
+cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const int* t, void* O,
+                          float* LSE, int B, int Hq, int Hkv, int D, int Tcap, int s, int c,
+                          float base, float scale, void* workspace, cudaStream_t stream);
+
+cudaError_t launch_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
+                             cudaStream_t stream);
+
+// Driver entry point for building TMA tensor maps (resolved once).
+bool encode_tensor_map_bf16(CUtensorMap* map, const void* base, int rank,
+                            const uint64_t* dims, const uint64_t* strides_bytes,
+                            const uint32_t* box, CUtensorMapSwizzle swizzle);
+
+}  // namespace dca

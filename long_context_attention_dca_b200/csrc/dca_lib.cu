@@ -1,0 +1,9 @@
+// Single translation unit of the library: every kernel file is included here
+// so that the device error word in dca_api.cu is one object shared by all
+// kernels without relocatable device code.
+#include "dca_api.cu"
+#include "rope.cu"
+#include "index_map.cu"
+#include "attn_prefill_mma.cu"
+#include "attn_prefill_sm100.cu"
+#include "attn_decode.cu"

@@ -1,0 +1,125 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+declared in include/dca.h, and rejects bad arguments before touching the GPU.
+
+Every call here returns from the library's argument checks; none launches a
+kernel, so the tests run on a machine without a GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_attention_dca_b200 as dca
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dca.h")
+
+
+def _header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dca_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_attention_dca_b200 import build
+    build.build()
+    return dca.lib()
+
+
+def test_header_declares_the_binding_surface():
+    assert _header_functions() == sorted(dca.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+    # C linkage: the dynamic symbol table has the plain names
+    out = os.popen(f"nm -D --defined-only {dca.lib_path}").read()
+    exported = set(re.findall(r"\bT (dca_[a-z0-9_]+)\b", out))
+    assert set(_header_functions()) <= exported
+
+
+def test_workspace_queries(lib):
+    # Qrot (3 planes) + Krot, bf16, each rounded up to 256 bytes
+    B, L, Hq, Hkv, D = 1, 1000, 4, 2, 64
+    q = 3 * B * L * Hq * D * 2
+    k = B * L * Hkv * D * 2
+    up = lambda x: (x + 255) // 256 * 256
+    assert dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D) == up(q) + up(k)
+    assert dca.dca_attn_prefill_workspace(1, 10, 3, 2, 64) == 0  # Hq % Hkv
+    assert dca.dca_attn_prefill_workspace(1, 10, 2, 2, 96) == 0  # D
+    # decode: one fp32 row + (max, sum) per (b, head, split of 1024 keys)
+    assert dca.dca_attn_decode_workspace(16, 64, 128, 65536) == 16 * 64 * 64 * 130 * 4
+    assert dca.dca_attn_decode_workspace(2, 8, 64, 1025) == 2 * 8 * 2 * 66 * 4
+
+
+def test_prefill_path_selection(lib):
+    assert dca.dca_prefill_path(16384, 128, 3072, 4096) in (dca.DCA_PATH_GENERAL,
+                                                              dca.DCA_PATH_TCGEN05)
+    assert dca.dca_prefill_path(1024, 64, 192, 256) == dca.DCA_PATH_GENERAL
+    assert dca.dca_prefill_path(1024, 128, 192, 256) == dca.DCA_PATH_GENERAL
+    assert dca.dca_prefill_path(1024, 128, 300, 256) == 0  # s > c
+    assert dca.dca_prefill_path(1024, 96, 128, 256) == 0
+
+
+P = ctypes.c_void_p
+
+
+def _code(ret):
+    return int(ret)
+
+
+def test_argument_errors_return_codes(lib):
+    fake = P(0x10000)      # 16-byte aligned, never dereferenced on these paths
+    odd = P(0x10008)       # 8-byte aligned only
+    ws = P(0x20000)
+    # rope: null input, misaligned output, bad D, bad rule, s > c
+    assert _code(lib.dca_rope_rotate(None, fake, 1, 8, 1, 64, 0, 4, 6, 1e4, 0, None)) == 1
+    assert _code(lib.dca_rope_rotate(fake, odd, 1, 8, 1, 64, 0, 4, 6, 1e4, 0, None)) == 1
+    assert _code(lib.dca_rope_rotate(fake, fake, 1, 8, 1, 80, 0, 4, 6, 1e4, 0, None)) == 2
+    assert _code(lib.dca_rope_rotate(fake, fake, 1, 8, 1, 64, 0, 4, 6, 1e4, 9, None)) == 2
+    assert _code(lib.dca_rope_rotate(fake, fake, 1, 8, 1, 64, 0, 7, 6, 1e4, 0, None)) == 2
+    assert _code(lib.dca_rope_rotate(fake, fake, 1, 8, 1, 64, -1, 4, 6, 1e4, 4, None)) == 1
+    assert "offset" in dca.dca_last_error_string()
+    # empty problems are no-ops even with null pointers
+    assert _code(lib.dca_rope_rotate(None, None, 0, 8, 1, 64, 0, 4, 6, 1e4, 0, None)) == 0
+    assert _code(lib.dca_attn_prefill(None, None, None, None, None, 1, 0, 4, 2, 128, 3072, 4096,
+                                      1e4, 0.0, None, 0, None)) == 0
+    # prefill: Hq % Hkv, s > c, short workspace, null workspace
+    args = (fake, fake, fake, fake, fake)
+    assert _code(lib.dca_attn_prefill(*args, 1, 64, 3, 2, 128, 16, 32, 1e4, 0.0, ws, 1 << 30,
+                                      None)) == 2
+    assert _code(lib.dca_attn_prefill(*args, 1, 64, 4, 2, 128, 64, 32, 1e4, 0.0, ws, 1 << 30,
+                                      None)) == 2
+    assert _code(lib.dca_attn_prefill(*args, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, ws, 100,
+                                      None)) == 5
+    assert "workspace" in dca.dca_last_error_string()
+    assert _code(lib.dca_attn_prefill(*args, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, None, 1 << 30,
+                                      None)) == 1
+    # tcgen05 path on a chunking it does not cover
+    assert _code(lib.dca_prefill_attention(fake, fake, fake, 1, 64, 4, 2, 128, 96, 128, 0.0,
+                                           2, ws, 1 << 30, None)) == 2
+    assert _code(lib.dca_prefill_attention(fake, fake, fake, 1, 64, 4, 2, 128, 96, 128, 0.0,
+                                           7, ws, 1 << 30, None)) == 1
+    # decode: null t, Tcap < 1, short workspace
+    dargs = (fake, fake, fake)
+    assert _code(lib.dca_attn_decode(*dargs, None, fake, fake, 2, 8, 1, 128, 64, 16, 32, 1e4,
+                                     0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_decode(*dargs, fake, fake, fake, 2, 8, 1, 128, 0, 16, 32, 1e4,
+                                     0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_decode(*dargs, fake, fake, fake, 2, 8, 1, 128, 64, 16, 32, 1e4,
+                                     0.0, ws, 8, None)) == 5
+    # index map: L too large, s > c
+    assert _code(lib.dca_debug_index_map(9000, 4, 6, fake, fake, fake, None)) == 1
+    assert _code(lib.dca_debug_index_map(16, 8, 6, fake, fake, fake, None)) == 2
+
+
+def test_binding_fails_loudly_without_cuda_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(dca.DcaError):
+        dca.dca_rope_rotate(x, dca.DCA_POS_KEY, 4, 6)
