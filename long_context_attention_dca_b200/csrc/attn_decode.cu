@@ -7,7 +7,8 @@
 // query heads, sequence):
 //   * prologue: rotate the group's queries at the three DCA positions of
 //     i = t[b] (intra i mod s, successive min(s + i mod s, c - 1), inter c - 1)
-//     in fp64-angle RoPE, kept in shared memory as bf16;
+//     in fp64-angle RoPE, kept in shared memory as a bf16 high part plus a
+//     bf16 remainder (two MMAs per score tile; the kernel is HBM-bound);
 //   * producer warp: TMA loads of 64-key K and V tiles (128-byte swizzle) into
 //     a 3-stage ring guarded by mbarriers (bounded waits);
 //   * 4 consumer warps, 16 keys each per tile: S[16 keys x 8 heads] by warp MMA
@@ -23,7 +24,7 @@
 #include "dca_kernels.cuh"
 
 namespace dca {
-namespace {
+namespace dec_path {
 
 constexpr int kDecKeys = 64;      // keys per pipeline stage
 constexpr int kDecStages = 3;
@@ -37,7 +38,7 @@ struct DecSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kStageBytes = 2 * kHalves * kBoxBytes;  // K halves then V halves
   static constexpr int kRing = kDecStages * kStageBytes;
-  static constexpr int kQ = 3 * kDecHeads * D * 2;
+  static constexpr int kQ = 2 * 3 * kDecHeads * D * 2;  // hi and lo parts
   static constexpr int kBars = 2 * kDecStages * 8 + 16;
   static constexpr int kTotal = 1024 /*align slack*/ + kRing + kQ + kBars;
 };
@@ -89,9 +90,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // Rotated queries: qs[piece][head][D], zero for padding heads.
+  // Rotated queries qs[part][piece][head][D] (zero for padding heads): the
+  // fp32 rotation split into a bf16 high part and a bf16 remainder, so the
+  // scores against the bf16 cache carry ~16 significant bits of q.
   {
     const int im = tb % s;
+    __nv_bfloat16* qs_lo = qs + 3 * kDecHeads * D;
     for (int idx = tid; idx < 3 * kDecHeads * (D / 2); idx += kDecThreads) {
       const int p = idx / (kDecHeads * (D / 2));
       const int hh = (idx / (D / 2)) % kDecHeads;
@@ -108,8 +112,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         o0 = fmaf(x0, cf, -x1 * sf);
         o1 = fmaf(x1, cf, x0 * sf);
       }
-      qs[(p * kDecHeads + hh) * D + k] = __float2bfloat16_rn(o0);
-      qs[(p * kDecHeads + hh) * D + k + D / 2] = __float2bfloat16_rn(o1);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(o0), h1 = __float2bfloat16_rn(o1);
+      const int at = (p * kDecHeads + hh) * D + k;
+      qs[at] = h0;
+      qs[at + D / 2] = h1;
+      qs_lo[at] = __float2bfloat16_rn(o0 - __bfloat162float(h0));
+      qs_lo[at + D / 2] = __float2bfloat16_rn(o1 - __bfloat162float(h1));
     }
   }
   __syncthreads();
@@ -148,7 +156,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     // ---------------- consumers ----------------
     const int ci = tb / s;
     int cur_piece = -1;
-    uint32_t qb[D / 16][2];
+    uint32_t qb[D / 16][2], qbl[D / 16][2];
     for (int it = 0; it < n_tiles; ++it) {
       const int st = it % kDecStages;
       if (!mbar_wait(full0 + 8 * st, (it / kDecStages) & 1, abort_flag, 102)) break;
@@ -165,10 +173,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
           if (p != cur_piece) {
             cur_piece = p;
             const uint32_t* qw = reinterpret_cast<const uint32_t*>(qs + (p * kDecHeads + g) * D);
+            const uint32_t* qwl = qw + 3 * kDecHeads * D / 2;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
               qb[ks][0] = qw[ks * 8 + t4];
               qb[ks][1] = qw[ks * 8 + 4 + t4];
+              qbl[ks][0] = qwl[ks * 8 + t4];
+              qbl[ks][1] = qwl[ks * 8 + 4 + t4];
             }
           }
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -178,6 +189,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
             ldsm_x4(a, kbase + dec_off(warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3),
                                        ks * 2 + (lane >> 4)));
             mma_bf16_16816(acc, a, qb[ks]);
+            mma_bf16_16816(acc, a, qbl[ks]);
           }
           // keep the entries whose key lies in piece p
 #pragma unroll
@@ -316,8 +328,10 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
   const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                                (uint64_t)Tcap * Hkv * D * 2};
   const uint32_t box[4] = {64, 1, kDecKeys, 1};
-  if (!encode_tensor_map_bf16(&tmK, Kc, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map_bf16(&tmV, Vc, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Kc, 4, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Vc, 4, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int nsplit = (Tcap + kDecSplit - 1) / kDecSplit;
   const int G = Hq / Hkv;
@@ -340,9 +354,11 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
   return cudaGetLastError();
 }
 
-}  // namespace
+}  // namespace dec_path
+
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap) {
+  using namespace dec_path;
   const size_t nsplit = ((size_t)Tcap + kDecSplit - 1) / kDecSplit;
   return (size_t)B * Hq * nsplit * (D + 2) * sizeof(float);
 }
@@ -350,6 +366,7 @@ size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap) {
 cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const int* t, void* O,
                           float* LSE, int B, int Hq, int Hkv, int D, int Tcap, int s, int c,
                           float base, float scale, void* workspace, cudaStream_t stream) {
+  using namespace dec_path;
   if (B == 0 || Hq == 0) return cudaSuccess;
   if (D == 64)
     return launch_decode_t<64>(q, Kc, Vc, t, O, LSE, B, Hq, Hkv, Tcap, s, c, base, scale,

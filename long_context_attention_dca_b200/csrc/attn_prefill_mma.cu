@@ -4,7 +4,8 @@
 // 128, D = 64) and doubles as an independent GPU cross-check of it.  Inputs
 // are the outputs of the fused RoPE kernel: Qrot [3][B][L][Hq][D] (the query
 // rotated for the intra, successive and inter pieces) and Krot [B][L][Hkv][D]
-// (keys at j mod s); V [B][L][Hkv][D] as given.
+// (keys at j mod s), both fp16; V [B][L][Hkv][D] bf16 as given.  S = Q K^T
+// runs on fp16 operands, O += P V on bf16 (P rounded to bf16), fp32 accumulate.
 //
 // Flash-style tiling (Dual-Chunk Attention: Training-Free 100k+ Context
 // Guide, "Flash-DCA: Fusing DCA into FlashAttention Tiling Loops"): a CTA owns
@@ -19,7 +20,7 @@
 #include "dca_kernels.cuh"
 
 namespace dca {
-namespace {
+namespace mma_path {
 
 constexpr int kBM = 64;
 constexpr int kBN = 64;
@@ -51,15 +52,15 @@ __device__ __forceinline__ void compute_s(float (&acc)[8][4], uint32_t q_base, u
                                   ks * 2 + ((lane >> 3) & 1)));
       const uint32_t b0[2] = {bk[0], bk[1]};
       const uint32_t b1[2] = {bk[2], bk[3]};
-      mma_bf16_16816(acc[2 * np], a, b0);
-      mma_bf16_16816(acc[2 * np + 1], a, b1);
+      mma_f16_16816(acc[2 * np], a, b0);
+      mma_f16_16816(acc[2 * np + 1], a, b1);
     }
   }
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
-    const __nv_bfloat16* __restrict__ Qrot, const __nv_bfloat16* __restrict__ Krot,
+    const __half* __restrict__ Qrot, const __half* __restrict__ Krot,
     const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ O, float* __restrict__ LSE,
     int B, int L, int Hq, int Hkv, int s, int c, float scale_log2) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
     const int v = idx / (kBM * CH), r = (idx / CH) % kBM, ch = idx % CH;
     const int row = q0 + r;
     const bool ok = row < L;
-    const __nv_bfloat16* src =
+    const __half* src =
         Qrot + v * plane + (((size_t)b * L + (ok ? row : 0)) * Hq + h) * D + ch * 8;
     cp_async_16(sQ + v * kBM * D * 2 + swz<D>(r, ch), src, ok);
   }
@@ -252,17 +253,19 @@ cudaError_t launch_mma(const void* Qrot, const void* Krot, const void* V, void* 
   dim3 grid((L + kBM - 1) / kBM, Hq, B);
   const float scale_log2 = scale * 1.4426950408889634f;
   kern<<<grid, kThreads, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(Qrot), static_cast<const __nv_bfloat16*>(Krot),
+      static_cast<const __half*>(Qrot), static_cast<const __half*>(Krot),
       static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(O), LSE, B, L, Hq, Hkv,
       s, c, scale_log2);
   return cudaGetLastError();
 }
 
-}  // namespace
+}  // namespace mma_path
+
 
 cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const void* V, void* O,
                                     float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
                                     int c, float scale, cudaStream_t stream) {
+  using namespace mma_path;
   if (L == 0 || B == 0 || Hq == 0) return cudaSuccess;
   if (D == 64) return launch_mma<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, stream);
   return launch_mma<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, stream);

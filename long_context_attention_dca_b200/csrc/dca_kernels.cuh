@@ -15,7 +15,7 @@ cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, in
                                int pos_offset, int s, int c, float base, int rule,
                                cudaStream_t stream);
 
-// Writes Krot [B][L][Hkv][D] and Qrot [3][B][L][Hq][D] (intra, succ, inter).
+// Writes Krot [B][L][Hkv][D] and Qrot [3][B][L][Hq][D] (intra, succ, inter), fp16.
 cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
                                 cudaStream_t stream);
@@ -40,8 +40,8 @@ cudaError_t launch_index_map(int L, int s, int c, int* qpos, int* kpos, signed c
                              cudaStream_t stream);
 
 // Driver entry point for building TMA tensor maps (resolved once).
-bool encode_tensor_map_bf16(CUtensorMap* map, const void* base, int rank,
-                            const uint64_t* dims, const uint64_t* strides_bytes,
-                            const uint32_t* box, CUtensorMapSwizzle swizzle);
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
 
 }  // namespace dca

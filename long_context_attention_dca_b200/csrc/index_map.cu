@@ -5,7 +5,7 @@
 #include "dca_kernels.cuh"
 
 namespace dca {
-namespace {
+namespace imap_path {
 
 __global__ void index_map_kernel(int L, int s, int c, int* __restrict__ qpos,
                                  int* __restrict__ kpos, signed char* __restrict__ piece) {
@@ -20,10 +20,12 @@ __global__ void index_map_kernel(int L, int s, int c, int* __restrict__ qpos,
   }
 }
 
-}  // namespace
+}  // namespace imap_path
+
 
 cudaError_t launch_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
                              cudaStream_t stream) {
+  using namespace imap_path;
   if (L == 0) return cudaSuccess;
   const long long n = (long long)L * L;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);

@@ -7,7 +7,8 @@
 //
 // Angles are evaluated in fp64 (positions are integers below c for the DCA
 // rules), cos/sin rounded to fp32, the rotation done in fp32 and the result
-// rounded to bf16 (round to nearest even).
+// rounded to nearest even: bf16 for dca_rope_rotate (a cache in the caller's
+// type), fp16 for the prefill workspace (operands of S = Q K^T only).
 //
 // Both kernels are HBM-bound: each thread owns one token row and one group of
 // 8 rotation pairs (16 bytes of the first half and the matching 16 bytes of
@@ -19,7 +20,7 @@
 
 namespace dca {
 
-namespace {
+namespace rope_path {
 
 struct CosSin8 {
   float c[8], s[8];
@@ -37,7 +38,14 @@ __device__ __forceinline__ void cos_sin_group(int pos, int k0, int D, double log
   }
 }
 
-// out_lo = lo*cos - hi*sin, out_hi = hi*cos + lo*sin for 8 pairs.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// out_lo = lo*cos - hi*sin, out_hi = hi*cos + lo*sin for 8 pairs; the result
+// is rounded to bf16 (kHalf = false) or fp16 (kHalf = true).
+template <bool kHalf = false>
 __device__ __forceinline__ void rotate8(const uint4& lo, const uint4& hi, const CosSin8& cs,
                                        uint4& olo, uint4& ohi) {
   const uint32_t* a = reinterpret_cast<const uint32_t*>(&lo);
@@ -50,8 +58,15 @@ __device__ __forceinline__ void rotate8(const uint4& lo, const uint4& hi, const 
     const float b0 = bf16_lo(b[w]), b1 = bf16_hi(b[w]);
     const float c0 = cs.c[2 * w], c1 = cs.c[2 * w + 1];
     const float s0 = cs.s[2 * w], s1 = cs.s[2 * w + 1];
-    oa[w] = pack_bf16(fmaf(a0, c0, -b0 * s0), fmaf(a1, c1, -b1 * s1));
-    ob[w] = pack_bf16(fmaf(b0, c0, a0 * s0), fmaf(b1, c1, a1 * s1));
+    const float r0 = fmaf(a0, c0, -b0 * s0), r1 = fmaf(a1, c1, -b1 * s1);
+    const float u0 = fmaf(b0, c0, a0 * s0), u1 = fmaf(b1, c1, a1 * s1);
+    if constexpr (kHalf) {
+      oa[w] = pack_f16(r0, r1);
+      ob[w] = pack_f16(u0, u1);
+    } else {
+      oa[w] = pack_bf16(r0, r1);
+      ob[w] = pack_bf16(u0, u1);
+    }
   }
 }
 
@@ -89,10 +104,12 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(
 }
 
 // K rotated once at j mod s; Q written three ways (intra, successive, inter).
-// Qrot layout: [3][B][L][Hq][D]; Krot: [B][L][Hkv][D].
+// Qrot layout: [3][B][L][Hq][D]; Krot: [B][L][Hkv][D].  Both are fp16: the
+// rotated operands of S = Q K^T keep 11 significant bits instead of bf16's 8,
+// which keeps the score error from rounding them near 4e-4 instead of 3e-3.
 __global__ void __launch_bounds__(256) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-    __nv_bfloat16* __restrict__ Qrot, __nv_bfloat16* __restrict__ Krot, int B, int L, int Hq,
+    __half* __restrict__ Qrot, __half* __restrict__ Krot, int B, int L, int Hq,
     int Hkv, int D, int s, int c, double log2_base) {
   const int groups = D / 16;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -115,7 +132,7 @@ __global__ void __launch_bounds__(256) prefill_rope_kernel(
       const uint4 lo = *reinterpret_cast<const uint4*>(K + off);
       const uint4 hi = *reinterpret_cast<const uint4*>(K + off + D / 2);
       uint4 olo, ohi;
-      rotate8(lo, hi, cs, olo, ohi);
+      rotate8<true>(lo, hi, cs, olo, ohi);
       *reinterpret_cast<uint4*>(Krot + off) = olo;
       *reinterpret_cast<uint4*>(Krot + off + D / 2) = ohi;
     }
@@ -130,24 +147,26 @@ __global__ void __launch_bounds__(256) prefill_rope_kernel(
     const uint4 lo = *reinterpret_cast<const uint4*>(Q + off);
     const uint4 hi = *reinterpret_cast<const uint4*>(Q + off + D / 2);
     uint4 olo, ohi;
-    rotate8(lo, hi, cs, olo, ohi);
+    rotate8<true>(lo, hi, cs, olo, ohi);
     *reinterpret_cast<uint4*>(Qrot + off) = olo;
     *reinterpret_cast<uint4*>(Qrot + off + D / 2) = ohi;
     uint4 ilo, ihi;
-    rotate8(lo, hi, cs_inter, ilo, ihi);
+    rotate8<true>(lo, hi, cs_inter, ilo, ihi);
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = ilo;
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + D / 2) = ihi;
-    if (!succ_is_inter) rotate8(lo, hi, cs_succ, ilo, ihi);
+    if (!succ_is_inter) rotate8<true>(lo, hi, cs_succ, ilo, ihi);
     *reinterpret_cast<uint4*>(Qrot + plane + off) = ilo;
     *reinterpret_cast<uint4*>(Qrot + plane + off + D / 2) = ihi;
   }
 }
 
-}  // namespace
+}  // namespace rope_path
+
 
 cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, int D,
                                int pos_offset, int s, int c, float base, int rule,
                                cudaStream_t stream) {
+  using namespace rope_path;
   const long long total = (long long)B * L * (D / 16);
   if (total == 0) return cudaSuccess;
   const int threads = 256;
@@ -161,13 +180,14 @@ cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, in
 cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
                                 cudaStream_t stream) {
+  using namespace rope_path;
   const long long total = (long long)B * L * (D / 16);
   if (total == 0) return cudaSuccess;
   const int threads = 256;
   const unsigned blocks = (unsigned)((total + threads - 1) / threads);
   prefill_rope_kernel<<<blocks, threads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-      static_cast<__nv_bfloat16*>(Qrot), static_cast<__nv_bfloat16*>(Krot), B, L, Hq, Hkv, D, s,
+      static_cast<__half*>(Qrot), static_cast<__half*>(Krot), B, L, Hq, Hkv, D, s,
       c, log2((double)base));
   return cudaGetLastError();
 }
