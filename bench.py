@@ -121,15 +121,15 @@ class _F64:
 _CPU_INPUTS = {}
 
 
-def oracle_sample(budget_s: float, seed: int = 0):
-    """Time the oracle on random (row, head) outputs of the prefill workload
+def oracle_sample(budget_s: float, seed: int = 0, name: str = PREFILL):
+    """Time the oracle on random (row, head) outputs of a prefill workload
     until `budget_s` seconds have passed; returns (TFLOP/s, rows, heads, s)."""
     import numpy as np
     from oracle import dca_oracle as orc
-    cfg = W.CONFIGS[PREFILL]
-    if PREFILL not in _CPU_INPUTS:
-        _CPU_INPUTS[PREFILL] = W.make_prefill_inputs(cfg)
-    Q, K, V = _CPU_INPUTS[PREFILL]
+    cfg = W.CONFIGS[name]
+    if name not in _CPU_INPUTS:
+        _CPU_INPUTS[name] = W.make_prefill_inputs(cfg)
+    Q, K, V = _CPU_INPUTS[name]
     rng = np.random.default_rng(seed)
     flops = 0.0
     n_rows = 0
@@ -202,7 +202,7 @@ def run_ours(args, rank, world, dev):
     import ctypes
     P = ctypes.c_void_p
 
-    pc = W.CONFIGS[PREFILL]
+    pc = W.CONFIGS[args.workload]
     dc = W.CONFIGS[DECODE]
     Q, K, V = W.make_prefill_inputs(pc, device=dev)
     B, L, Hq, D = Q.shape
@@ -292,15 +292,16 @@ def run_ours(args, rank, world, dev):
     hbm = peaks["hbm_gbs"]
 
     # ---- e2e through the public API with host buffers ----
-    e2e = run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc)
+    e2e = None if args.no_e2e else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
+                                           t_dec, Kc, Vc)
 
     line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            tf, n_rows, n_heads, dt = oracle_sample(args.cpu_seconds)
+            tf, n_rows, n_heads, dt = oracle_sample(args.cpu_seconds, name=args.workload)
             cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                   "sample": f"{n_rows} random query rows x {n_heads} head of the {PREFILL} "
+                   "sample": f"{n_rows} random query rows x {n_heads} head of the {args.workload} "
                              f"prefill workload, fp64 oracle, {dt:.1f} s"}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -308,12 +309,13 @@ def run_ours(args, rank, world, dev):
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16, Llama-2 attention shapes)",
-            "config": {"workload": PREFILL, **_cfg_summary(pc),
+            "config": {"workload": args.workload, **_cfg_summary(pc),
                        "decode_workload": DECODE, "decode": _cfg_summary(dc),
                        "prefill_path": {1: "general (warp MMA)",
                                         2: "tcgen05/TMEM/TMA"}.get(path, str(path)),
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (Q,K,V 402 MB; decode KV 3.2 GB)"},
+                       "l2": "inputs larger than L2 (prefill Q,K,V >= 402 MB; decode KV "
+                             "3.2 GB); no flush"},
             "prefill": {"tflops_rope_plus_attn": value / world, "attn_tflops": attn_tflops,
                         "attn_ms": attn_sum / args.steps, "rope_ms": rope_sum / args.steps,
                         "rope_gbs": rope_gbs, "frac_of_peak": attn_tflops / tpk},
@@ -411,6 +413,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--workload", default=PREFILL, choices=sorted(
+        k for k, v in W.CONFIGS.items() if v["kind"] == "prefill" and v["D"] == 128),
+                    help="prefill workload of the step (default: the 7B-shaped one)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
