@@ -143,6 +143,27 @@ dca_status_t dca_attn_decode(const void* q, const void* Kcache, const void* Vcac
                              int Tcap, int s, int c, float base, float scale, void* workspace,
                              size_t ws_bytes, void* stream);
 
+/* dca_attn_decode for callers that cannot allocate device memory (e.g. a
+ * plugin inside a serving framework whose allocator owns the GPU's memory, or
+ * a decode loop that must avoid cudaMalloc's implicit synchronisation).  Same
+ * arguments and results as dca_attn_decode minus the workspace: the split-KV
+ * scratch lives in a fixed 48 MiB array in the library's device memory, held
+ * by every GPU that loads the library until the process exits.  The paper has
+ * no counterpart; this is a deployment variant of the decode call.
+ *   - The first call on each device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current); make it before any
+ *     stream capture.
+ *   - All calls share the array: calls whose kernels overlap on the GPU race.
+ *     Nothing in it needs to start at zero.
+ *   - Sizes whose scratch (dca_attn_decode_workspace) exceeds 48 MiB return
+ *     DCA_ERR_WORKSPACE; the 16-sequence, 64-head, Tcap 65536 decode workload
+ *     needs 32.5 MiB.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_decode_noalloc(const void* q, const void* Kcache, const void* Vcache,
+                                     const int* t, void* O, float* LSE, int B, int Hq, int Hkv,
+                                     int D, int Tcap, int s, int c, float base, float scale,
+                                     void* stream);
+
 /* Dense L x L tables of the index rule for small L (L <= 8192): qpos and
  * kpos (int32, -1 where masked) and piece (int8: 0 intra, 1 successive,
  * 2 inter, -1 masked, i.e. j > i), row-major [i][j].

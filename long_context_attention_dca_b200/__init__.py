@@ -23,7 +23,8 @@ __all__ = [
     "DCA_PATH_AUTO", "DCA_PATH_GENERAL", "DCA_PATH_TCGEN05",
     "dca_rope_rotate", "dca_attn_prefill_workspace", "dca_prefill_rope",
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
-    "dca_attn_decode_workspace", "dca_attn_decode", "dca_debug_index_map",
+    "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc",
+    "dca_debug_index_map",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
 ]
 
@@ -47,6 +48,8 @@ _SIGS = {
     "dca_attn_decode_workspace": (_Z, [_I, _I, _I, _I]),
     "dca_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
                              _Z, _P]),
+    "dca_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
+                                     _F, _P]),
     "dca_debug_index_map": (_I, [_I, _I, _I, _P, _P, _P, _P]),
     "dca_sync_status": (_I, [_P]),
     "dca_last_error_string": (ctypes.c_char_p, []),
@@ -202,6 +205,25 @@ def dca_attn_decode(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, workspa
     _check(lib().dca_attn_decode(_ptr(q), _ptr(Kcache), _ptr(Vcache), _ptr(t), _ptr(O),
                                  _ptr(LSE), B, Hq, Hkv, D, Tcap, s, c, base, scale, _ptr(ws),
                                  ws.numel(), _stream(q)))
+    return O, LSE
+
+
+def dca_attn_decode_noalloc(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, O=None,
+                            LSE=None):
+    """dca_attn_decode without a workspace: for callers that cannot allocate
+    device memory, the library uses its fixed 48 MiB scratch array (shared by
+    all calls; see include/dca.h).  Outputs may be passed in preallocated."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    _need(t, "t", torch.int32, 1)
+    B, Hq, D = q.shape
+    Tcap, Hkv = Kcache.shape[1], Kcache.shape[2]
+    O = torch.empty_like(q) if O is None else O
+    LSE = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if LSE is None else LSE
+    _check(lib().dca_attn_decode_noalloc(_ptr(q), _ptr(Kcache), _ptr(Vcache), _ptr(t), _ptr(O),
+                                         _ptr(LSE), B, Hq, Hkv, D, Tcap, s, c, base, scale,
+                                         _stream(q)))
     return O, LSE
 
 

@@ -7,3 +7,4 @@
 #include "attn_prefill_mma.cu"
 #include "attn_prefill_sm100.cu"
 #include "attn_decode.cu"
+#include "decode_noalloc.cu"
