@@ -214,6 +214,10 @@ def run_ours(args, rank, world, dev):
     LSE = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
     path = dca.dca_prefill_path(L, D, s, c)
 
+    do_pre = args.only in ("all", "prefill")
+    do_dec = args.only in ("all", "decode")
+    if not do_dec:  # profiling run: a 1-sequence, 1k-token stand-in keeps memory small
+        dc = W.scaled(dc, B=1, Tcap=1024, t_lo=1000, t_hi=1001)
     t_dec, q_dec, Kc, Vc = W.make_decode_inputs(dc, device=dev)
     Bd, Hqd, Dd = q_dec.shape
     Tcap, Hkvd = Kc.shape[1], Kc.shape[2]
@@ -243,7 +247,10 @@ def run_ours(args, rank, world, dev):
                                 P(dws.data_ptr()), dws_bytes, P(sptr)))
 
     for _ in range(args.warmup):
-        rope(); attn(); decode()
+        if do_pre:
+            rope(); attn()
+        if do_dec:
+            decode()
     torch.cuda.synchronize(dev)
     dca.dca_sync_status(dev)
 
@@ -258,9 +265,15 @@ def run_ours(args, rank, world, dev):
     t_start.record(stream)
     for k in range(args.steps):
         e = ev[k]
-        e[0].record(stream); rope()
-        e[1].record(stream); attn()
-        e[2].record(stream); decode()
+        e[0].record(stream)
+        if do_pre:
+            rope()
+        e[1].record(stream)
+        if do_pre:
+            attn()
+        e[2].record(stream)
+        if do_dec:
+            decode()
         e[3].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -281,10 +294,11 @@ def run_ours(args, rank, world, dev):
     flops = W.prefill_flops(pc)
     dec_bytes = W.decode_bytes(dc, t_host.tolist())
     rope_bytes = float(B * L * (Hq + Hkv) * D * 2 + B * L * (3 * Hq + Hkv) * D * 2)
-    value = world * flops * args.steps / (prefill_ms * 1e-3) / 1e12
-    attn_tflops = flops * args.steps / (attn_sum * 1e-3) / 1e12
-    dec_gbs = world * dec_bytes * args.steps / (dec_sum * 1e-3) / 1e9
-    rope_gbs = rope_bytes * args.steps / (rope_sum * 1e-3) / 1e9
+    rate = lambda work, ms: work * args.steps / (ms * 1e-3) if ms > 1e-6 else 0.0
+    value = world * rate(flops, prefill_ms) / 1e12
+    attn_tflops = rate(flops, attn_sum) / 1e12
+    dec_gbs = world * rate(dec_bytes, dec_sum) / 1e9
+    rope_gbs = rate(rope_bytes, rope_sum) / 1e9
 
     peaks, peak_kind = load_peaks()
     traffic = load_traffic()
@@ -292,7 +306,7 @@ def run_ours(args, rank, world, dev):
     hbm = peaks["hbm_gbs"]
 
     # ---- e2e through the public API with host buffers ----
-    e2e = None if args.no_e2e else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
+    e2e = None if (args.no_e2e or args.only != "all") else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
                                            t_dec, Kc, Vc)
 
     line = None
@@ -334,7 +348,7 @@ def run_ours(args, rank, world, dev):
                                  "unit": "GB/s", "frac": rope_gbs / hbm,
                                  "traffic": traffic.get("prefill_rope")}},
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (2 * do_pre + 2 * do_dec) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -413,6 +427,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="profiling runs: time only one half of the step")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default=PREFILL, choices=sorted(

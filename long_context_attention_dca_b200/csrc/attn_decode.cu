@@ -90,13 +90,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     *abort_flag = 0;
     fence_barrier_init();
   }
+  __syncthreads();
   // Rotated queries qs[part][piece][head][D] (zero for padding heads): the
   // fp32 rotation split into a bf16 high part and a bf16 remainder, so the
-  // scores against the bf16 cache carry ~16 significant bits of q.
-  {
+  // scores against the bf16 cache carry ~16 significant bits of q.  The four
+  // consumer warps build them while the producer warp already streams K/V.
+  if (warp < 4) {
     const int im = tb % s;
     __nv_bfloat16* qs_lo = qs + 3 * kDecHeads * D;
-    for (int idx = tid; idx < 3 * kDecHeads * (D / 2); idx += kDecThreads) {
+    for (int idx = tid; idx < 3 * kDecHeads * (D / 2); idx += 128) {
       const int p = idx / (kDecHeads * (D / 2));
       const int hh = (idx / (D / 2)) % kDecHeads;
       const int k = idx % (D / 2);
@@ -105,10 +107,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         const __nv_bfloat16* qrow = q + ((size_t)b * Hq + h_base + hh) * D;
         const float x0 = __bfloat162float(qrow[k]), x1 = __bfloat162float(qrow[k + D / 2]);
         const int pos = query_pos_for_piece(p, im, s, c);
+        // angle formed and reduced to [-pi, pi] in fp64, evaluated in fp32
+        constexpr double kTwoPi = 6.283185307179586476925286766559;
         const double theta = exp2(-(2.0 * (double)k / (double)D) * log2_base);
-        double sn, cn;
-        sincos((double)pos * theta, &sn, &cn);
-        const float cf = (float)cn, sf = (float)sn;
+        const double a = (double)pos * theta;
+        float sf, cf;
+        sincosf((float)fma(-rint(a * (1.0 / kTwoPi)), kTwoPi, a), &sf, &cf);
         o0 = fmaf(x0, cf, -x1 * sf);
         o1 = fmaf(x1, cf, x0 * sf);
       }
@@ -119,8 +123,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       qs_lo[at] = __float2bfloat16_rn(o0 - __bfloat162float(h0));
       qs_lo[at + D / 2] = __float2bfloat16_rn(o1 - __bfloat162float(h1));
     }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // consumer warps only
   }
-  __syncthreads();
 
   const int g = lane >> 2, t4 = lane & 3;
   float m_run[2] = {-INFINITY, -INFINITY};  // heads 2*t4, 2*t4 + 1
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const float* __restrict
                                                          __nv_bfloat16* __restrict__ O,
                                                          float* __restrict__ LSE, int Hq,
                                                          int Tcap, int nsplit_max) {
+  __shared__ float stat_s[2];
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int tb = t[b];
   if (tb < 0 || tb >= Tcap) {
@@ -307,15 +312,34 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const float* __restrict
   }
   const int n = (tb + 1 + kDecSplit - 1) / kDecSplit;
   const size_t base = ((size_t)b * Hq + h) * nsplit_max;
-  float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, MLpart[(base + p) * 2]);
-  float acc = 0.f, lsum = 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float f = fast_exp2(MLpart[(base + p) * 2] - M);
-    acc += f * Opart[(base + p) * D + d];
-    lsum += f * MLpart[(base + p) * 2 + 1];
+  // warp 0: max of the split maxima and the total weighted sum, reading the
+  // splits' (max, sum) pairs in parallel
+  if (d < 32) {
+    float M = -INFINITY;
+    for (int p = d; p < n; p += 32) M = fmaxf(M, MLpart[(base + p) * 2]);
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+    float lsum = 0.f;
+    for (int p = d; p < n; p += 32)
+      lsum += fast_exp2(MLpart[(base + p) * 2] - M) * MLpart[(base + p) * 2 + 1];
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, sh);
+    if (d == 0) {
+      stat_s[0] = M;
+      stat_s[1] = lsum;
+    }
   }
-  O[((size_t)b * Hq + h) * D + d] = __float2bfloat16_rn(acc / lsum);
+  __syncthreads();
+  const float M = stat_s[0];
+  float acc0 = 0.f, acc1 = 0.f;
+  int p = 0;
+  for (; p + 1 < n; p += 2) {
+    acc0 += fast_exp2(MLpart[(base + p) * 2] - M) * Opart[(base + p) * D + d];
+    acc1 += fast_exp2(MLpart[(base + p + 1) * 2] - M) * Opart[(base + p + 1) * D + d];
+  }
+  if (p < n) acc0 += fast_exp2(MLpart[(base + p) * 2] - M) * Opart[(base + p) * D + d];
+  const float lsum = stat_s[1];
+  O[((size_t)b * Hq + h) * D + d] = __float2bfloat16_rn((acc0 + acc1) / lsum);
   if (d == 0) LSE[(size_t)b * Hq + h] = (M + log2f(lsum)) * 0.69314718055994530942f;
 }
 

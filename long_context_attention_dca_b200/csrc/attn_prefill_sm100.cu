@@ -31,6 +31,7 @@
 #include "dca_common.cuh"
 #include "dca_index.cuh"
 #include "dca_kernels.cuh"
+#include "softmax_sm100.cuh"
 
 namespace dca {
 namespace tc_path {
@@ -253,16 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_sm100_kernel(
       for (int q = 0; q < 4; ++q) tmem_ld32(s_addr + 32u * q, v[q]);
       tmem_wait_ld();
       const bool diag = (j == n_kt - 1);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(v[q][e]);
-          if (diag && (q * 32 + e) > row) x = -INFINITY;
-          v[q][e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+      float mx;
+      if (diag) mx = row_max_causal(v, row);  // causal mask on the diagonal tile only
+      else mx = row_max(v);
       const float m_tile = mx * scale_log2;
       if (j == 0) {
         m_run = m_tile;
@@ -289,19 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_sm100_kernel(
         m_run = m_new;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      float lsum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(v[q][2 * e]), scale_log2, -m_use));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(v[q][2 * e + 1]), scale_log2, -m_use));
-          lsum += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
-        }
-        tmem_st16(s_addr + 16u * q, pk);
-      }
+      const float lsum = row_exp_store(v, scale_log2, m_use, s_addr);
       tmem_wait_st();
       l_run += lsum;
       tc_fence_before();

@@ -1,0 +1,388 @@
+// DCA prefill attention, tcgen05 ping-pong variant: two 128-row query tiles
+// (A = rows q0 .. q0+127, B = rows q0+128 .. q0+255) share every K and V tile.
+// Shape contract: D = 128 and s % 256 == 0, so both tiles lie in one chunk and
+// meet the DCA pieces at the same key tiles (Dual-Chunk Attention:
+// Training-Free 100k+ Context Guide, "Flash-DCA": chunk a multiple of the
+// tile, piece known per tile from its indices).
+//
+// While softmax warpgroup A turns S_A into P_A, the tensor core computes S_B
+// and accumulates O_B; then the roles swap.  The single-thread issuer runs,
+// per key tile i:
+//     S_A(i) = Q_A K_i^T,  O_B += P_B(i-1) V_{i-1},  S_B(i) = Q_B K_i^T,
+//     O_A += P_A(i) V_i
+// P_X(i) is written by the softmax into the columns of S_X (bf16, 64 columns)
+// and read by the TMEM-A form of the MMA; the next S_X overwrites those
+// columns only after the PV that reads them, relying on tcgen05.mma
+// executing in issue order.
+//
+// Warps (384 threads, 3 warpgroups): 0-3 softmax A, 4-7 softmax B (row =
+// TMEM lane), 8 TMA producer, 9 TMEM allocator + UMMA issuer, 10-11 idle.
+// Registers are rebalanced after set-up: the producer/issuer warpgroup drops
+// to 72 per thread, the softmax warpgroups rise to 216 (2*128*216 + 128*72 =
+// 384 * 168, the launch allotment).
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// Shared memory: 3 rotating Q slots (the query rotation of each piece, loaded
+// in order of first use: A then B for each piece), K ring of 2, V ring of 2.
+// The online softmax keeps running max / sum in fp32 (log2 domain); O is
+// rescaled in TMEM only when a warp's max grew by more than 2^8.
+// Every mbarrier wait is bounded; on expiry the CTA records an error, drains
+// its copies and MMAs and frees TMEM.
+#include "dca_common.cuh"
+#include "dca_index.cuh"
+#include "dca_kernels.cuh"
+#include "softmax_sm100.cuh"
+
+namespace dca {
+namespace pp_path {
+
+constexpr int kTile = 128;
+constexpr int kHD = 128;
+constexpr int kBox = kTile * 64 * 2;   // [128 rows x 64 cols] 16-bit = 16 KB
+constexpr int kTileBytes = 2 * kBox;   // 32 KB
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allotment");
+constexpr int kNumQSlots = 3;
+constexpr int kSmQ = 0;
+constexpr int kSmK = kNumQSlots * kTileBytes;
+constexpr int kSmV = kSmK + 2 * kTileBytes;
+constexpr int kSmBar = kSmV + 2 * kTileBytes;
+enum Bar {
+  kQFull = 0, kQEmpty = 3, kKFull = 6, kKEmpty = 8, kVFull = 10, kVEmpty = 12,
+  kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kNumBars = 21
+};
+constexpr int kSmMisc = kSmBar + kNumBars * 8;
+constexpr int kSmTotal = kSmMisc + 16 + 1024;
+static_assert(kSmTotal <= 232448, "shared memory budget");
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct Phases {
+  int n;
+  int piece[3];
+  int begin[3];
+};
+
+__device__ __forceinline__ Phases make_phases(int ci, int tiles_per_chunk) {
+  Phases p;
+  p.n = 0;
+  if (ci >= 2) { p.piece[p.n] = kInter; p.begin[p.n] = 0; ++p.n; }
+  if (ci >= 1) { p.piece[p.n] = kSucc; p.begin[p.n] = (ci - 1) * tiles_per_chunk; ++p.n; }
+  p.piece[p.n] = kIntra; p.begin[p.n] = ci * tiles_per_chunk; ++p.n;
+  return p;
+}
+
+__device__ __forceinline__ int phase_of(const Phases& p, int j) {
+  int ph = 0;
+#pragma unroll
+  for (int k = 1; k < 3; ++k)
+    if (k < p.n && j >= p.begin[k]) ph = k;
+  return ph;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
+    float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kSmBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmMisc + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int num_qt = (L + kTile - 1) / kTile;
+  const int num_pairs = (num_qt + 1) / 2;
+  const int m = num_pairs - 1 - (int)blockIdx.x;  // longest pairs first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (Hq / Hkv);
+  const int q0 = m * 2 * kTile;
+  const int tpc = s / kTile;
+  const Phases ph = make_phases(q0 / s, tpc);
+  const int nA = 2 * m + 1;  // key tiles 0 .. 2m   (diagonal of A)
+  const int nB = 2 * m + 2;  // key tiles 0 .. 2m+1 (diagonal of B)
+
+  if (tid == 0) {
+    for (int i = 0; i < kNumQSlots; ++i) {
+      mbar_init(bar(kQFull + i), 1);
+      mbar_init(bar(kQEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kKFull + i), 1);
+      mbar_init(bar(kKEmpty + i), 1);
+      mbar_init(bar(kVFull + i), 1);
+      mbar_init(bar(kVEmpty + i), 1);
+      mbar_init(bar(kSFull + i), 1);
+      mbar_init(bar(kPFull + i), 4);
+      mbar_init(bar(kODone + i), 1);
+    }
+    mbar_init(bar(kMmaEnd), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp >= 8) {
+  reg_dealloc<kControlRegs>();
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      // Q load n (n = 2 * phase + tile) goes to slot n % 3.
+      int q_last[kNumQSlots] = {-1, -1, -1};
+      bool ok = true;
+      auto load_q = [&](int n) -> bool {
+        const int slot = n % kNumQSlots;
+        if (n >= kNumQSlots &&
+            !mbar_wait(bar(kQEmpty + slot), ((n / kNumQSlots) - 1) & 1, abort_flag, 401))
+          return false;
+        const int p = n >> 1, x = n & 1;
+        const uint32_t fb = bar(kQFull + slot);
+        mbar_arrive_expect_tx(fb, kTileBytes);
+        const uint32_t dst = sbase + kSmQ + slot * kTileBytes;
+        const int row = q0 + x * kTile;
+        tma_load_4d(dst, &tmQ, fb, 0, h, row, ph.piece[p] * B + b);
+        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, ph.piece[p] * B + b);
+        q_last[slot] = n;
+        return true;
+      };
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+      ok = load_q(0) && load_q(1);
+      for (int i = 0; i < nB && ok; ++i) {
+        const int p = phase_of(ph, i);
+        const bool boundary = (p > 0 && i == ph.begin[p]);
+        if (boundary && !(ok = load_q(2 * p))) break;
+        const int st = i & 1;
+        if (i >= 2 && !(ok = mbar_wait(bar(kKEmpty + st), ((i >> 1) + 1) & 1, abort_flag, 402)))
+          break;
+        mbar_arrive_expect_tx(bar(kKFull + st), kTileBytes);
+        const uint32_t kd = sbase + kSmK + st * kTileBytes;
+        tma_load_4d(kd, &tmK, bar(kKFull + st), 0, hk, i * kTile, b);
+        tma_load_4d(kd + kBox, &tmK, bar(kKFull + st), 64, hk, i * kTile, b);
+        k_last[st] = i;
+        if (boundary && !(ok = load_q(2 * p + 1))) break;
+        if (i >= 2 && !(ok = mbar_wait(bar(kVEmpty + st), ((i >> 1) + 1) & 1, abort_flag, 403)))
+          break;
+        mbar_arrive_expect_tx(bar(kVFull + st), kTileBytes);
+        const uint32_t vd = sbase + kSmV + st * kTileBytes;
+        tma_load_4d(vd, &tmV, bar(kVFull + st), 0, hk, i * kTile, b);
+        tma_load_4d(vd + kBox, &tmV, bar(kVFull + st), 64, hk, i * kTile, b);
+        v_last[st] = i;
+      }
+      // drain: every issued copy has landed before shared memory is released
+      for (int k = 0; k < kNumQSlots; ++k)
+        if (q_last[k] >= 0)
+          mbar_wait(bar(kQFull + k), (q_last[k] / kNumQSlots) & 1, nullptr, 404);
+      for (int st = 0; st < 2; ++st) {
+        if (k_last[st] >= 0) mbar_wait(bar(kKFull + st), (k_last[st] >> 1) & 1, nullptr, 405);
+        if (v_last[st] >= 0) mbar_wait(bar(kVFull + st), (v_last[st] >> 1) & 1, nullptr, 406);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc(128, 128, /*bf16=*/false, 0, 0);  // fp16 Q, K
+      const uint32_t idesc_o = umma_idesc(128, 128, /*bf16=*/true, 0, 1);   // bf16 P, V
+      auto issue_s = [&](int x, int i) -> bool {
+        const int p = phase_of(ph, i);
+        const int n = 2 * p + x;
+        const int slot = n % kNumQSlots;
+        if (i == ph.begin[p] &&
+            !mbar_wait(bar(kQFull + slot), (n / kNumQSlots) & 1, abort_flag, 411))
+          return false;
+        const bool first_user = (x == 0) || (i >= nA);
+        if (first_user && !mbar_wait(bar(kKFull + (i & 1)), (i >> 1) & 1, abort_flag, 412))
+          return false;
+        tc_fence_after();
+        const uint32_t qa = sbase + kSmQ + slot * kTileBytes;
+        const uint32_t ka = sbase + kSmK + (i & 1) * kTileBytes;
+        const uint32_t d = tmem + 128u * (uint32_t)x;
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * kBox + (kk & 3) * 32);
+          umma_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(kSFull + x));
+        if (x == 1) umma_commit(bar(kKEmpty + (i & 1)));  // B is the last reader of K_i
+        const bool last_of_phase = (p + 1 < ph.n) ? (i == ph.begin[p + 1] - 1)
+                                                  : (i == (x ? nB : nA) - 1);
+        if (last_of_phase) umma_commit(bar(kQEmpty + slot));
+        return true;
+      };
+      auto issue_pv = [&](int x, int i) -> bool {
+        if (!mbar_wait(bar(kPFull + x), i & 1, abort_flag, 413)) return false;
+        const bool first_user = (x == 0) || (i >= nA);
+        if (first_user && !mbar_wait(bar(kVFull + (i & 1)), (i >> 1) & 1, abort_flag, 414))
+          return false;
+        tc_fence_after();
+        const uint32_t va = sbase + kSmV + (i & 1) * kTileBytes;
+        const uint32_t pa = tmem + 128u * (uint32_t)x;
+        const uint32_t od = tmem + 256u + 128u * (uint32_t)x;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(od, pa + 8u * (uint32_t)kk,
+                  smem_desc_sw128(va + (uint32_t)kk * 2048u, kBox, 1024), idesc_o,
+                  (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(kODone + x));
+        if (x == 1) umma_commit(bar(kVEmpty + (i & 1)));  // B is the last reader of V_i
+        return true;
+      };
+      bool ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0);
+      for (int i = 1; i < nB && ok; ++i) {
+        if (i < nA && !(ok = issue_s(0, i))) break;
+        if (!(ok = issue_pv(1, i - 1))) break;
+        if (!(ok = issue_s(1, i))) break;
+        if (i < nA && !(ok = issue_pv(0, i))) break;
+      }
+      if (ok) issue_pv(1, nB - 1);
+      umma_commit(bar(kMmaEnd));
+      mbar_wait(bar(kMmaEnd), 0, nullptr, 415);
+    }
+    __syncwarp();
+  }
+  } else {
+    reg_alloc<kSoftmaxRegs>();
+    // ------------------------------------------------------------ softmax A / B
+    const int x = warp >> 2;               // 0 = tile A, 1 = tile B
+    const int wq = warp & 3;               // TMEM lane quarter
+    const int row = wq * 32 + lane;        // row within the tile
+    const int i_row = q0 + x * kTile + row;
+    const int n_x = x ? nB : nA;
+    const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t s_addr = t_lane + 128u * (uint32_t)x;
+    const uint32_t o_addr = t_lane + 256u + 128u * (uint32_t)x;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_x; ++i) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + x), i & 1, abort_flag, 421));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(s_addr + 32u * q, v[q]);
+      tmem_wait_ld();
+      const bool diag = (i == n_x - 1);
+      float mx;
+      if (diag) mx = row_max_causal(v, row);  // causal mask on the diagonal tile only
+      else mx = row_max(v);
+      const float m_tile = mx * scale_log2;
+      if (i == 0) {
+        m_run = m_tile;
+      } else if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kODone + x), (i - 1) & 1, abort_flag, 422));
+        if (!ok) break;
+        tc_fence_after();
+        const float m_new = fmaxf(m_run, m_tile);
+        const float alpha = fast_exp2(m_run - m_new);
+        l_run *= alpha;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + 32u * q, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(o_addr + 32u * q, o);
+        }
+        tmem_wait_st();
+        m_run = m_new;
+      }
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const float lsum = row_exp_store(v, scale_log2, m_use, s_addr);
+      tmem_wait_st();
+      l_run += lsum;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kPFull + x));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kODone + x), (n_x - 1) & 1, abort_flag, 423));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const bool valid = i_row < L;
+      __nv_bfloat16* orow = O + (((size_t)b * L + (valid ? i_row : 0)) * Hq + h) * kHD;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + 32u * q, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+            w.y = pack_bf16(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            w.z = pack_bf16(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+            w.w = pack_bf16(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + q * 32 + e) = w;
+          }
+        }
+      }
+      if (valid)
+        LSE[((size_t)b * Hq + h) * L + i_row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace pp_path
+
+// Ping-pong tcgen05 prefill attention (D = 128, s % 256 == 0).
+cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
+                                         void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                         int D, int s, float scale, cudaStream_t stream) {
+  using namespace pp_path;
+  if (D != kHD || s % (2 * kTile) != 0) return cudaErrorInvalidValue;
+  if (L == 0 || B == 0) return cudaSuccess;
+  CUtensorMap tmQ, tmK, tmV;
+  const uint32_t box[4] = {64, 1, (uint32_t)kTile, 1};
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)L, (uint64_t)3 * B};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hq * D * 2,
+                                 (uint64_t)L * Hq * D * 2};
+    if (!encode_tensor_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Qrot, 4, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)L, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
+                                 (uint64_t)L * Hkv * D * 2};
+    if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  auto kern = prefill_attn_pp_kernel;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+  if (e != cudaSuccess) return e;
+  const int num_qt = (L + kTile - 1) / kTile;
+  dim3 grid((num_qt + 1) / 2, Hq, B);
+  kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
+                                             B, L, Hq, Hkv, s, scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
+}  // namespace dca

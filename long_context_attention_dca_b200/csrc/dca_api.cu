@@ -204,7 +204,9 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (path == DCA_PATH_TCGEN05)
+  if (path == DCA_PATH_TCGEN05 && s % 256 == 0)
+    e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
+  else if (path == DCA_PATH_TCGEN05)
     e = launch_prefill_attn_sm100(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, c, sc,
                                   sm_count(), strm);
   else

@@ -12,6 +12,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "this library targets sm_100a only"
 #endif
@@ -98,6 +100,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+
+// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
+// the same one).  The counts used by a kernel must sum, over its warpgroups,
+// to no more than the registers the block was launched with.
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------

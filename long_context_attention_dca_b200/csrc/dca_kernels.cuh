@@ -30,6 +30,11 @@ cudaError_t launch_prefill_attn_sm100(const void* Qrot, const void* Krot, const 
                                       float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
                                       int c, float scale, int num_sms, cudaStream_t stream);
 
+// tcgen05 ping-pong variant: two query tiles per CTA (D = 128, s % 256 == 0).
+cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
+                                         void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                         int D, int s, float scale, cudaStream_t stream);
+
 // Split-KV decode + LSE merge.
 size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap);
 cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const int* t, void* O,

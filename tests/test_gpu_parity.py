@@ -140,6 +140,13 @@ SMALL = [  # (B, L, Hq, Hkv, D, s, c)
     (1, 900, 2, 2, 128, 256, 384),
     (1, 640, 2, 1, 128, 128, 1000),    # w > s
     (1, 129, 3, 3, 64, 16, 20),
+    # s % 256 == 0: the two-tile (ping-pong) tensor-core kernel
+    (1, 1, 1, 1, 128, 256, 256),
+    (2, 1000, 4, 2, 128, 256, 256),    # w = 0
+    (1, 1500, 2, 1, 128, 512, 768),
+    (1, 1300, 2, 2, 128, 256, 4096),   # w > s
+    (1, 129, 2, 2, 128, 256, 300),
+    (1, 2200, 4, 1, 128, 512, 640),
 ]
 
 
