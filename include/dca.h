@@ -143,6 +143,19 @@ dca_status_t dca_attn_decode(const void* q, const void* Kcache, const void* Vcac
                              int Tcap, int s, int c, float base, float scale, void* workspace,
                              size_t ws_bytes, void* stream);
 
+/* Append one decoded token per sequence to the caches: k_new, v_new
+ * [B][Hkv][D] bf16 hold the new token's UNROTATED key and its value; the key
+ * is rotated at t[b] mod s (the DCA key rule, as dca_rope_rotate with
+ * DCA_POS_KEY) and both are written to cache row t[b] of Kcache / Vcache
+ * [B][Tcap][Hkv][D].  Other rows are untouched.  t int32 [B] on the device;
+ * a t[b] outside [0, Tcap) is skipped and reported by dca_sync_status
+ * (INVALID_ARG).  Source: the key rule above; decode then reads keys 0 .. t[b]
+ * (Guide, "Strategic Recommendations", item 3: FlashDecoding over the cache).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+dca_status_t dca_kv_append(const void* k_new, const void* v_new, void* Kcache, void* Vcache,
+                           const int* t, int B, int Hkv, int D, int Tcap, int s, int c,
+                           float base, void* stream);
+
 /* dca_attn_decode for callers that cannot allocate device memory (e.g. a
  * plugin inside a serving framework whose allocator owns the GPU's memory, or
  * a decode loop that must avoid cudaMalloc's implicit synchronisation).  Same

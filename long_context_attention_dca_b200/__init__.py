@@ -23,7 +23,7 @@ __all__ = [
     "DCA_PATH_AUTO", "DCA_PATH_GENERAL", "DCA_PATH_TCGEN05",
     "dca_rope_rotate", "dca_attn_prefill_workspace", "dca_prefill_rope",
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
-    "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc",
+    "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
     "dca_debug_index_map",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
 ]
@@ -48,6 +48,7 @@ _SIGS = {
     "dca_attn_decode_workspace": (_Z, [_I, _I, _I, _I]),
     "dca_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
                              _Z, _P]),
+    "dca_kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "dca_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                                      _F, _P]),
     "dca_debug_index_map": (_I, [_I, _I, _I, _P, _P, _P, _P]),
@@ -206,6 +207,18 @@ def dca_attn_decode(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, workspa
                                  _ptr(LSE), B, Hq, Hkv, D, Tcap, s, c, base, scale, _ptr(ws),
                                  ws.numel(), _stream(q)))
     return O, LSE
+
+
+def dca_kv_append(k_new, v_new, Kcache, Vcache, t, s, c, base=10000.0):
+    """Write each sequence's new token (key rotated at t mod s) to cache row t."""
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    _need(t, "t", torch.int32, 1)
+    B, Hkv, D = k_new.shape
+    _check(lib().dca_kv_append(_ptr(k_new), _ptr(v_new), _ptr(Kcache), _ptr(Vcache), _ptr(t), B,
+                               Hkv, D, Kcache.shape[1], s, c, base, _stream(k_new)))
 
 
 def dca_attn_decode_noalloc(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, O=None,

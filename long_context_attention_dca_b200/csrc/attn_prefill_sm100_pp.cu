@@ -59,6 +59,11 @@ constexpr int kSmTotal = kSmMisc + 16 + 1024;
 static_assert(kSmTotal <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+// Of every 8 column pairs of an off-diagonal tile, this many could be
+// exponentiated on the FMA pipe instead of the special-function unit; measured
+// on B200 the softmax here is latency-bound, not exponent-throughput-bound
+// (1 of 8: no change, 2-3 of 8: slower), so none are.
+constexpr int kPolyPairs = 0;
 
 struct Phases {
   int n;
@@ -272,10 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
       if (!ok) break;
       tc_fence_after();
       uint32_t v[4][32];
+      const bool diag = (i == n_x - 1);
 #pragma unroll
       for (int q = 0; q < 4; ++q) tmem_ld32(s_addr + 32u * q, v[q]);
       tmem_wait_ld();
-      const bool diag = (i == n_x - 1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_reg_fence(v[q]);
       float mx;
       if (diag) mx = row_max_causal(v, row);  // causal mask on the diagonal tile only
       else mx = row_max(v);
@@ -302,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         m_run = m_new;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const float lsum = row_exp_store(v, scale_log2, m_use, s_addr);
+      const float lsum = diag ? row_exp_store<0>(v, scale_log2, m_use, s_addr)
+                              : row_exp_store<kPolyPairs>(v, scale_log2, m_use, s_addr);
       tmem_wait_st();
       l_run += lsum;
       tc_fence_before();

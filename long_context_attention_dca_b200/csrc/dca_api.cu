@@ -256,6 +256,25 @@ dca_status_t dca_attn_decode(const void* q, const void* Kcache, const void* Vcac
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 
+dca_status_t dca_kv_append(const void* k_new, const void* v_new, void* Kcache, void* Vcache,
+                           const int* t, int B, int Hkv, int D, int Tcap, int s, int c,
+                           float base, void* stream) {
+  const char* fn = "dca_kv_append";
+  dca_status_t st = check_heads(fn, B, 1, Hkv, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (Tcap < 1) return fail(DCA_ERR_INVALID_ARG, "%s: Tcap=%d", fn, Tcap);
+  if (B == 0) return DCA_OK;
+  DCA_CHECK_PTR(k_new);
+  DCA_CHECK_PTR(v_new);
+  DCA_CHECK_PTR(Kcache);
+  DCA_CHECK_PTR(Vcache);
+  if (t == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: t is null", fn);
+  cudaError_t e = launch_kv_append(k_new, v_new, Kcache, Vcache, t, B, Hkv, D, Tcap, s, base,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 dca_status_t dca_debug_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
                                  void* stream) {
   const char* fn = "dca_debug_index_map";

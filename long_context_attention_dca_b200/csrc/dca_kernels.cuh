@@ -35,6 +35,11 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream);
 
+// Decode-time append of one token per sequence into pre-rotated caches.
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, void* Vc,
+                             const int* t, int B, int Hkv, int D, int Tcap, int s, float base,
+                             cudaStream_t stream);
+
 // Split-KV decode + LSE merge.
 size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap);
 cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const int* t, void* O,

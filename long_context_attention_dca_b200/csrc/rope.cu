@@ -10,10 +10,10 @@
 // rounded to nearest even: bf16 for dca_rope_rotate (a cache in the caller's
 // type), fp16 for the prefill workspace (operands of S = Q K^T only).
 //
-// Both kernels are HBM-bound: each thread owns one token row and one group of
-// 8 rotation pairs (16 bytes of the first half and the matching 16 bytes of
-// the second half) and loops over the heads, so the cos/sin of a row are
-// computed once and reused by every head.
+// Both kernels are HBM-bound.  dca_rope_rotate's kernel: each thread owns one
+// token row and one group of 8 rotation pairs (16 bytes of the first half and
+// the matching 16 bytes of the second half) and loops over the heads, so the
+// cos/sin of a row are computed once and reused by every head.
 #include "dca_common.cuh"
 #include "dca_index.cuh"
 #include "dca_kernels.cuh"
@@ -112,57 +112,124 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(
 // Qrot layout: [3][B][L][Hq][D]; Krot: [B][L][Hkv][D].  Both are fp16: the
 // rotated operands of S = Q K^T keep 11 significant bits instead of bf16's 8,
 // which keeps the score error from rounding them near 4e-4 instead of 3e-3.
-__global__ void __launch_bounds__(256) prefill_rope_kernel(
-    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-    __half* __restrict__ Qrot, __half* __restrict__ Krot, int B, int L, int Hq,
-    int Hkv, int D, int s, int c, double log2_base) {
-  const int groups = D / 16;
-  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long total = (long long)B * L * groups;
-  if (gid >= total) return;
-  const int g = (int)(gid % groups);
-  const long long row = gid / groups;
-  const int im = (int)((row % L) % s);
-  const int p_succ = query_pos_for_piece(kSucc, im, s, c);
-  const bool succ_is_inter = (p_succ == c - 1);
-  const size_t plane = (size_t)B * L * Hq * D;
+//
+// HBM-bound layout: a block owns kRopeRows consecutive token rows.  It first
+// evaluates the cos/sin of the rows' three positions (j mod s, the successive
+// position, c - 1) into shared memory, then every thread streams independent
+// (row, head, 16-byte pair group) items, so many loads are in flight per SM
+// and each thread needs few registers.
+constexpr int kRopeRows = 4;
+constexpr int kRopeThreads = 256;
 
-  CosSin8 cs;
-  cos_sin_group(im, g * 8, D, log2_base, cs);  // key position == intra position
-  {
-    const size_t base_off = (size_t)row * Hkv * D + g * 8;
-#pragma unroll 4
-    for (int h = 0; h < Hkv; ++h) {
-      const size_t off = base_off + (size_t)h * D;
-      const uint4 lo = *reinterpret_cast<const uint4*>(K + off);
-      const uint4 hi = *reinterpret_cast<const uint4*>(K + off + D / 2);
-      uint4 olo, ohi;
-      rotate8<true>(lo, hi, cs, olo, ohi);
-      *reinterpret_cast<uint4*>(Krot + off) = olo;
-      *reinterpret_cast<uint4*>(Krot + off + D / 2) = ohi;
-    }
+template <int D>
+__global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+    __half* __restrict__ Qrot, __half* __restrict__ Krot, int B, int L, int Hq, int Hkv, int s,
+    int c, double log2_base) {
+  constexpr int kHalf = D / 2;
+  constexpr int kGroups = D / 16;
+  __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
+  const long long total_rows = (long long)B * L;
+  const long long row0 = (long long)blockIdx.x * kRopeRows;
+  const int nrows = (int)min((long long)kRopeRows, total_rows - row0);
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  for (int idx = threadIdx.x; idx < nrows * 3 * kHalf; idx += kRopeThreads) {
+    const int r = idx / (3 * kHalf), kind = (idx / kHalf) % 3, k = idx % kHalf;
+    const int im = (int)(((row0 + r) % L) % s);
+    const int pos = kind == 0 ? im : (kind == 1 ? query_pos_for_piece(kSucc, im, s, c) : c - 1);
+    const double theta = exp2(-(2.0 * (double)k / (double)D) * log2_base);
+    const double a = (double)pos * theta;
+    float sn, cn;
+    sincosf((float)fma(-rint(a * (1.0 / kTwoPi)), kTwoPi, a), &sn, &cn);
+    cs_s[r][kind][k] = make_float2(cn, sn);
   }
-  CosSin8 cs_succ, cs_inter;
-  cos_sin_group(c - 1, g * 8, D, log2_base, cs_inter);
-  if (!succ_is_inter) cos_sin_group(p_succ, g * 8, D, log2_base, cs_succ);
-  const size_t base_off = (size_t)row * Hq * D + g * 8;
+  __syncthreads();
+  const size_t plane = (size_t)B * L * Hq * D;
+  const int heads = Hq + Hkv;
+  const int items = nrows * heads * kGroups;
 #pragma unroll 2
-  for (int h = 0; h < Hq; ++h) {
-    const size_t off = base_off + (size_t)h * D;
-    const uint4 lo = *reinterpret_cast<const uint4*>(Q + off);
-    const uint4 hi = *reinterpret_cast<const uint4*>(Q + off + D / 2);
+  for (int it = threadIdx.x; it < items; it += kRopeThreads) {
+    const int g = it % kGroups;
+    const int hh = (it / kGroups) % heads;
+    const int r = it / (kGroups * heads);
+    const long long row = row0 + r;
+    const bool is_k = hh < Hkv;
+    const int h = is_k ? hh : hh - Hkv;
+    const size_t off = (size_t)row * (is_k ? Hkv : Hq) * D + (size_t)h * D + g * 8;
+    const __nv_bfloat16* src = is_k ? K : Q;
+    const uint4 lo = __ldg(reinterpret_cast<const uint4*>(src + off));
+    const uint4 hi = __ldg(reinterpret_cast<const uint4*>(src + off + kHalf));
+    CosSin8 cs;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 v = cs_s[r][0][g * 8 + e];
+      cs.c[e] = v.x;
+      cs.s[e] = v.y;
+    }
     uint4 olo, ohi;
     rotate8<true>(lo, hi, cs, olo, ohi);
-    *reinterpret_cast<uint4*>(Qrot + off) = olo;
-    *reinterpret_cast<uint4*>(Qrot + off + D / 2) = ohi;
-    uint4 ilo, ihi;
-    rotate8<true>(lo, hi, cs_inter, ilo, ihi);
-    *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = ilo;
-    *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + D / 2) = ihi;
-    if (!succ_is_inter) rotate8<true>(lo, hi, cs_succ, ilo, ihi);
-    *reinterpret_cast<uint4*>(Qrot + plane + off) = ilo;
-    *reinterpret_cast<uint4*>(Qrot + plane + off + D / 2) = ihi;
+    if (is_k) {
+      *reinterpret_cast<uint4*>(Krot + off) = olo;
+      *reinterpret_cast<uint4*>(Krot + off + kHalf) = ohi;
+      continue;
+    }
+    *reinterpret_cast<uint4*>(Qrot + off) = olo;  // intra plane
+    *reinterpret_cast<uint4*>(Qrot + off + kHalf) = ohi;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 v = cs_s[r][2][g * 8 + e];
+      cs.c[e] = v.x;
+      cs.s[e] = v.y;
+    }
+    rotate8<true>(lo, hi, cs, olo, ohi);  // inter plane (c - 1)
+    *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = olo;
+    *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + kHalf) = ohi;
+    const int im = (int)((row % L) % s);
+    if (query_pos_for_piece(kSucc, im, s, c) != c - 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float2 v = cs_s[r][1][g * 8 + e];
+        cs.c[e] = v.x;
+        cs.s[e] = v.y;
+      }
+      rotate8<true>(lo, hi, cs, olo, ohi);
+    }
+    *reinterpret_cast<uint4*>(Qrot + plane + off) = olo;  // successive plane
+    *reinterpret_cast<uint4*>(Qrot + plane + off + kHalf) = ohi;
   }
+}
+
+// Decode-time append: rotate the new key of sequence b at t[b] mod s and
+// store it, with the new value, at cache row t[b].  One thread per
+// (sequence, kv head, 16-byte pair group).
+__global__ void __launch_bounds__(256) kv_append_kernel(
+    const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
+    __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Vc, const int* __restrict__ t,
+    int B, int Hkv, int D, int Tcap, int s, double log2_base) {
+  const int groups = D / 16;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)B * Hkv * groups) return;
+  const int g = (int)(gid % groups);
+  const int h = (int)((gid / groups) % Hkv);
+  const int b = (int)(gid / ((long long)groups * Hkv));
+  const int tb = t[b];
+  if (tb < 0 || tb >= Tcap) {
+    if (g == 0 && h == 0) report_error(kDevBadArg, 202);
+    return;
+  }
+  CosSin8 cs;
+  cos_sin_group(tb % s, g * 8, D, log2_base, cs);
+  const size_t src = ((size_t)b * Hkv + h) * D + g * 8;
+  const size_t dst = (((size_t)b * Tcap + tb) * Hkv + h) * D + g * 8;
+  const uint4 lo = *reinterpret_cast<const uint4*>(k_new + src);
+  const uint4 hi = *reinterpret_cast<const uint4*>(k_new + src + D / 2);
+  uint4 olo, ohi;
+  rotate8(lo, hi, cs, olo, ohi);
+  *reinterpret_cast<uint4*>(Kc + dst) = olo;
+  *reinterpret_cast<uint4*>(Kc + dst + D / 2) = ohi;
+  *reinterpret_cast<uint4*>(Vc + dst) = *reinterpret_cast<const uint4*>(v_new + src);
+  *reinterpret_cast<uint4*>(Vc + dst + D / 2) =
+      *reinterpret_cast<const uint4*>(v_new + src + D / 2);
 }
 
 }  // namespace rope_path
@@ -186,15 +253,33 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
                                 cudaStream_t stream) {
   using namespace rope_path;
-  const long long total = (long long)B * L * (D / 16);
-  if (total == 0) return cudaSuccess;
-  const int threads = 256;
-  const unsigned blocks = (unsigned)((total + threads - 1) / threads);
-  prefill_rope_kernel<<<blocks, threads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-      static_cast<__half*>(Qrot), static_cast<__half*>(Krot), B, L, Hq, Hkv, D, s,
-      c, log2((double)base));
+  const long long rows = (long long)B * L;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + kRopeRows - 1) / kRopeRows);
+  auto args = [&](auto kern) {
+    kern<<<blocks, kRopeThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+        static_cast<__half*>(Qrot), static_cast<__half*>(Krot), B, L, Hq, Hkv, s, c,
+        log2((double)base));
+  };
+  if (D == 64) args(prefill_rope_kernel<64>);
+  else args(prefill_rope_kernel<128>);
   return cudaGetLastError();
 }
 
+}  // namespace dca
+
+namespace dca {
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, void* Vc,
+                             const int* t, int B, int Hkv, int D, int Tcap, int s, float base,
+                             cudaStream_t stream) {
+  using namespace rope_path;
+  const long long total = (long long)B * Hkv * (D / 16);
+  if (total == 0) return cudaSuccess;
+  kv_append_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+      static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), t, B, Hkv, D, Tcap, s,
+      log2((double)base));
+  return cudaGetLastError();
+}
 }  // namespace dca
