@@ -52,7 +52,7 @@ constexpr int kSmV = kSmK + 2 * kTileBytes;
 constexpr int kSmBar = kSmV + 2 * kTileBytes;
 enum Bar {
   kQFull = 0, kQEmpty = 3, kKFull = 6, kKEmpty = 8, kVFull = 10, kVEmpty = 12,
-  kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kNumBars = 21
+  kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kTokA = 21, kTokB = 25, kNumBars = 29
 };
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
 constexpr int kSmTotal = kSmMisc + 16 + 1024;
@@ -64,29 +64,6 @@ constexpr float kRescaleThreshold = 8.0f;
 // on B200 the softmax here is latency-bound, not exponent-throughput-bound
 // (1 of 8: no change, 2-3 of 8: slower), so none are.
 constexpr int kPolyPairs = 0;
-
-struct Phases {
-  int n;
-  int piece[3];
-  int begin[3];
-};
-
-__device__ __forceinline__ Phases make_phases(int ci, int tiles_per_chunk) {
-  Phases p;
-  p.n = 0;
-  if (ci >= 2) { p.piece[p.n] = kInter; p.begin[p.n] = 0; ++p.n; }
-  if (ci >= 1) { p.piece[p.n] = kSucc; p.begin[p.n] = (ci - 1) * tiles_per_chunk; ++p.n; }
-  p.piece[p.n] = kIntra; p.begin[p.n] = ci * tiles_per_chunk; ++p.n;
-  return p;
-}
-
-__device__ __forceinline__ int phase_of(const Phases& p, int j) {
-  int ph = 0;
-#pragma unroll
-  for (int k = 1; k < 3; ++k)
-    if (k < p.n && j >= p.begin[k]) ph = k;
-  return ph;
-}
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -108,7 +85,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   const int hk = h / (Hq / Hkv);
   const int q0 = m * 2 * kTile;
   const int tpc = s / kTile;
-  const Phases ph = make_phases(q0 / s, tpc);
+  // DCA pieces met by this query-tile pair, in walk order: phase p uses Qrot
+  // plane n_ph - 1 - p (inter = 2, successive = 1, intra = 0) and starts at key
+  // tile 0, b1 or b2 (kNever when the phase does not exist).
+  const int ci = q0 / s;
+  const int n_ph = ci >= 2 ? 3 : ci + 1;
+  constexpr int kNever = 0x7fffffff;
+  const int b1 = ci >= 2 ? (ci - 1) * tpc : (ci == 1 ? tpc : kNever);
+  const int b2 = ci >= 2 ? ci * tpc : kNever;
   const int nA = 2 * m + 1;  // key tiles 0 .. 2m   (diagonal of A)
   const int nB = 2 * m + 2;  // key tiles 0 .. 2m+1 (diagonal of B)
 
@@ -127,6 +111,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
       mbar_init(bar(kODone + i), 1);
     }
     mbar_init(bar(kMmaEnd), 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bar(kTokA + i), 1);
+      mbar_init(bar(kTokB + i), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -159,16 +147,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         mbar_arrive_expect_tx(fb, kTileBytes);
         const uint32_t dst = sbase + kSmQ + slot * kTileBytes;
         const int row = q0 + x * kTile;
-        tma_load_4d(dst, &tmQ, fb, 0, h, row, ph.piece[p] * B + b);
-        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, ph.piece[p] * B + b);
+        const int plane = n_ph - 1 - p;
+        tma_load_4d(dst, &tmQ, fb, 0, h, row, plane * B + b);
+        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, plane * B + b);
         q_last[slot] = n;
         return true;
       };
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
       ok = load_q(0) && load_q(1);
       for (int i = 0; i < nB && ok; ++i) {
-        const int p = phase_of(ph, i);
-        const bool boundary = (p > 0 && i == ph.begin[p]);
+        const int p = i >= b2 ? 2 : (i >= b1 ? 1 : 0);
+        const bool boundary = (i == b1) || (i == b2);
         if (boundary && !(ok = load_q(2 * p))) break;
         const int st = i & 1;
         if (i >= 2 && !(ok = mbar_wait(bar(kKEmpty + st), ((i >> 1) + 1) & 1, abort_flag, 402)))
@@ -201,30 +190,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc(128, 128, /*bf16=*/false, 0, 0);  // fp16 Q, K
       const uint32_t idesc_o = umma_idesc(128, 128, /*bf16=*/true, 0, 1);   // bf16 P, V
+      // Shared-memory descriptors built once; a buffer or k-step is selected by
+      // adding its byte offset / 16 to the start-address field (bits 0-13),
+      // which cannot carry out of the field for offsets inside shared memory.
+      const uint64_t dq0 = smem_desc_sw128(sbase + kSmQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sbase + kSmK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sbase + kSmV, kBox, 1024);
+      constexpr uint64_t kTileU = kTileBytes >> 4;
       auto issue_s = [&](int x, int i) -> bool {
-        const int p = phase_of(ph, i);
-        const int n = 2 * p + x;
-        const int slot = n % kNumQSlots;
-        if (i == ph.begin[p] &&
-            !mbar_wait(bar(kQFull + slot), (n / kNumQSlots) & 1, abort_flag, 411))
+        const int p = i >= b2 ? 2 : (i >= b1 ? 1 : 0);
+        const int n = 2 * p + x;              // Q load index: slot n % 3, use n / 3
+        const int slot = n >= 3 ? n - 3 : n;
+        if ((i == 0 || i == b1 || i == b2) &&
+            !mbar_wait(bar(kQFull + slot), n >= 3 ? 1u : 0u, abort_flag, 411))
           return false;
         const bool first_user = (x == 0) || (i >= nA);
         if (first_user && !mbar_wait(bar(kKFull + (i & 1)), (i >> 1) & 1, abort_flag, 412))
           return false;
         tc_fence_after();
-        const uint32_t qa = sbase + kSmQ + slot * kTileBytes;
-        const uint32_t ka = sbase + kSmK + (i & 1) * kTileBytes;
+        const uint64_t dq = dq0 + (uint64_t)slot * kTileU;
+        const uint64_t dk = dk0 + (uint64_t)(i & 1) * kTileU;
         const uint32_t d = tmem + 128u * (uint32_t)x;
 #pragma unroll
         for (int kk = 0; kk < kHD / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * kBox + (kk & 3) * 32);
-          umma_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                  idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+          umma_ss(d, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(kSFull + x));
         if (x == 1) umma_commit(bar(kKEmpty + (i & 1)));  // B is the last reader of K_i
-        const bool last_of_phase = (p + 1 < ph.n) ? (i == ph.begin[p + 1] - 1)
-                                                  : (i == (x ? nB : nA) - 1);
+        const int next_begin = p == 0 ? b1 : (p == 1 ? b2 : kNever);
+        const bool last_of_phase =
+            next_begin != kNever ? (i == next_begin - 1) : (i == (x ? nB : nA) - 1);
         if (last_of_phase) umma_commit(bar(kQEmpty + slot));
         return true;
       };
@@ -234,14 +230,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         if (first_user && !mbar_wait(bar(kVFull + (i & 1)), (i >> 1) & 1, abort_flag, 414))
           return false;
         tc_fence_after();
-        const uint32_t va = sbase + kSmV + (i & 1) * kTileBytes;
+        const uint64_t dv = dv0 + (uint64_t)(i & 1) * kTileU;
         const uint32_t pa = tmem + 128u * (uint32_t)x;
         const uint32_t od = tmem + 256u + 128u * (uint32_t)x;
+        umma_ts(od, pa, dv, idesc_o, i > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(od, pa + 8u * (uint32_t)kk,
-                  smem_desc_sw128(va + (uint32_t)kk * 2048u, kBox, 1024), idesc_o,
-                  (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < kTile / 16; ++kk)
+          umma_ts(od, pa + 8u * (uint32_t)kk, dv + (uint64_t)((kk * 2048) >> 4), idesc_o, 1u);
         umma_commit(bar(kODone + x));
         if (x == 1) umma_commit(bar(kVEmpty + (i & 1)));  // B is the last reader of V_i
         return true;
@@ -309,13 +304,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         m_run = m_new;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const float lsum = diag ? row_exp_store<0>(v, scale_log2, m_use, s_addr)
-                              : row_exp_store<kPolyPairs>(v, scale_log2, m_use, s_addr);
+      // The exponent phases of the two warps sharing this SMSP (A warp wq and
+      // B warp wq + 4) take turns: A(i), B(i), A(i+1), ... so neither runs its
+      // special-function-unit work at half rate.
+      const bool take_turn = (x == 0) ? (i > 0) : (i < nA);
+      if (take_turn) {
+        const uint32_t tb = x == 0 ? bar(kTokA + wq) : bar(kTokB + wq);
+        const int k = x == 0 ? i - 1 : i;
+        ok = __all_sync(0xffffffffu, mbar_wait(tb, k & 1, abort_flag, 425));
+        if (!ok) break;
+      }
+      row_exp_store_keep(v, scale_log2, m_use, s_addr);
       tmem_wait_st();
-      l_run += lsum;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kPFull + x));
+      if (lane == 0) {
+        mbar_arrive(bar(kPFull + x));
+        const bool pass_turn = (x == 0) ? (i < nB) : (i + 1 < nA);
+        if (pass_turn) mbar_arrive(x == 0 ? bar(kTokB + wq) : bar(kTokA + wq));
+      }
+      l_run += row_sum_of_p(v);  // off the path to the PV MMA
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kODone + x), (n_x - 1) & 1, abort_flag, 423));
     if (ok) {

@@ -143,6 +143,46 @@ __device__ __forceinline__ float row_exp_store(const uint32_t (&v)[4][32], float
   return a + b;
 }
 
+// P = exp2(S * scale_log2 - m) written as bf16 pairs to TMEM (p_addr ..
+// p_addr+63); the fp32 values of P replace the scores in v, so the row sum can
+// be taken after P has been handed to the MMA (row_sum_of_p).
+__device__ __forceinline__ void row_exp_store_keep(uint32_t (&v)[4][32], float scale_log2,
+                                                   float m_use, uint32_t p_addr) {
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t nm2 = f2_pack(-m_use, -m_use);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[q][2 * e]),
+                                         __uint_as_float(v[q][2 * e + 1])), sc2, nm2);
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      v[q][2 * e] = __float_as_uint(p0);
+      v[q][2 * e + 1] = __float_as_uint(p1);
+      pk[e] = pack_bf16(p0, p1);
+    }
+    tmem_st16(p_addr + 16u * q, pk);
+  }
+}
+
+__device__ __forceinline__ float row_sum_of_p(const uint32_t (&v)[4][32]) {
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      acc[e & 3] = f2_add(acc[e & 3], f2_pack(__uint_as_float(v[q][2 * e]),
+                                              __uint_as_float(v[q][2 * e + 1])));
+  const uint64_t s01 = f2_add(acc[0], acc[1]);
+  const uint64_t s23 = f2_add(acc[2], acc[3]);
+  float a, b;
+  f2_unpack(f2_add(s01, s23), a, b);
+  return a + b;
+}
+
 // ---- half rows (64 scores per thread): two threads share a row ----
 
 __device__ __forceinline__ float half_row_max(const uint32_t (&v)[2][32]) {
