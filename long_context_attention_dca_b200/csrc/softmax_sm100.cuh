@@ -183,57 +183,4 @@ __device__ __forceinline__ float row_sum_of_p(const uint32_t (&v)[4][32]) {
   return a + b;
 }
 
-// ---- half rows (64 scores per thread): two threads share a row ----
-
-__device__ __forceinline__ float half_row_max(const uint32_t (&v)[2][32]) {
-  float m[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) m[k] = fmaxf(__uint_as_float(v[0][2 * k]), __uint_as_float(v[0][2 * k + 1]));
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int e = (q == 0 ? 4 : 0); e < 16; ++e)
-      m[e & 3] = fmax3(m[e & 3], __uint_as_float(v[q][2 * e]), __uint_as_float(v[q][2 * e + 1]));
-  return fmax3(fmaxf(m[0], m[1]), m[2], m[3]);
-}
-
-// Diagonal tile: column col0 + c of row `row` is masked when col0 + c > row.
-__device__ __forceinline__ float half_row_max_causal(uint32_t (&v)[2][32], int row, int col0) {
-  const uint32_t neg_inf = 0xff800000u;
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (col0 + q * 32 + e > row) v[q][e] = neg_inf;
-  return half_row_max(v);
-}
-
-// P for 64 columns -> 32 packed bf16 columns at p_addr; returns the fp32 sum.
-__device__ __forceinline__ float half_row_exp_store(const uint32_t (&v)[2][32], float scale_log2,
-                                                    float m_use, uint32_t p_addr) {
-  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-  const uint64_t nm2 = f2_pack(-m_use, -m_use);
-  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[q][2 * e]),
-                                         __uint_as_float(v[q][2 * e + 1])), sc2, nm2);
-      float x0, x1;
-      f2_unpack(x2, x0, x1);
-      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-      acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
-      pk[e] = pack_bf16(p0, p1);
-    }
-    tmem_st16(p_addr + 16u * q, pk);
-  }
-  const uint64_t s01 = f2_add(acc[0], acc[1]);
-  const uint64_t s23 = f2_add(acc[2], acc[3]);
-  float a, b;
-  f2_unpack(f2_add(s01, s23), a, b);
-  return a + b;
-}
-
 }  // namespace dca
