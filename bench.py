@@ -218,6 +218,8 @@ def run_ours(args, rank, world, dev):
     do_dec = args.only in ("all", "decode")
     if not do_dec:  # profiling run: a 1-sequence, 1k-token stand-in keeps memory small
         dc = W.scaled(dc, B=1, Tcap=1024, t_lo=1000, t_hi=1001)
+    elif args.decode_seqs:
+        dc = W.scaled(dc, B=args.decode_seqs)
     t_dec, q_dec, Kc, Vc = W.make_decode_inputs(dc, device=dev)
     Bd, Hqd, Dd = q_dec.shape
     Tcap, Hkvd = Kc.shape[1], Kc.shape[2]
@@ -427,6 +429,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--decode-seqs", type=int, default=0,
+                    help="profiling runs: decode this many sequences instead of 16")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="profiling runs: time only one half of the step")
     ap.add_argument("--no-e2e", action="store_true",

@@ -184,6 +184,14 @@ dca_status_t dca_attn_decode_noalloc(const void* q, const void* Kcache, const vo
 dca_status_t dca_debug_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
                                  void* stream);
 
+/* Self-test of the failure path: enqueue a one-warp kernel that waits on an
+ * mbarrier nothing ever completes, bounded by deadline_us (1 .. 2e6).  The
+ * wait gives up, the kernel records a timeout in the error word and returns,
+ * so the next dca_sync_status() reports DCA_ERR_TIMEOUT and the context stays
+ * usable.  No fault, trap or unbounded wait is involved.
+ * Errors: INVALID_ARG (deadline out of range), CUDA. */
+dca_status_t dca_debug_wait_timeout(int deadline_us, void* stream);
+
 /* Synchronise `stream`, then read and clear the current device's kernel error
  * word: DCA_OK, DCA_ERR_TIMEOUT (a pipeline wait gave up), DCA_ERR_INVALID_ARG
  * (a device-side argument check failed) or DCA_ERR_CUDA. */

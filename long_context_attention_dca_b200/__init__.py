@@ -24,7 +24,7 @@ __all__ = [
     "dca_rope_rotate", "dca_attn_prefill_workspace", "dca_prefill_rope",
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
     "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
-    "dca_debug_index_map",
+    "dca_debug_index_map", "dca_debug_wait_timeout",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
 ]
 
@@ -52,6 +52,7 @@ _SIGS = {
     "dca_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                                      _F, _P]),
     "dca_debug_index_map": (_I, [_I, _I, _I, _P, _P, _P, _P]),
+    "dca_debug_wait_timeout": (_I, [_I, _P]),
     "dca_sync_status": (_I, [_P]),
     "dca_last_error_string": (ctypes.c_char_p, []),
 }
@@ -116,6 +117,11 @@ def dca_sync_status(device=None) -> None:
     """Synchronise the current stream and raise if a kernel reported an error."""
     dev = torch.device(device) if device is not None else torch.device("cuda")
     _check(lib().dca_sync_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+def dca_debug_wait_timeout(deadline_us: int = 20000) -> None:
+    """Enqueue the bounded-wait self-test (see include/dca.h)."""
+    _check(lib().dca_debug_wait_timeout(deadline_us, _stream()))
 
 
 def dca_rope_rotate(x: torch.Tensor, rule: int, s: int, c: int, base: float = 10000.0,

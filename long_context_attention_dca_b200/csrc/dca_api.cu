@@ -287,6 +287,14 @@ dca_status_t dca_debug_index_map(int L, int s, int c, int* qpos, int* kpos, sign
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 
+dca_status_t dca_debug_wait_timeout(int deadline_us, void* stream) {
+  const char* fn = "dca_debug_wait_timeout";
+  if (deadline_us < 1 || deadline_us > 2000000)
+    return fail(DCA_ERR_INVALID_ARG, "%s: deadline %d us (1 .. 2000000)", fn, deadline_us);
+  cudaError_t e = launch_wait_timeout(deadline_us, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 dca_status_t dca_sync_status(void* stream) {
   const char* fn = "dca_sync_status";
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

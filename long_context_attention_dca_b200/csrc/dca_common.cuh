@@ -86,14 +86,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  `abort_flag`
 // (shared memory) lets one role that gave up release the others quickly.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag, int site) {
+                                          volatile int* abort_flag, int site,
+                                          unsigned long long deadline_ns = kWaitDeadlineNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitDeadlineNs) {
+      if (global_timer_ns() - t0 > deadline_ns) {
         if (abort_flag != nullptr) *abort_flag = 1;
         report_error(kDevTimeout, site);
         return false;

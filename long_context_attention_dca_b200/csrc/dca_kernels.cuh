@@ -46,6 +46,8 @@ cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const i
                           float* LSE, int B, int Hq, int Hkv, int D, int Tcap, int s, int c,
                           float base, float scale, void* workspace, cudaStream_t stream);
 
+cudaError_t launch_wait_timeout(int deadline_us, cudaStream_t stream);
+
 cudaError_t launch_index_map(int L, int s, int c, int* qpos, int* kpos, signed char* piece,
                              cudaStream_t stream);
 

@@ -20,6 +20,19 @@ __global__ void index_map_kernel(int L, int s, int c, int* __restrict__ qpos,
   }
 }
 
+// Self-test of the bounded-wait failure path: wait on an mbarrier that nothing
+// ever arrives on.  The wait gives up after `deadline_ns`, records
+// kDevTimeout in the error word and the kernel returns normally.
+__global__ void wait_timeout_kernel(unsigned long long deadline_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, nullptr, 901, deadline_ns);
+}
+
 }  // namespace imap_path
 
 
@@ -30,6 +43,12 @@ cudaError_t launch_index_map(int L, int s, int c, int* qpos, int* kpos, signed c
   const long long n = (long long)L * L;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   index_map_kernel<<<blocks, 256, 0, stream>>>(L, s, c, qpos, kpos, piece);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout(int deadline_us, cudaStream_t stream) {
+  using namespace imap_path;
+  wait_timeout_kernel<<<1, 32, 0, stream>>>((unsigned long long)deadline_us * 1000ull);
   return cudaGetLastError();
 }
 

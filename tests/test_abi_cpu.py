@@ -113,6 +113,9 @@ def test_argument_errors_return_codes(lib):
                                      0.0, ws, 1 << 30, None)) == 1
     assert _code(lib.dca_attn_decode(*dargs, fake, fake, fake, 2, 8, 1, 128, 64, 16, 32, 1e4,
                                      0.0, ws, 8, None)) == 5
+    # wait self-test: deadline out of range
+    assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
+    assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1
     # index map: L too large, s > c
     assert _code(lib.dca_debug_index_map(9000, 4, 6, fake, fake, fake, None)) == 1
     assert _code(lib.dca_debug_index_map(16, 8, 6, fake, fake, fake, None)) == 2

@@ -93,3 +93,17 @@ def test_kv_append_rejects_position_outside_cache():
     assert ei.value.status == 1
     assert Vc[0, 3].float().eq(1).all() and Vc[1].float().eq(0).all()
     dca.dca_sync_status()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # a wait on a barrier that nothing completes gives up after 20 ms
+    dca.dca_debug_wait_timeout(20000)
+    with pytest.raises(dca.DcaError) as ei:
+        dca.dca_sync_status()
+    assert ei.value.status == 4  # DCA_ERR_TIMEOUT
+    dca.dca_sync_status()        # cleared
+    # the context still runs kernels correctly afterwards
+    qpos, kpos, piece = dca.dca_debug_index_map(12, 4, 6)
+    dca.dca_sync_status()
+    want = orc.index_map(12, 4, 6)
+    assert (qpos.cpu().numpy() == want[0]).all() and (piece.cpu().numpy() == want[2]).all()
