@@ -262,6 +262,46 @@ def dca_prefill(Q, K, V, s: int, c: int, base: float = 10000.0, scale: float = 0
     return O, LSE
 
 
+def dca_prefill_chunk(Qc, Kc, Vc, k_cache_rot, v_cache, t0: int, s: int, c: int,
+                      base: float = 10000.0, scale: float = 0.0, rows=None, heads=None,
+                      batches=None):
+    """Rows t0 .. t0+Lq-1 of a DCA prefill whose first t0 keys come from a cache.
+
+    Qc: [B, Lq, Hq, D], Kc, Vc: [B, Lq, Hkv, D] - the chunk's unrotated
+    queries and keys and its values; chunk row r is token t0 + r.
+    k_cache_rot, v_cache: [B, >= t0, Hkv, D] - keys 0 .. t0-1 ALREADY rotated
+    at j mod s (taken as stored) and their values.
+    The chunk's keys are rotated here at (t0 + r) mod s; chunk row r is query
+    i = t0 + r over keys 0 .. i, exactly as in dca_prefill_rows (the rule
+    depends only on the absolute indices).  Returns {(b, h, r): (O, LSE)}.
+    """
+    check_chunking(s, c)
+    B, Lq, Hq, D = Qc.shape
+    Hkv = Kc.shape[2]
+    sc = _scale(D, scale)
+    rows = range(Lq) if rows is None else rows
+    heads = range(Hq) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    rows = sorted(int(r) for r in rows)
+    out = {}
+    n = rows[-1] + 1
+    for b in batches:
+        for hk in sorted({kv_head(h, Hq, Hkv) for h in heads}):
+            k_new = rotate(np.asarray(Kc[b, :n, hk, :], np.float64),
+                           key_position(t0 + np.arange(n), s), base)
+            k_rot = np.concatenate([np.asarray(k_cache_rot[b, :t0, hk, :], np.float64), k_new])
+            v = np.concatenate([np.asarray(v_cache[b, :t0, hk, :], np.float64),
+                                np.asarray(Vc[b, :n, hk, :], np.float64)])
+            for h in heads:
+                if kv_head(h, Hq, Hkv) != hk:
+                    continue
+                for r in rows:
+                    i = t0 + r
+                    q = np.asarray(Qc[b, r, h, :], np.float64)
+                    out[(b, h, r)] = dca_row(q, k_rot[:i + 1], v[:i + 1], i, s, c, base, sc)
+    return out
+
+
 def dca_decode(q, k_cache_rot, v_cache, t, s: int, c: int,
                base: float = 10000.0, scale: float = 0.0, batches=None,
                heads=None):

@@ -5,7 +5,8 @@ with a version carrying a typical slip: an off-by-one in the successive rule,
 a dropped modulo, interleaved instead of half-split RoPE pairing, a flipped
 sign, a wrong frequency exponent, a missing softmax scale, a log2 LSE, a
 causal off-by-one, a wrong GQA mapping, a shifted chunk origin, a broken
-partial merge, or a decode that reads one key too few.  The pins of
+partial merge, a decode that reads one key too few, or a chunked prefill
+that ignores or misaligns its cache.  The pins of
 ``test_oracle_pins`` must reject each one.
 """
 
@@ -119,6 +120,18 @@ def _decode_short(q, k_cache_rot, v_cache, t, s, c, base=10000.0, scale=0.0,
 
 
 _ORIG_DECODE = orc.dca_decode
+_ORIG_CHUNK = orc.dca_prefill_chunk
+
+
+def _chunk_ignores_cache(Qc, Kc, Vc, k_cache_rot, v_cache, t0, s, c, *args, **kw):
+    # the chunk attends to its own keys only, as if it started the sequence
+    return _ORIG_CHUNK(Qc, Kc, Vc, k_cache_rot[:, :0], v_cache[:, :0], 0, s, c, *args, **kw)
+
+
+def _chunk_start_early(Qc, Kc, Vc, k_cache_rot, v_cache, t0, s, c, *args, **kw):
+    # off-by-one chunk start: one cached key too few, the chunk placed at t0 - 1
+    t = max(t0 - 1, 0)
+    return _ORIG_CHUNK(Qc, Kc, Vc, k_cache_rot[:, :t], v_cache[:, :t], t, s, c, *args, **kw)
 
 MUTANTS = {
     "succ_rule_le": ("query_position", _qpos_succ_le),
@@ -136,6 +149,8 @@ MUTANTS = {
     "chunk_origin_shift": ("piece", _piece_shift),
     "merge_mean": ("merge_partials", _merge_mean),
     "decode_short": ("dca_decode", _decode_short),
+    "chunk_ignores_cache": ("dca_prefill_chunk", _chunk_ignores_cache),
+    "chunk_start_early": ("dca_prefill_chunk", _chunk_start_early),
 }
 
 

@@ -239,6 +239,24 @@ def pin_decode_equals_prefill_row():
             np.testing.assert_allclose(LSE[b, h], lse, atol=1e-12)
 
 
+def pin_chunk_equals_prefill_rows():
+    # a chunk at t0 over a cache holding the earlier keys (rotated here by the
+    # independent complex-number RoPE at j mod s) gives rows t0 + r of the
+    # whole-sequence prefill, for chunk starts inside and at chunk boundaries
+    B, L, s, c = 2, 31, 6, 10
+    Q, K, V = _rand((B, L, 4, 8), 40), _rand((B, L, 2, 8), 41), _rand((B, L, 2, 8), 42)
+    k_rot = _complex_rotate(K, (np.arange(L) % s)[None, :, None], 10000.0)
+    full = orc.dca_prefill_rows(Q, K, V, s, c)
+    for t0, e in [(0, 9), (6, 13), (13, 31), (30, 31)]:
+        got = orc.dca_prefill_chunk(Q[:, t0:e], K[:, t0:e], V[:, t0:e], k_rot[:, :t0],
+                                    V[:, :t0], t0, s, c)
+        assert len(got) == B * 4 * (e - t0)
+        for (b, h, r), (o, lse) in got.items():
+            o_ref, lse_ref = full[(b, h, t0 + r)]
+            np.testing.assert_allclose(o, o_ref, atol=1e-12)
+            np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
 def pin_merge_partials():
     z, v = _rand(50, 27) * 3, _rand((50, 8), 28)
     o_full, lse_full = orc.softmax_row(z, v)
@@ -275,7 +293,8 @@ PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_rotation_literals, pin_rope_relativity, pin_plain_rope_matches_sdpa,
         pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
         pin_q_zero_closed_form, pin_constant_v, pin_gqa_mapping,
-        pin_decode_equals_prefill_row, pin_merge_partials, pin_rule_positions]
+        pin_decode_equals_prefill_row, pin_chunk_equals_prefill_rows, pin_merge_partials,
+        pin_rule_positions]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
