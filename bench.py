@@ -311,6 +311,10 @@ def run_ours(args, rank, world, dev):
     e2e = None if (args.no_e2e or args.only != "all") else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
                                            t_dec, Kc, Vc)
 
+    next_rows = None
+    if args.next_rows and args.only == "all":
+        next_rows = run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc)
+
     line = None
     if rank == 0:
         cpu = None
@@ -345,11 +349,12 @@ def run_ours(args, rank, world, dev):
                 "decode_split_kv+merge": {"bound": "hbm", "achieved": dec_gbs / world,
                                           "peak": hbm, "unit": "GB/s",
                                           "frac": dec_gbs / world / hbm,
-                                          "traffic": traffic.get("decode")},
+                                          "traffic": traffic.get("decode")} if do_dec else None,
                 "prefill_rope": {"bound": "hbm", "achieved": rope_gbs, "peak": hbm,
                                  "unit": "GB/s", "frac": rope_gbs / hbm,
-                                 "traffic": traffic.get("prefill_rope")}},
+                                 "traffic": traffic.get("prefill_rope")} if do_pre else None},
             "e2e": e2e,
+            "next_rows": next_rows,
             "gpu_launches": (2 * do_pre + 2 * do_dec) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
@@ -408,6 +413,118 @@ def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
             "api": "dca_attn_prefill + dca_attn_decode (decode KV cache device-resident)"}
 
 
+def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3):
+    """Device time of the calls beyond the step, each on the launching stream
+    with CUDA events, after one untimed call:
+      prefill_chunk  the prefill workload as four equal chunks against a cache
+                     (dca_attn_prefill_chunk, chunk starts 0, L/4, L/2, 3L/4);
+      prefill_3pass  the prefill workload as three single-piece passes merged
+                     by LSE (dca_attn_prefill_3pass);
+      kv_append      one decoded token appended per sequence of the decode
+                     batch (dca_kv_append), 100 calls back to back."""
+    import ctypes
+    P = ctypes.c_void_p
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    s, c, base = pc["s"], pc["c"], pc["base"]
+    flops = W.prefill_flops(pc)
+    out = {}
+
+    def timed(fn, n=reps):
+        fn()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dca.dca_sync_status(dev)
+        return a.elapsed_time(b) / n
+
+    # chunked prefill
+    n_chunks = 4
+    bounds = [L * k // n_chunks for k in range(n_chunks + 1)]
+    Kcache = torch.empty(B, L, Hkv, D, dtype=torch.bfloat16, device=dev)
+    Vcache = torch.empty_like(Kcache)
+    Qs = [Q[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+    Ks = [K[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+    Vs = [V[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+    wsz = max(dca.dca_attn_prefill_chunk_workspace(B, e - a, Hq, Hkv, D, a)
+              for a, e in zip(bounds[:-1], bounds[1:]))
+    cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    Oc = torch.empty_like(Q)
+    Lc = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    Ob = [torch.empty_like(q) for q in Qs]
+    Lb = [torch.empty(B, Hq, q.shape[1], dtype=torch.float32, device=dev) for q in Qs]
+
+    def chunks():
+        for k, (a, e) in enumerate(zip(bounds[:-1], bounds[1:])):
+            st = lib.dca_attn_prefill_chunk(
+                P(Qs[k].data_ptr()), P(Ks[k].data_ptr()), P(Vs[k].data_ptr()),
+                P(Kcache.data_ptr()), P(Vcache.data_ptr()), P(Ob[k].data_ptr()),
+                P(Lb[k].data_ptr()), B, e - a, Hq, Hkv, D, a, L, s, c, base, 0.0,
+                P(cws.data_ptr()), wsz, P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(chunks)
+    tc = all(a % 256 == 0 for a in bounds[:-1]) and s % 256 == 0 and D == 128
+    out["prefill_chunk"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                            "ms": ms, "chunks": n_chunks,
+                            "path": "tcgen05/TMEM/TMA" if tc else "general (warp MMA)",
+                            "launches_per_call": 3 if tc else 2}
+    del Kcache, Vcache, cws, Oc, Lc, Ob, Lb, Qs, Ks, Vs
+
+    # three passes + LSE merge
+    wsz = dca.dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D)
+    pws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    O3 = torch.empty_like(Q)
+    L3 = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+
+    def three():
+        st = lib.dca_attn_prefill_3pass(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
+                                        P(O3.data_ptr()), P(L3.data_ptr()), B, L, Hq, Hkv, D, s,
+                                        c, base, 0.0, P(pws.data_ptr()), wsz,
+                                        P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(three)
+    out["prefill_3pass"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
+                            "path": "general (warp MMA) x3 + merge", "launches_per_call": 5}
+    del pws, O3, L3
+
+    # decode-time append of one token per sequence (positions t_dec + 1 < Tcap)
+    Bd, Tcap, Hkvd, Dd = Kc.shape
+    kn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
+    vn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
+    t_app = torch.clamp(t_dec + 1, max=Tcap - 1).to(torch.int32)
+    Kc2, Vc2 = Kc.clone(), Vc.clone()  # the step's caches stay as they are
+
+    def append(strm):
+        for _ in range(100):
+            st = lib.dca_kv_append(P(kn.data_ptr()), P(vn.data_ptr()), P(Kc2.data_ptr()),
+                                   P(Vc2.data_ptr()), P(t_app.data_ptr()), Bd, Hkvd, Dd, Tcap,
+                                   dc["s"], dc["c"], dc["base"], P(strm.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+    ms_stream = timed(lambda: append(stream), 1) / 100
+    # the same 100 appends replayed from a CUDA graph (no host launch overhead)
+    side = torch.cuda.Stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        append(side)
+    ms_graph = timed(graph.replay, 1) / 100
+    del graph
+    nbytes = Bd * Hkvd * Dd * 2 * 4  # read k, v; write the two cache rows
+    out["kv_append"] = {"us_per_call": ms_graph * 1e3, "us_per_call_stream": ms_stream * 1e3,
+                        "bytes_per_call": nbytes, "timing": "100 appends in a CUDA graph",
+                        "bound": "launch latency (a few hundred KB per call)",
+                        "launches_per_call": 1}
+    del Kc2, Vc2
+    return out
+
+
 def _barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -433,6 +550,9 @@ def main():
                     help="profiling runs: decode this many sequences instead of 16")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="profiling runs: time only one half of the step")
+    ap.add_argument("--next-rows", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time chunked prefill, the 3-pass variant and KV append "
+                         "(outside the timed step)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default=PREFILL, choices=sorted(

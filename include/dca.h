@@ -120,6 +120,60 @@ dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void*
                               int B, int L, int Hq, int Hkv, int D, int s, int c, float base,
                               float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/* Workspace bytes for dca_attn_prefill_3pass: the prefill workspace plus, for
+ * each of the three pieces, an fp32 output [B][L][Hq][D] and an fp32 LSE
+ * [B][Hq][L].  Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_3pass_workspace(int B, int L, int Hq, int Hkv, int D);
+
+/* DCA prefill as three flash passes merged by their LSE: the intra-chunk,
+ * successive-chunk and inter-chunk pieces are each attended with their own
+ * softmax (the reading of "decomposing the attention into chunk-based
+ * modules ... integrates with Flash Attention", arXiv Abstract), then
+ * O = sum_p e^{LSE_p - LSE} O_p and LSE = ln sum_p e^{LSE_p}.  Same inputs,
+ * outputs and conventions as dca_attn_prefill; mathematically equal to it (one
+ * softmax over the union of the pieces) and computed by the warp-MMA path, so
+ * it is an independent cross-check of the fused kernels.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_3pass(const void* Q, const void* K, const void* V, void* O,
+                                    float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
+                                    int c, float base, float scale, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/* Workspace bytes for dca_attn_prefill_chunk: the three fp16 query rotations
+ * [3][B][Lq][Hq][D] of the chunk plus the fp16 keys [B][t0+Lq][Hkv][D] the
+ * attention reads (cache rows 0 .. t0-1 converted, then the chunk's), each
+ * rounded up to 256 bytes.
+ * Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_chunk_workspace(int B, int Lq, int Hq, int Hkv, int D, int t0);
+
+/* Chunked prefill against an existing cache: the rows t0 .. t0+Lq-1 of a DCA
+ * prefill whose earlier rows 0 .. t0-1 were already processed.  The index rule
+ * depends only on the absolute indices i and j, so these rows are the same
+ * rows of a one-shot prefill over the whole sequence in which keys 0 .. t0-1
+ * are the cached (pre-rotated, bf16) values; the chunk's own keys are rotated
+ * in fp32 and, like dca_attn_prefill's, rounded once to fp16 for the score
+ * product.  Serves DCA as a drop-in wrapper of a serving
+ * stack that prefills long prompts piece by piece (Guide, "Strategic
+ * Recommendations", item 1) and builds the cache that dca_attn_decode reads.
+ *   Q [B][Lq][Hq][D], K, V [B][Lq][Hkv][D]: the chunk's UNROTATED queries and
+ *     keys and its values, bf16, dense.
+ *   Kcache, Vcache [B][Tcap][Hkv][D] bf16: rows 0 .. t0-1 hold keys already
+ *     rotated at j mod s (as written by earlier calls, dca_rope_rotate with
+ *     DCA_POS_KEY or dca_kv_append) and their values.  This call writes the
+ *     chunk's rotated keys and values to rows t0 .. t0+Lq-1 and leaves every
+ *     other row untouched.
+ *   O [B][Lq][Hq][D] bf16 and LSE [B][Hq][Lq] fp32: results for the chunk.
+ *   t0 (host int) is the same for every sequence; 0 <= t0, t0 + Lq <= Tcap.
+ * The call owns no memory; `workspace` (dca_attn_prefill_chunk_workspace
+ * bytes, 256-byte aligned) is scratch for the call's duration.  Path: with
+ * D == 128, s % 256 == 0 and t0 % 256 == 0 the tcgen05 kernel runs with the
+ * query offset; otherwise the warp-MMA kernel (any s, D in {64, 128}).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V, void* Kcache,
+                                    void* Vcache, void* O, float* LSE, int B, int Lq, int Hq,
+                                    int Hkv, int D, int t0, int Tcap, int s, int c, float base,
+                                    float scale, void* workspace, size_t ws_bytes, void* stream);
+
 /* Which prefill path DCA_PATH_AUTO takes for these sizes (1 general,
  * 2 tcgen05), or 0 for unsupported arguments. */
 int dca_prefill_path(int L, int D, int s, int c);

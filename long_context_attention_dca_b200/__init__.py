@@ -23,6 +23,8 @@ __all__ = [
     "DCA_PATH_AUTO", "DCA_PATH_GENERAL", "DCA_PATH_TCGEN05",
     "dca_rope_rotate", "dca_attn_prefill_workspace", "dca_prefill_rope",
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
+    "dca_attn_prefill_3pass_workspace", "dca_attn_prefill_3pass",
+    "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
     "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
     "dca_debug_index_map", "dca_debug_wait_timeout",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
@@ -45,6 +47,12 @@ _SIGS = {
     "dca_attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _Z,
                               _P]),
     "dca_prefill_path": (_I, [_I, _I, _I, _I]),
+    "dca_attn_prefill_3pass_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "dca_attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                    _I, _F, _F, _P, _Z, _P]),
+    "dca_attn_prefill_3pass": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
+                                    _Z, _P]),
     "dca_attn_decode_workspace": (_Z, [_I, _I, _I, _I]),
     "dca_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
                              _Z, _P]),
@@ -188,6 +196,53 @@ def dca_attn_prefill(Q, K, V, s, c, base=10000.0, scale=0.0, workspace=None, O=N
     _need(LSE, "LSE", torch.float32, 3)
     _check(lib().dca_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L, Hq, Hkv,
                                   D, s, c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_3pass_workspace(B: int, L: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D))
+
+
+def dca_attn_prefill_3pass(Q, K, V, s, c, base=10000.0, scale=0.0):
+    """DCA prefill as three single-piece flash passes merged by LSE."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    nbytes = dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
+    _check(lib().dca_attn_prefill_3pass(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L, Hq,
+                                        Hkv, D, s, c, base, scale, _ptr(ws), ws.numel(),
+                                        _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_chunk_workspace(B: int, Lq: int, Hq: int, Hkv: int, D: int, t0: int) -> int:
+    return int(lib().dca_attn_prefill_chunk_workspace(B, Lq, Hq, Hkv, D, t0))
+
+
+def dca_attn_prefill_chunk(Q, K, V, Kcache, Vcache, t0, s, c, base=10000.0, scale=0.0):
+    """Prefill of the chunk Q/K/V at absolute rows t0 .. t0+Lq-1 against the
+    caches (rotated keys and values of rows 0 .. t0-1); appends the chunk to
+    the caches in place and returns its (O, LSE)."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    B, Lq, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    Tcap = Kcache.shape[1]
+    nbytes = dca_attn_prefill_chunk_workspace(B, Lq, Hq, Hkv, D, int(t0))
+    ws = _workspace(nbytes, Q.device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((B, Hq, Lq), dtype=torch.float32, device=Q.device)
+    _check(lib().dca_attn_prefill_chunk(_ptr(Q), _ptr(K), _ptr(V), _ptr(Kcache), _ptr(Vcache),
+                                        _ptr(O), _ptr(LSE), B, Lq, Hq, Hkv, D, int(t0), Tcap, s,
+                                        c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
     return O, LSE
 
 

@@ -52,7 +52,7 @@ constexpr int kSmV = kSmK + 2 * kTileBytes;
 constexpr int kSmBar = kSmV + 2 * kTileBytes;
 enum Bar {
   kQFull = 0, kQEmpty = 3, kKFull = 6, kKEmpty = 8, kVFull = 10, kVEmpty = 12,
-  kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kTokA = 21, kTokB = 25, kNumBars = 29
+  kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kNumBars = 21
 };
 constexpr int kSmMisc = kSmBar + kNumBars * 8;
 constexpr int kSmTotal = kSmMisc + 16 + 1024;
@@ -68,7 +68,8 @@ constexpr int kPolyPairs = 0;
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-    float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2) {
+    float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2,
+    int pair_off) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -80,10 +81,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_qt = (L + kTile - 1) / kTile;
   const int num_pairs = (num_qt + 1) / 2;
-  const int m = num_pairs - 1 - (int)blockIdx.x;  // longest pairs first
+  // Pair m covers absolute rows m*256 .. m*256+255; the call's query row r
+  // has absolute index pair_off*256 + r (pair_off > 0 for a chunk appended to
+  // a cache).
+  const int m = num_pairs - 1 - (int)blockIdx.x + pair_off;  // longest pairs first
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (Hq / Hkv);
-  const int q0 = m * 2 * kTile;
+  const int q0 = m * 2 * kTile;              // absolute
+  const int q0_loc = q0 - pair_off * 2 * kTile;
   const int tpc = s / kTile;
   // DCA pieces met by this query-tile pair, in walk order: phase p uses Qrot
   // plane n_ph - 1 - p (inter = 2, successive = 1, intra = 0) and starts at key
@@ -111,10 +116,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
       mbar_init(bar(kODone + i), 1);
     }
     mbar_init(bar(kMmaEnd), 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(bar(kTokA + i), 1);
-      mbar_init(bar(kTokB + i), 1);
-    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         const uint32_t fb = bar(kQFull + slot);
         mbar_arrive_expect_tx(fb, kTileBytes);
         const uint32_t dst = sbase + kSmQ + slot * kTileBytes;
-        const int row = q0 + x * kTile;
+        const int row = q0_loc + x * kTile;
         const int plane = n_ph - 1 - p;
         tma_load_4d(dst, &tmQ, fb, 0, h, row, plane * B + b);
         tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, plane * B + b);
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const int x = warp >> 2;               // 0 = tile A, 1 = tile B
     const int wq = warp & 3;               // TMEM lane quarter
     const int row = wq * 32 + lane;        // row within the tile
-    const int i_row = q0 + x * kTile + row;
+    const int i_row = q0_loc + x * kTile + row;  // row of this call
     const int n_x = x ? nB : nA;
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_addr = t_lane + 128u * (uint32_t)x;
@@ -304,25 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         m_run = m_new;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      // The exponent phases of the two warps sharing this SMSP (A warp wq and
-      // B warp wq + 4) take turns: A(i), B(i), A(i+1), ... so neither runs its
-      // special-function-unit work at half rate.
-      const bool take_turn = (x == 0) ? (i > 0) : (i < nA);
-      if (take_turn) {
-        const uint32_t tb = x == 0 ? bar(kTokA + wq) : bar(kTokB + wq);
-        const int k = x == 0 ? i - 1 : i;
-        ok = __all_sync(0xffffffffu, mbar_wait(tb, k & 1, abort_flag, 425));
-        if (!ok) break;
-      }
       row_exp_store_keep(v, scale_log2, m_use, s_addr);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(kPFull + x));
-        const bool pass_turn = (x == 0) ? (i < nB) : (i + 1 < nA);
-        if (pass_turn) mbar_arrive(x == 0 ? bar(kTokB + wq) : bar(kTokA + wq));
-      }
+      if (lane == 0) mbar_arrive(bar(kPFull + x));
       l_run += row_sum_of_p(v);  // off the path to the PV MMA
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kODone + x), (n_x - 1) & 1, abort_flag, 423));
@@ -363,13 +350,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
 
 }  // namespace pp_path
 
-// Ping-pong tcgen05 prefill attention (D = 128, s % 256 == 0).
+// Ping-pong tcgen05 prefill attention (D = 128, s % 256 == 0).  Query rows
+// are q_off .. q_off+L-1 (q_off % 256 == 0) of sequences whose keys 0 ..
+// q_off+L-1 sit in Krot / V with kv_rows rows per sequence.
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
-                                         int D, int s, float scale, cudaStream_t stream) {
+                                         int D, int s, float scale, cudaStream_t stream,
+                                         int q_off, int k_rows, int v_rows) {
   using namespace pp_path;
-  if (D != kHD || s % (2 * kTile) != 0) return cudaErrorInvalidValue;
+  if (D != kHD || s % (2 * kTile) != 0 || q_off % (2 * kTile) != 0) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
+  const int Lkv = q_off + L;
+  if (k_rows == 0) k_rows = Lkv;
+  if (v_rows == 0) v_rows = Lkv;
   CUtensorMap tmQ, tmK, tmV;
   const uint32_t box[4] = {64, 1, (uint32_t)kTile, 1};
   {
@@ -381,12 +374,14 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)L, (uint64_t)B};
-    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
-                                 (uint64_t)L * Hkv * D * 2};
-    if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, dims, strides, box,
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)B};
+    const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
+                            (uint64_t)k_rows * Hkv * D * 2};
+    const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
+                            (uint64_t)v_rows * Hkv * D * 2};
+    if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, dims, ks, box,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, dims, strides, box,
+        !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, dims, vs, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -397,7 +392,8 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
   const int num_qt = (L + kTile - 1) / kTile;
   dim3 grid((num_qt + 1) / 2, Hq, B);
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
-                                             B, L, Hq, Hkv, s, scale * 1.4426950408889634f);
+                                             B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
+                                             q_off / (2 * kTile));
   return cudaGetLastError();
 }
 

@@ -224,6 +224,93 @@ dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void*
                                workspace, ws_bytes, stream);
 }
 
+size_t dca_attn_prefill_3pass_workspace(int B, int L, int Hq, int Hkv, int D) {
+  const size_t base = dca_attn_prefill_workspace(B, L, Hq, Hkv, D);
+  if (base == 0 && !(B == 0 || L == 0)) return 0;
+  return base + align256((size_t)3 * B * L * Hq * D * 4) + align256((size_t)3 * B * Hq * L * 4);
+}
+
+dca_status_t dca_attn_prefill_3pass(const void* Q, const void* K, const void* V, void* O,
+                                    float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
+                                    int c, float base, float scale, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_prefill_3pass";
+  dca_status_t st = check_heads(fn, B, L, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if ((long long)B * L == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
+  PrefillWs ws = prefill_ws_layout(workspace, B, L, Hq, Hkv, D);
+  float* Op = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws.bytes);
+  float* LSEp = reinterpret_cast<float*>(reinterpret_cast<char*>(Op) +
+                                         align256((size_t)3 * B * L * Hq * D * 4));
+  const size_t o_plane = (size_t)B * L * Hq * D, l_plane = (size_t)B * Hq * L;
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_prefill_rope(Q, K, ws.qrot, ws.krot, B, L, Hq, Hkv, D, s, c, base, strm);
+  for (int p = 0; p < 3 && e == cudaSuccess; ++p)  // intra, successive, inter
+    e = launch_prefill_attn_mma(ws.qrot, ws.krot, V, nullptr, LSEp + p * l_plane, B, L, Hq, Hkv,
+                                D, s, c, sc, strm, 1 << p, Op + p * o_plane);
+  if (e == cudaSuccess) e = launch_merge3(Op, LSEp, O, LSE, B, L, Hq, D, strm);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+size_t dca_attn_prefill_chunk_workspace(int B, int Lq, int Hq, int Hkv, int D, int t0) {
+  if (B < 0 || Lq < 0 || t0 < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128))
+    return 0;
+  return align256((size_t)3 * B * Lq * Hq * D * 2) +
+         align256((size_t)B * ((size_t)t0 + Lq) * Hkv * D * 2);
+}
+
+dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V, void* Kcache,
+                                    void* Vcache, void* O, float* LSE, int B, int Lq, int Hq,
+                                    int Hkv, int D, int t0, int Tcap, int s, int c, float base,
+                                    float scale, void* workspace, size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_prefill_chunk";
+  dca_status_t st = check_heads(fn, B, Lq, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (t0 < 0 || Tcap < 1 || (long long)t0 + Lq > Tcap)
+    return fail(DCA_ERR_INVALID_ARG, "%s: chunk rows [%d, %lld) outside cache of %d rows", fn,
+                t0, (long long)t0 + Lq, Tcap);
+  if ((long long)B * Lq == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(Kcache);
+  DCA_CHECK_PTR(Vcache);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = dca_attn_prefill_chunk_workspace(B, Lq, Hq, Hkv, D, t0);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  // Keys 0 .. t0-1 come from the cache (bf16, exact in fp16); the chunk's own
+  // keys are rotated here and rounded once, to fp16, like a one-shot prefill.
+  void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * B * Lq * Hq * D * 2);
+  cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, B, Lq, Hq, Hkv, D,
+                                    t0, Tcap, s, c, base, strm);
+  if (e == cudaSuccess) e = launch_keys_to_f16(Kcache, kf16, B, t0, Tcap, t0 + Lq, Hkv, D, strm);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (auto_path(D, s) == DCA_PATH_TCGEN05 && s % 256 == 0 && t0 % 256 == 0)
+    e = launch_prefill_attn_sm100_pp(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
+                                     strm, t0, t0 + Lq, Tcap);
+  else
+    e = launch_prefill_attn_mma_chunk(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, c, sc,
+                                      t0, Tcap, strm);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 size_t dca_attn_decode_workspace(int B, int Hq, int D, int Tcap) {
   if (B < 0 || Hq < 1 || (D != 64 && D != 128) || Tcap < 1) return 0;
   return decode_workspace_bytes(B, Hq, D, Tcap);

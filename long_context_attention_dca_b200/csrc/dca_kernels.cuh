@@ -20,10 +20,30 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
                                 cudaStream_t stream);
 
-// General prefill attention (warp MMA; any s, D in {64, 128}).
+// Chunk of Lq rows at absolute positions t0 .. t0+Lq-1: Qrot [3][B][Lq][Hq][D]
+// fp16; rotated keys go in bf16 to cache rows t0 + r (pitch Tcap) and in fp16
+// to rows t0 + r of Kf16 [B][t0+Lq][Hkv][D]; values to cache rows t0 + r.
+cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
+                              void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
+                              int Hkv, int D, int t0, int Tcap, int s, int c, float base,
+                              cudaStream_t stream);
+// Attention of that chunk over keys 0 .. t0+Lq-1 of Kf16 and the value cache
+// (general path).
+cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* Vcache,
+                                          void* O, float* LSE, int B, int Lq, int Hq, int Hkv,
+                                          int D, int s, int c, float scale, int t0, int Tcap,
+                                          cudaStream_t stream);
+
+// General prefill attention (warp MMA; any s, D in {64, 128}).  piece_mask
+// selects the pieces the softmax covers (1 intra, 2 successive, 4 inter; 7 =
+// DCA); with Of32 set, the normalised O is written there in fp32 instead.
 cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const void* V, void* O,
                                     float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
-                                    int c, float scale, cudaStream_t stream);
+                                    int c, float scale, cudaStream_t stream, int piece_mask = 7,
+                                    float* Of32 = nullptr);
+// Merge of the three single-piece passes (Op [3][B][L][Hq][D], LSEp [3][B][Hq][L]).
+cudaError_t launch_merge3(const float* Op, const float* LSEp, void* O, float* LSE, int B, int L,
+                          int Hq, int D, cudaStream_t stream);
 
 // tcgen05/TMEM/TMA prefill attention (D = 128, s % 128 == 0).
 cudaError_t launch_prefill_attn_sm100(const void* Qrot, const void* Krot, const void* V, void* O,
@@ -31,9 +51,16 @@ cudaError_t launch_prefill_attn_sm100(const void* Qrot, const void* Krot, const 
                                       int c, float scale, int num_sms, cudaStream_t stream);
 
 // tcgen05 ping-pong variant: two query tiles per CTA (D = 128, s % 256 == 0).
+// Chunk form: query rows q_off .. q_off+L-1 (q_off % 256 == 0) against keys
+// 0 .. q_off+L-1 held with k_rows / v_rows rows per sequence (0: q_off + L).
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
-                                         int D, int s, float scale, cudaStream_t stream);
+                                         int D, int s, float scale, cudaStream_t stream,
+                                         int q_off = 0, int k_rows = 0, int v_rows = 0);
+// Rows 0 .. rows-1 of a bf16 key cache [B][Tcap][Hkv][D] -> the same rows of
+// fp16 [B][out_rows][Hkv][D].
+cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
+                               int out_rows, int Hkv, int D, cudaStream_t stream);
 
 // Decode-time append of one token per sequence into pre-rotated caches.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, void* Vc,

@@ -121,11 +121,18 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(
 constexpr int kRopeRows = 4;
 constexpr int kRopeThreads = 256;
 
-template <int D>
+// Rows are the B x L query/key rows of one call.  Row r of a sequence sits at
+// absolute index q_off + r.  Whole-sequence prefill (kChunk false, q_off 0)
+// writes the rotated keys to the fp16 workspace Kout laid out like K.  A chunk
+// against a cache (kChunk true) writes them in bf16 to cache rows q_off + r of
+// pitch Tcap (Kout) and in fp16 to rows q_off + r of Kh (pitch q_off + L), and
+// copies the chunk's values into the value cache.
+template <int D, bool kChunk>
 __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-    __half* __restrict__ Qrot, __half* __restrict__ Krot, int B, int L, int Hq, int Hkv, int s,
-    int c, double log2_base) {
+    __half* __restrict__ Qrot, void* __restrict__ Kout, int B, int L, int Hq, int Hkv, int s,
+    int c, double log2_base, int q_off, int Tcap, const __nv_bfloat16* __restrict__ Vsrc,
+    __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh) {
   constexpr int kHalf = D / 2;
   constexpr int kGroups = D / 16;
   __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
@@ -135,7 +142,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   for (int idx = threadIdx.x; idx < nrows * 3 * kHalf; idx += kRopeThreads) {
     const int r = idx / (3 * kHalf), kind = (idx / kHalf) % 3, k = idx % kHalf;
-    const int im = (int)(((row0 + r) % L) % s);
+    const int im = (int)((((row0 + r) % L) + q_off) % s);
     const int pos = kind == 0 ? im : (kind == 1 ? query_pos_for_piece(kSucc, im, s, c) : c - 1);
     const double theta = exp2(-(2.0 * (double)k / (double)D) * log2_base);
     const double a = (double)pos * theta;
@@ -145,14 +152,50 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   }
   __syncthreads();
   const size_t plane = (size_t)B * L * Hq * D;
-  const int heads = Hq + Hkv;
+  const int heads = Hq + (kChunk ? 2 : 1) * Hkv;  // [keys | (values) | queries]
   const int items = nrows * heads * kGroups;
 #pragma unroll 2
   for (int it = threadIdx.x; it < items; it += kRopeThreads) {
     const int g = it % kGroups;
-    const int hh = (it / kGroups) % heads;
+    int hh = (it / kGroups) % heads;
     const int r = it / (kGroups * heads);
     const long long row = row0 + r;
+    if constexpr (kChunk) {
+      const long long seq = row / L;
+      const size_t cache_row = (size_t)(seq * Tcap + (row % L) + q_off);
+      if (hh >= Hkv && hh < 2 * Hkv) {  // value copy
+        const size_t src = (size_t)row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
+        const size_t dst = cache_row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
+        *reinterpret_cast<uint4*>(Vc + dst) = __ldg(reinterpret_cast<const uint4*>(Vsrc + src));
+        *reinterpret_cast<uint4*>(Vc + dst + kHalf) =
+            __ldg(reinterpret_cast<const uint4*>(Vsrc + src + kHalf));
+        continue;
+      }
+      if (hh < Hkv) {
+        const size_t src = (size_t)row * Hkv * D + (size_t)hh * D + g * 8;
+        const size_t dst = cache_row * Hkv * D + (size_t)hh * D + g * 8;
+        const uint4 lo = __ldg(reinterpret_cast<const uint4*>(K + src));
+        const uint4 hi = __ldg(reinterpret_cast<const uint4*>(K + src + kHalf));
+        CosSin8 cs;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float2 v = cs_s[r][0][g * 8 + e];
+          cs.c[e] = v.x;
+          cs.s[e] = v.y;
+        }
+        uint4 olo, ohi;
+        rotate8<false>(lo, hi, cs, olo, ohi);
+        __nv_bfloat16* Kc = static_cast<__nv_bfloat16*>(Kout);
+        *reinterpret_cast<uint4*>(Kc + dst) = olo;
+        *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
+        rotate8<true>(lo, hi, cs, olo, ohi);
+        const size_t hdst = ((size_t)(seq * (q_off + L) + (row % L) + q_off) * Hkv + hh) * D + g * 8;
+        *reinterpret_cast<uint4*>(Kh + hdst) = olo;
+        *reinterpret_cast<uint4*>(Kh + hdst + kHalf) = ohi;
+        continue;
+      }
+      hh -= Hkv;  // queries follow keys and values
+    }
     const bool is_k = hh < Hkv;
     const int h = is_k ? hh : hh - Hkv;
     const size_t off = (size_t)row * (is_k ? Hkv : Hq) * D + (size_t)h * D + g * 8;
@@ -169,6 +212,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     uint4 olo, ohi;
     rotate8<true>(lo, hi, cs, olo, ohi);
     if (is_k) {
+      __half* Krot = static_cast<__half*>(Kout);
       *reinterpret_cast<uint4*>(Krot + off) = olo;
       *reinterpret_cast<uint4*>(Krot + off + kHalf) = ohi;
       continue;
@@ -184,7 +228,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     rotate8<true>(lo, hi, cs, olo, ohi);  // inter plane (c - 1)
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = olo;
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + kHalf) = ohi;
-    const int im = (int)((row % L) % s);
+    const int im = (int)(((row % L) + q_off) % s);
     if (query_pos_for_piece(kSucc, im, s, c) != c - 1) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -232,6 +276,26 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
       *reinterpret_cast<const uint4*>(v_new + src + D / 2);
 }
 
+// bf16 -> fp16 copy of cache rows 0 .. rows-1 (pitch Tcap) to rows of pitch
+// out_rows (exact inside the fp16 range), one 16-byte group per thread,
+// grid-stride.
+__global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restrict__ Kc,
+                                                          uint4* __restrict__ Kh, int rows,
+                                                          int Tcap, int out_rows,
+                                                          long long groups_per_row,
+                                                          long long total) {
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const long long r = gid / groups_per_row, g = gid % groups_per_row;
+    const long long seq = r / rows, row = r % rows;
+    uint4 w = __ldg(Kc + (seq * Tcap + row) * groups_per_row + g);
+    uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = pack_f16(bf16_lo(u[k]), bf16_hi(u[k]));
+    Kh[(seq * out_rows + row) * groups_per_row + g] = w;
+  }
+}
+
 }  // namespace rope_path
 
 
@@ -259,11 +323,31 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
   auto args = [&](auto kern) {
     kern<<<blocks, kRopeThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-        static_cast<__half*>(Qrot), static_cast<__half*>(Krot), B, L, Hq, Hkv, s, c,
-        log2((double)base));
+        static_cast<__half*>(Qrot), Krot, B, L, Hq, Hkv, s, c, log2((double)base), 0, L,
+        nullptr, nullptr, nullptr);
   };
-  if (D == 64) args(prefill_rope_kernel<64>);
-  else args(prefill_rope_kernel<128>);
+  if (D == 64) args(prefill_rope_kernel<64, false>);
+  else args(prefill_rope_kernel<128, false>);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
+                              void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
+                              int Hkv, int D, int t0, int Tcap, int s, int c, float base,
+                              cudaStream_t stream) {
+  using namespace rope_path;
+  const long long rows = (long long)B * Lq;
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((rows + kRopeRows - 1) / kRopeRows);
+  auto args = [&](auto kern) {
+    kern<<<blocks, kRopeThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+        static_cast<__half*>(Qrot), Kcache, B, Lq, Hq, Hkv, s, c, log2((double)base), t0, Tcap,
+        static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(Vcache),
+        static_cast<__half*>(Kf16));
+  };
+  if (D == 64) args(prefill_rope_kernel<64, true>);
+  else args(prefill_rope_kernel<128, true>);
   return cudaGetLastError();
 }
 
@@ -280,6 +364,22 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, voi
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), t, B, Hkv, D, Tcap, s,
       log2((double)base));
+  return cudaGetLastError();
+}
+}  // namespace dca
+
+namespace dca {
+cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
+                               int out_rows, int Hkv, int D, cudaStream_t stream) {
+  using namespace rope_path;
+  const long long gpr = (long long)Hkv * D / 8;
+  const long long total = (long long)B * rows * gpr;
+  if (total == 0) return cudaSuccess;
+  const long long want = (total + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+  keys_to_f16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(Kcache),
+                                                 static_cast<uint4*>(Kf16), rows, Tcap,
+                                                 out_rows, gpr, total);
   return cudaGetLastError();
 }
 }  // namespace dca

@@ -55,6 +55,10 @@ def test_workspace_queries(lib):
     # decode: one fp32 row + (max, sum) per (b, head, split of 1024 keys)
     assert dca.dca_attn_decode_workspace(16, 64, 128, 65536) == 16 * 64 * 64 * 130 * 4
     assert dca.dca_attn_decode_workspace(2, 8, 64, 1025) == 2 * 8 * 2 * 66 * 4
+    # chunked prefill: three fp16 query rotations of the chunk + fp16 keys 0 .. t0+Lq-1
+    assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, 50) == (
+        up(3 * 2 * 100 * 8 * 128 * 2) + up(2 * 150 * 2 * 128 * 2))
+    assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, -1) == 0
 
 
 def test_prefill_path_selection(lib):
@@ -113,6 +117,15 @@ def test_argument_errors_return_codes(lib):
                                      0.0, ws, 1 << 30, None)) == 1
     assert _code(lib.dca_attn_decode(*dargs, fake, fake, fake, 2, 8, 1, 128, 64, 16, 32, 1e4,
                                      0.0, ws, 8, None)) == 5
+    # chunked prefill: chunk past the cache end, negative t0, short workspace
+    cargs = (fake,) * 7
+    assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, 100, 128, 16, 32, 1e4,
+                                            0.0, ws, 1 << 30, None)) == 1
+    assert "outside cache" in dca.dca_last_error_string()
+    assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, -1, 128, 16, 32, 1e4,
+                                            0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, 64, 128, 16, 32, 1e4,
+                                            0.0, ws, 64, None)) == 5
     # wait self-test: deadline out of range
     assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
     assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1

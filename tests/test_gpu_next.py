@@ -60,6 +60,7 @@ def test_cache_built_by_append_decodes_like_prefill():
     Vc = torch.zeros_like(Kc)
     Kd, Vd = K.cuda(), V.cuda()
     checkpoints = {0, 255, 256, 383, 384, 511, 512, 699}
+    model = _model_cache(K, s, L)
     for tt in range(L):
         t = torch.tensor([tt], dtype=torch.int32, device="cuda")
         dca.dca_kv_append(Kd[:, tt].contiguous(), Vd[:, tt].contiguous(), Kc, Vc, t, s, c)
@@ -68,12 +69,12 @@ def test_cache_built_by_append_decodes_like_prefill():
             dca.dca_sync_status()
             assert (O_d.cpu().float() - O_p[:, tt].cpu().float()).abs().max() < 2e-2, tt
             assert (LSE_d.cpu() - LSE_p[:, :, tt].cpu()).abs().max() < 2e-3, tt
-            ref = orc.dca_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), s, c,
-                                       rows=[tt])
-            o_ref = np.stack([ref[(0, h, tt)][0] for h in range(Hq)])
-            l_ref = np.array([ref[(0, h, tt)][1] for h in range(Hq)])
-            err = np.abs(O_d[0].cpu().double().numpy() - o_ref)
-            lse_rel = np.abs(LSE_d[0].cpu().double().numpy() - l_ref) / np.maximum(
+            # oracle over the cache as stored: bf16 roundings of the oracle's
+            # own rotation of keys 0 .. tt
+            o_ref, l_ref = orc.dca_decode(Q[:, tt].double().numpy(), model, V.double().numpy(),
+                                          np.array([tt]), s, c)
+            err = np.abs(O_d.cpu().double().numpy() - o_ref)
+            lse_rel = np.abs(LSE_d.cpu().double().numpy() - l_ref) / np.maximum(
                 np.abs(l_ref), 1.0)
             pu.assert_close(err.max(), err.mean(), lse_rel.max(), f"append+decode t={tt}")
     # the appended cache equals the library's own RoPE of the whole K at j mod s
@@ -107,3 +108,190 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     dca.dca_sync_status()
     want = orc.index_map(12, 4, 6)
     assert (qpos.cpu().numpy() == want[0]).all() and (piece.cpu().numpy() == want[2]).all()
+
+
+# ---------------------------------------------------------------------------
+# three single-piece flash passes merged by LSE
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [(1, 1024, 1, 1, 64, 192, 256), (2, 300, 4, 2, 128, 64, 96),
+                                  (1, 777, 2, 1, 64, 100, 150), (1, 900, 2, 2, 128, 256, 384),
+                                  (1, 5, 2, 1, 128, 2, 3)], ids=str)
+def test_three_pass_matches_oracle_and_one_pass(case):
+    B, L, Hq, Hkv, D, s, c = case
+    Q, K, V = W.make_prefill_inputs(dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=L + 3)
+    O3, L3 = dca.dca_attn_prefill_3pass(Q.cuda(), K.cuda(), V.cuda(), s, c)
+    O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), s, c)
+    dca.dca_sync_status()
+    O_ref, LSE_ref = orc.dca_prefill(Q.float().numpy(), K.float().numpy(), V.float().numpy(), s, c)
+    err = np.abs(O3.cpu().double().numpy() - O_ref)
+    lse_rel = np.abs(L3.cpu().double().numpy() - LSE_ref) / np.maximum(np.abs(LSE_ref), 1.0)
+    print(f"3-pass {case}: O max {err.max():.3e} mean {err.mean():.3e} LSE rel {lse_rel.max():.3e}")
+    pu.assert_close(err.max(), err.mean(), lse_rel.max(), f"3-pass {case}")
+    assert (O3.float() - O1.float()).abs().max().item() < 2e-2
+    assert (L3 - L1).abs().max().item() < 1e-3
+
+
+def test_three_pass_workload_sampled():
+    cfg = W.CONFIGS["llama2_7b_16k"]
+    Q, K, V = W.make_prefill_inputs(cfg)
+    O3, L3 = dca.dca_attn_prefill_3pass(Q.cuda(), K.cuda(), V.cuda(), cfg["s"], cfg["c"])
+    O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), cfg["s"], cfg["c"])
+    dca.dca_sync_status()
+    d = (O3.float() - O1.float()).abs()
+    print(f"3-pass vs fused (7B): O max {d.max():.3e} mean {d.mean():.3e} "
+          f"LSE max {(L3 - L1).abs().max():.3e}")
+    assert d.max() < 2e-2 and d.mean() < 1e-3 and (L3 - L1).abs().max() < 1e-3
+    rows = pu.sample_rows(cfg["L"], cfg["s"], cfg["c"], n_random=64)
+    ref = orc.dca_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), cfg["s"], cfg["c"],
+                               rows=rows, heads=[0, 31])
+    mx, mean, lse = pu.compare_rows(O3.cpu(), L3.cpu(), ref)
+    pu.assert_close(mx, mean, lse, "3-pass 7B")
+
+
+# ---------------------------------------------------------------------------
+# chunked prefill against an existing cache (query offset t0 > 0)
+#
+# The oracle takes the cached keys 0 .. t0-1 as stored: bf16 roundings of the
+# keys rotated at j mod s, which the tests form from the oracle's own fp64
+# rotation (never from the library's cache).
+# ---------------------------------------------------------------------------
+
+def _model_cache(K, s, t0, kv_heads=None, base=10000.0):
+    """bf16-rounded keys 0 .. t0-1 rotated at j mod s by the oracle (fp64 numpy)."""
+    B, _, Hkv, D = K.shape
+    out = np.zeros((B, t0, Hkv, D))
+    for hk in (range(Hkv) if kv_heads is None else kv_heads):
+        rot = orc.rotate(K[:, :t0, hk].double().numpy(),
+                         orc.key_position(np.arange(t0), s)[None, :], base)
+        out[:, :, hk] = torch.from_numpy(rot).to(torch.bfloat16).double().numpy()
+    return out
+
+
+def _check_chunk(O, LSE, ref, what):
+    mx, mean, lse = pu.compare_rows(O.cpu(), LSE.cpu(), ref)
+    print(f"{what}: O max {mx:.3e} mean {mean:.3e} LSE rel {lse:.3e}")
+    pu.assert_close(mx, mean, lse, what)
+
+
+CHUNK_CASES = [
+    # B, L, Hq, Hkv, D, s, c, chunk bounds (ragged, off tile and chunk edges)
+    (1, 700, 8, 2, 128, 256, 384, [0, 1, 63, 200, 256, 257, 511, 640, 700]),
+    (2, 450, 4, 4, 64, 64, 96, [0, 100, 129, 330, 450]),
+    (1, 333, 2, 1, 128, 40, 50, [0, 37, 38, 333]),
+    (1, 260, 4, 1, 64, 3, 5, [0, 1, 2, 3, 100, 260]),
+    # D 128, s % 256 == 0, chunk starts % 256 == 0: the tcgen05 kernel with offset
+    (2, 1100, 8, 2, 128, 512, 640, [0, 256, 768, 1024, 1100]),
+    (1, 1300, 4, 4, 128, 256, 300, [0, 512, 513, 1024, 1300]),
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_CASES,
+                         ids=lambda c: f"B{c[0]}L{c[1]}H{c[2]}/{c[3]}D{c[4]}s{c[5]}c{c[6]}")
+def test_chunked_prefill_matches_oracle(case):
+    B, L, Hq, Hkv, D, s, c, bounds = case
+    Tcap = L + 37
+    Q, K, V = W.make_prefill_inputs(dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=L + 9)
+    Kc = torch.full((B, Tcap, Hkv, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.full_like(Kc, -3.0)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    model = _model_cache(K, s, L)
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        O, LSE = dca.dca_attn_prefill_chunk(Qd[:, a:e].contiguous(), Kd[:, a:e].contiguous(),
+                                            Vd[:, a:e].contiguous(), Kc, Vc, a, s, c)
+        dca.dca_sync_status()
+        ref = orc.dca_prefill_chunk(pu.F64View(Q[:, a:e]), pu.F64View(K[:, a:e]),
+                                    pu.F64View(V[:, a:e]), model[:, :a], pu.F64View(V[:, :a]),
+                                    a, s, c)
+        _check_chunk(O, LSE, ref, f"chunk [{a}, {e}) of {case[:7]}")
+    # the cache holds exactly the library's key rotation and the values; rows
+    # past the sequence are untouched
+    Kr = dca.dca_rope_rotate(Kd, dca.DCA_POS_KEY, s, c)
+    assert torch.equal(Kc[:, :L], Kr) and torch.equal(Vc[:, :L].cpu(), V)
+    assert Kc[:, L:].float().eq(7).all() and Vc[:, L:].float().eq(-3).all()
+    # and the library's bf16 rotation is the oracle's rounded one but for rare
+    # rounding-boundary ties
+    diff = (Kr.cpu().double().numpy() != model)
+    assert diff.mean() < 1e-3
+
+
+@pytest.mark.parametrize("D,s,c,t0", [(128, 256, 384, 300), (128, 512, 640, 512),
+                                      (64, 48, 64, 97)], ids=str)
+def test_chunk_over_host_written_cache(D, s, c, t0):
+    # the cache prefix comes from the oracle's model (not from the library)
+    B, L, Hq, Hkv = 2, t0 + 200, 8, 2
+    Q, K, V = W.make_prefill_inputs(dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=t0)
+    model = _model_cache(K, s, t0)
+    Kc = torch.zeros(B, L + 5, Hkv, D, dtype=torch.bfloat16)
+    Vc = torch.zeros_like(Kc)
+    Kc[:, :t0] = torch.from_numpy(model).to(torch.bfloat16)
+    Vc[:, :t0] = V[:, :t0]
+    Kc, Vc = Kc.cuda(), Vc.cuda()
+    O, LSE = dca.dca_attn_prefill_chunk(Q[:, t0:].contiguous().cuda(),
+                                        K[:, t0:].contiguous().cuda(),
+                                        V[:, t0:].contiguous().cuda(), Kc, Vc, t0, s, c)
+    dca.dca_sync_status()
+    ref = orc.dca_prefill_chunk(pu.F64View(Q[:, t0:]), pu.F64View(K[:, t0:]),
+                                pu.F64View(V[:, t0:]), model, pu.F64View(V[:, :t0]), t0, s, c)
+    _check_chunk(O, LSE, ref, f"host cache D{D} s{s} c{c} t0={t0}")
+    assert torch.equal(Kc[:, :t0].cpu(), torch.from_numpy(model).to(torch.bfloat16))
+
+
+def test_chunked_prefill_then_decode_continues_the_sequence():
+    # serving flow: prefill 600 rows in two chunks, then append + decode 100
+    L, Lp, Hq, Hkv, D, s, c = 700, 600, 8, 2, 128, 256, 384
+    Q, K, V = W.make_prefill_inputs(dict(B=1, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=5)
+    Kc = torch.zeros(1, L, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.zeros_like(Kc)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    for a, e in [(0, 317), (317, Lp)]:
+        dca.dca_attn_prefill_chunk(Qd[:, a:e].contiguous(), Kd[:, a:e].contiguous(),
+                                   Vd[:, a:e].contiguous(), Kc, Vc, a, s, c)
+    rows = [Lp, Lp + 1, 639, 640, 641, 699]
+    got = {}
+    for tt in range(Lp, L):
+        t = torch.tensor([tt], dtype=torch.int32, device="cuda")
+        dca.dca_kv_append(Kd[:, tt].contiguous(), Vd[:, tt].contiguous(), Kc, Vc, t, s, c)
+        if tt in rows:
+            got[tt] = dca.dca_attn_decode(Qd[:, tt].contiguous(), Kc, Vc, t, s, c)
+    dca.dca_sync_status()
+    model = _model_cache(K, s, L)
+    for tt in rows:
+        O_ref, L_ref = orc.dca_decode(Q[:, tt].double().numpy(), model, V.double().numpy(),
+                                      np.array([tt]), s, c)
+        err = np.abs(got[tt][0].cpu().double().numpy() - O_ref)
+        lse_rel = np.abs(got[tt][1].cpu().double().numpy() - L_ref) / np.maximum(
+            np.abs(L_ref), 1.0)
+        pu.assert_close(err.max(), err.mean(), lse_rel.max(), f"decode after chunks t={tt}")
+
+
+def test_chunked_prefill_workload_sampled():
+    # the 16k-token 7B workload prefilled in four 4096-row chunks (tcgen05 path)
+    cfg = W.CONFIGS["llama2_7b_16k"]
+    B, L, Hq, Hkv, s, c = cfg["B"], cfg["L"], cfg["Hq"], cfg["Hkv"], cfg["s"], cfg["c"]
+    Q, K, V = W.make_prefill_inputs(cfg)
+    bounds = [0, 4096, 8192, 12288, L]
+    Kc = torch.empty(B, L, Hkv, cfg["D"], dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    outs = []
+    for a, e in zip(bounds[:-1], bounds[1:]):
+        outs.append(dca.dca_attn_prefill_chunk(Qd[:, a:e].contiguous(), Kd[:, a:e].contiguous(),
+                                               Vd[:, a:e].contiguous(), Kc, Vc, a, s, c))
+    O1, L1 = dca.dca_attn_prefill(Qd, Kd, Vd, s, c)
+    dca.dca_sync_status()
+    O = torch.cat([o for o, _ in outs], 1)
+    LSE = torch.cat([l for _, l in outs], 2)
+    d = (O.float() - O1.float()).abs()
+    print(f"chunked vs one-shot (7B): O max {d.max():.3e} mean {d.mean():.3e} "
+          f"LSE max {(LSE - L1).abs().max():.3e}")
+    assert d.max() < 2e-2 and d.mean() < 1e-3
+    heads = [0, Hq - 1]
+    model = _model_cache(K, s, L, kv_heads=sorted({orc.kv_head(h, Hq, Hkv) for h in heads}))
+    sample = set(pu.sample_rows(L, s, c, n_random=32)) | {4095, 4096, 8191, 8192, 12288}
+    for k, (a, e) in enumerate(zip(bounds[:-1], bounds[1:])):
+        rows = sorted(r - a for r in sample if a <= r < e)
+        ref = orc.dca_prefill_chunk(pu.F64View(Q[:, a:e]), pu.F64View(K[:, a:e]),
+                                    pu.F64View(V[:, a:e]), model[:, :a], pu.F64View(V[:, :a]),
+                                    a, s, c, rows=rows, heads=heads)
+        _check_chunk(outs[k][0], outs[k][1], ref, f"7B chunk [{a}, {e})")
