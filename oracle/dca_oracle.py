@@ -27,6 +27,11 @@ fusion or reordering:
   and all causal keys j <= i share one softmax.
 * Attention: z_j = scale * <R(p_q) q_i, R(p_k) k_j>,  m = max z,
   l = sum exp(z - m),  O_i = sum exp(z_j - m) v_j / l,  LSE_i = m + ln l.
+* Chunked prefill (dca_prefill_chunk): rows t0 .. t0+Lq-1 of the same
+  definition with keys 0 .. t0-1 read, already rotated, from a cache.
+* SelfExtend (prior art; LLM Maybe LongLM: Self-Extend LLM Context Window
+  Without Tuning, abstract): neighbour pairs (i - j < W) at positions (i, j),
+  grouped pairs at (floor(i/G) + W - floor(W/G), floor(j/G)), one softmax.
 
 Inputs are bf16 values upcast exactly to float64 (any float array works).
 Every function is fp64 end to end; nothing is rounded to bf16.
@@ -34,7 +39,9 @@ Every function is fp64 end to end; nothing is rounded to bf16.
 Pins that hold this module to something other than itself live in
 ``tests/test_oracle_pins.py`` (worked index table, closed-form piece counts,
 reduction to plain RoPE attention, Q = 0 and constant-V closed forms, RoPE
-relativity, decode = prefill row) and ``tests/test_oracle_mutations.py``
+relativity, decode = prefill row, chunk = whole-sequence rows, hand-worked
+SelfExtend distance tables and its reductions to plain RoPE attention) and
+``tests/test_oracle_mutations.py``
 (plausible mistakes planted here must each fail a pin).
 """
 
@@ -369,3 +376,65 @@ def merge_partials(o_parts, lse_parts):
     wts = np.exp(lse_parts - m)
     tot = np.sum(wts)
     return (wts @ np.asarray(o_parts, np.float64)) / tot, m + np.log(tot)
+
+
+# ---------------------------------------------------------------------------
+# SelfExtend (prior art: "LLM Maybe LongLM: Self-Extend LLM Context Window
+# Without Tuning", abstract): bi-level attention over the original model's
+# RoPE attention.  Neighbour attention keeps the original positions for keys
+# within a window of W tokens; grouped attention maps far keys and the query to
+# floor-divided positions (group size G).  The abstract leaves the join of the
+# two levels open; the reading taken here shifts the grouped query position by
+# W - floor(W / G), so a grouped pair is never closer than W (the neighbour
+# distances are 0 .. W-1) and one softmax spans both levels.
+# ---------------------------------------------------------------------------
+
+def selfextend_positions(i, j, G: int, W: int):
+    """(query position, key position) of query i meeting key j (j <= i).
+
+    Neighbour (i - j < W): (i, j).  Grouped (i - j >= W):
+    (floor(i / G) + W - floor(W / G), floor(j / G)).
+    """
+    if G < 1 or W < 1:
+        raise ValueError(f"SelfExtend needs G >= 1 and W >= 1, got G={G}, W={W}")
+    i = np.asarray(i, np.int64)
+    j = np.asarray(j, np.int64)
+    near = (i - j) < W
+    qpos = np.where(near, i, i // G + W - W // G)
+    kpos = np.where(near, j, j // G)
+    return qpos, kpos
+
+
+def selfextend_row(q, k, v, i: int, G: int, W: int, base: float, scale: float):
+    """One query row: q [D] unrotated at index i; k, v [i+1, D] unrotated keys
+    0..i and values.  Each (query, key) pair is rotated at its own positions."""
+    j = np.arange(i + 1, dtype=np.int64)
+    qpos, kpos = selfextend_positions(i, j, G, W)
+    k_rot = rotate(k, kpos, base)
+    z = np.empty(i + 1, dtype=np.float64)
+    for p in np.unique(qpos):
+        sel = qpos == p
+        z[sel] = k_rot[sel] @ rotate(q, p, base)
+    return softmax_row(scale * z, v)
+
+
+def selfextend_prefill_rows(Q, K, V, G: int, W: int, base: float = 10000.0,
+                            scale: float = 0.0, rows=None, heads=None, batches=None):
+    """SelfExtend prefill on selected (batch, head, row) outputs; Q [B, L, Hq, D],
+    K, V [B, L, Hkv, D] unrotated.  Returns {(b, h, i): (O, LSE)}."""
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    sc = _scale(D, scale)
+    rows = range(L) if rows is None else rows
+    heads = range(Hq) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    out = {}
+    for b in batches:
+        for h in heads:
+            hk = kv_head(h, Hq, Hkv)
+            for i in sorted(int(r) for r in rows):
+                k = np.asarray(K[b, :i + 1, hk, :], np.float64)
+                v = np.asarray(V[b, :i + 1, hk, :], np.float64)
+                q = np.asarray(Q[b, i, h, :], np.float64)
+                out[(b, h, i)] = selfextend_row(q, k, v, i, G, W, base, sc)
+    return out

@@ -121,6 +121,27 @@ def _decode_short(q, k_cache_rot, v_cache, t, s, c, base=10000.0, scale=0.0,
 
 _ORIG_DECODE = orc.dca_decode
 _ORIG_CHUNK = orc.dca_prefill_chunk
+_ORIG_SE_POS = orc.selfextend_positions
+
+
+def _se_no_shift(i, j, G, W):
+    # grouped query at floor(i/G) without the W - floor(W/G) shift
+    q, k = _ORIG_SE_POS(i, j, G, W)
+    far = (np.asarray(i) - np.asarray(j)) >= W
+    return np.where(far, np.asarray(i) // G, q), k
+
+
+def _se_window_le(i, j, G, W):
+    # neighbour window one too wide (i - j <= W)
+    q, k = _ORIG_SE_POS(i, j, G, W)
+    at = (np.asarray(i) - np.asarray(j)) == W
+    return np.where(at, np.asarray(i), q), np.where(at, np.asarray(j), k)
+
+
+def _se_key_not_grouped(i, j, G, W):
+    q, k = _ORIG_SE_POS(i, j, G, W)
+    far = (np.asarray(i) - np.asarray(j)) >= W
+    return q, np.where(far, np.asarray(j), k)
 
 
 def _chunk_ignores_cache(Qc, Kc, Vc, k_cache_rot, v_cache, t0, s, c, *args, **kw):
@@ -151,6 +172,9 @@ MUTANTS = {
     "decode_short": ("dca_decode", _decode_short),
     "chunk_ignores_cache": ("dca_prefill_chunk", _chunk_ignores_cache),
     "chunk_start_early": ("dca_prefill_chunk", _chunk_start_early),
+    "selfextend_no_shift": ("selfextend_positions", _se_no_shift),
+    "selfextend_window_le": ("selfextend_positions", _se_window_le),
+    "selfextend_key_not_grouped": ("selfextend_positions", _se_key_not_grouped),
 }
 
 

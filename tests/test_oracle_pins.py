@@ -16,7 +16,12 @@ them against the oracle as committed.  Sources of each fact:
   rotation done by complex multiplication;
 * closed forms for Q = 0 and constant V, RoPE relativity (Guide, "The
   Problem": the score depends only on the position difference), literal
-  rotation values, and the split-softmax identity.
+  rotation values, and the split-softmax identity;
+* a chunk at t0 over a cache of the earlier keys equals the whole-sequence
+  rows (the rule depends only on absolute indices);
+* SelfExtend (LLM Maybe LongLM, abstract): hand-worked neighbour / grouped
+  distance tables under ``tests/golden/``, its reduction to plain RoPE
+  attention for G = 1 or W >= L (torch SDPA), and distance bounds.
 """
 
 import math
@@ -33,7 +38,11 @@ TABLES = [("dca_index_s4_c6_L12.txt", 4, 6), ("dca_index_s3_c5_L9.txt", 3, 5),
           ("dca_index_s3_c3_L7.txt", 3, 3), ("dca_index_s2_c5_L7.txt", 2, 5)]
 
 
-def parse_table(name):
+SE_TABLES = [("selfextend_G2_W3_L10.txt", 2, 3), ("selfextend_G3_W4_L12.txt", 3, 4)]
+
+
+def parse_table(name, letters=None):
+    letters = letters or {"A": 0, "S": 1, "I": 2}
     lines = [ln for ln in (GOLDEN / name).read_text().splitlines()
              if ln.strip() and not ln.startswith("#")]
     rows = lines[1:]
@@ -47,7 +56,7 @@ def parse_table(name):
         for j, tok in enumerate(toks[1:]):
             if tok == ".":
                 continue
-            pc[r, j] = {"A": 0, "S": 1, "I": 2}[tok[0]]
+            pc[r, j] = letters[tok[0]]
             dist[r, j] = int(tok[1:])
     return pc, dist
 
@@ -289,12 +298,57 @@ def pin_rule_positions():
         assert qpos[r, (r // s - 1) * s] == succ[r]
 
 
+def pin_selfextend_worked_tables():
+    # hand-worked neighbour / grouped distance tables
+    for name, G, W in SE_TABLES:
+        want_lv, want_d = parse_table(name, {"N": 0, "G": 1})
+        L = want_lv.shape[0]
+        for i in range(L):
+            j = np.arange(i + 1)
+            qpos, kpos = orc.selfextend_positions(i, j, G, W)
+            assert (qpos - kpos == want_d[i, :i + 1]).all(), (name, i)
+            grouped = (i - j) >= W
+            assert (grouped.astype(np.int8) == want_lv[i, :i + 1]).all(), (name, i)
+            # neighbours keep the original absolute positions
+            assert (qpos[~grouped] == i).all() and (kpos[~grouped] == j[~grouped]).all()
+
+
+def pin_selfextend_reduces_to_plain_rope():
+    # G = 1 (no grouping) and W >= L (every key a neighbour) are plain RoPE
+    # attention, checked against torch SDPA over complex-rotated inputs
+    Q, K, V = _rand((1, 17, 4, 8), 50), _rand((1, 17, 2, 8), 51), _rand((1, 17, 2, 8), 52)
+    O_ref, LSE_ref = _sdpa_reference(Q, K, V, 100.0)
+    for G, W in [(1, 1), (1, 5), (4, 17), (3, 40)]:
+        got = orc.selfextend_prefill_rows(Q, K, V, G, W, base=100.0)
+        for (b, h, i), (o, lse) in got.items():
+            np.testing.assert_allclose(o, O_ref[b, i, h], atol=1e-12)
+            np.testing.assert_allclose(lse, LSE_ref[b, h, i], atol=1e-12)
+    # with grouping active beyond W the result must differ from plain RoPE
+    got = orc.selfextend_prefill_rows(Q, K, V, 2, 3, base=2.0, rows=[16])
+    O2, _ = _sdpa_reference(Q, K, V, 2.0)
+    assert np.abs(got[(0, 0, 16)][0] - O2[0, 16, 0]).max() > 1e-3
+
+
+def pin_selfextend_distance_bounds():
+    # grouped pairs are never closer than the window; the largest distance is
+    # floor((L-1)/G) + W - floor(W/G); distances never decrease as j moves away
+    for G, W, L in [(2, 3, 40), (4, 16, 200), (8, 5, 120), (3, 1, 50)]:
+        for i in range(L):
+            j = np.arange(i + 1)
+            qpos, kpos = orc.selfextend_positions(i, j, G, W)
+            d = qpos - kpos
+            assert (d[(i - j) >= W] >= W).all()
+            assert d.max() <= (L - 1) // G + W - W // G
+            assert (np.diff(d[::-1]) >= 0).all()
+
+
 PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_rotation_literals, pin_rope_relativity, pin_plain_rope_matches_sdpa,
         pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
         pin_q_zero_closed_form, pin_constant_v, pin_gqa_mapping,
         pin_decode_equals_prefill_row, pin_chunk_equals_prefill_rows, pin_merge_partials,
-        pin_rule_positions]
+        pin_rule_positions, pin_selfextend_worked_tables, pin_selfextend_reduces_to_plain_rope,
+        pin_selfextend_distance_bounds]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
