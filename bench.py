@@ -420,6 +420,8 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                      (dca_attn_prefill_chunk, chunk starts 0, L/4, L/2, 3L/4);
       prefill_3pass  the prefill workload as three single-piece passes merged
                      by LSE (dca_attn_prefill_3pass);
+      prefill_selfextend  the prefill workload under the SelfExtend position
+                     map, G = 8, W = 1024 (dca_attn_prefill_selfextend);
       kv_append      one decoded token appended per sequence of the decode
                      batch (dca_kv_append), 100 calls back to back."""
     import ctypes
@@ -493,6 +495,27 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
     out["prefill_3pass"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
                             "path": "general (warp MMA) x3 + merge", "launches_per_call": 5}
     del pws, O3, L3
+
+    # SelfExtend position map on the general kernel (group 8, window 1024)
+    G_se, W_se = 8, 1024
+    wsz = dca.dca_selfextend_workspace(B, L, Hq, Hkv, D)
+    sws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    Ose = torch.empty_like(Q)
+    Lse = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+
+    def selfextend():
+        st = lib.dca_attn_prefill_selfextend(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
+                                             P(Ose.data_ptr()), P(Lse.data_ptr()), B, L, Hq, Hkv,
+                                             D, G_se, W_se, base, 0.0, P(sws.data_ptr()), wsz,
+                                             P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(selfextend)
+    out["prefill_selfextend"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                 "ms": ms, "G": G_se, "W": W_se,
+                                 "path": "RoPE (2 planes) + general (warp MMA)",
+                                 "launches_per_call": 2}
+    del sws, Ose, Lse
 
     # decode-time append of one token per sequence (positions t_dec + 1 < Tcap)
     Bd, Tcap, Hkvd, Dd = Kc.shape

@@ -174,6 +174,31 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
                                     int Hkv, int D, int t0, int Tcap, int s, int c, float base,
                                     float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/* Workspace bytes for dca_attn_prefill_selfextend: the neighbour and grouped
+ * rotations of Q [2][B][L][Hq][D] and K [2][B][L][Hkv][D], fp16, each rounded
+ * up to 256 bytes.  Returns 0 for unsupported arguments. */
+size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D);
+
+/* SelfExtend prefill: the prior-art bi-level position map ("LLM Maybe LongLM:
+ * Self-Extend LLM Context Window Without Tuning", abstract: grouped attention
+ * for tokens far apart, neighbour attention for tokens within a range) on the
+ * same tiled online-softmax kernel as DCA.  For a causal pair (i, j):
+ *   i - j <  W  (neighbour): query rotated at i, key at j;
+ *   i - j >= W  (grouped):   query at floor(i/G) + W - floor(W/G), key at
+ *                            floor(j/G);
+ * one softmax over all keys 0 .. i.  The abstract leaves the join of the two
+ * levels open; the shift W - floor(W/G) is the reading that keeps every
+ * grouped distance >= W, above all neighbour distances.  G = 1 or W >= L is
+ * plain RoPE attention.  Same tensors and conventions as dca_attn_prefill
+ * (Q, K unrotated bf16; O bf16; LSE fp32 [B][Hq][L]); any G >= 1, W >= 1,
+ * D in {64, 128}; warp-MMA kernel.  `workspace`: dca_selfextend_workspace
+ * bytes, 256-byte aligned, scratch for the call.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const void* V, void* O,
+                                         float* LSE, int B, int L, int Hq, int Hkv, int D, int G,
+                                         int W, float base, float scale, void* workspace,
+                                         size_t ws_bytes, void* stream);
+
 /* Which prefill path DCA_PATH_AUTO takes for these sizes (1 general,
  * 2 tcgen05), or 0 for unsupported arguments. */
 int dca_prefill_path(int L, int D, int s, int c);

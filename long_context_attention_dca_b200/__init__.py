@@ -25,6 +25,7 @@ __all__ = [
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
     "dca_attn_prefill_3pass_workspace", "dca_attn_prefill_3pass",
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
+    "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
     "dca_debug_index_map", "dca_debug_wait_timeout",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
@@ -49,6 +50,9 @@ _SIGS = {
     "dca_prefill_path": (_I, [_I, _I, _I, _I]),
     "dca_attn_prefill_3pass_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "dca_selfextend_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_attn_prefill_selfextend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F,
+                                         _P, _Z, _P]),
     "dca_attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                                     _I, _F, _F, _P, _Z, _P]),
     "dca_attn_prefill_3pass": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P,
@@ -243,6 +247,26 @@ def dca_attn_prefill_chunk(Q, K, V, Kcache, Vcache, t0, s, c, base=10000.0, scal
     _check(lib().dca_attn_prefill_chunk(_ptr(Q), _ptr(K), _ptr(V), _ptr(Kcache), _ptr(Vcache),
                                         _ptr(O), _ptr(LSE), B, Lq, Hq, Hkv, D, int(t0), Tcap, s,
                                         c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_selfextend_workspace(B: int, L: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().dca_selfextend_workspace(B, L, Hq, Hkv, D))
+
+
+def dca_attn_prefill_selfextend(Q, K, V, G, W, base=10000.0, scale=0.0):
+    """SelfExtend prefill (neighbour window W, group size G) -> (O, LSE)."""
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    ws = _workspace(dca_selfextend_workspace(B, L, Hq, Hkv, D), Q.device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
+    _check(lib().dca_attn_prefill_selfextend(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L,
+                                             Hq, Hkv, D, int(G), int(W), base, scale, _ptr(ws),
+                                             ws.numel(), _stream(Q)))
     return O, LSE
 
 

@@ -59,21 +59,65 @@ __device__ __forceinline__ void compute_s(float (&acc)[8][4], uint32_t q_base, u
   }
 }
 
+// Position rules of the general kernel.  A rule names the pieces a causal
+// (query i, key j) pair can fall in, the query and key planes a piece reads,
+// the pieces a warp's 16 rows can meet in a key tile, and the piece of one
+// pair (from a per-row key computed once).
+struct DcaRule {
+  // pieces 0 intra, 1 successive, 2 inter: query planes 0..2, one key plane
+  // (keys at j mod s)
+  static constexpr int kPieces = 3, kQPlanes = 3, kKPlanes = 1;
+  static constexpr bool kDca = true;
+  int s;
+  __device__ __forceinline__ int kplane(int) const { return 0; }
+  __device__ __forceinline__ void meets(int r0, int k0, bool (&pr)[3]) const {
+    // chunk differences of the tile's pairs form an interval; causal >= 0
+    const int ci_lo = r0 / s, ci_hi = (r0 + 15) / s;
+    const int cj_lo = k0 / s, cj_hi = (k0 + kBN - 1) / s;
+    const int dmin = max(ci_lo - cj_hi, 0), dmax = ci_hi - cj_lo;
+    pr[0] = dmin == 0;
+    pr[1] = dmin <= 1 && dmax >= 1;
+    pr[2] = dmax >= 2;
+  }
+  __device__ __forceinline__ int row_key(int i) const { return i / s; }
+  __device__ __forceinline__ int piece(int rk, int j) const {
+    const int d = rk - j / s;
+    return d <= 0 ? 0 : (d == 1 ? 1 : 2);
+  }
+};
+
+struct SelfExtendRule {
+  // pieces 0 neighbour (i - j < W), 1 grouped: query plane p with key plane p
+  static constexpr int kPieces = 2, kQPlanes = 2, kKPlanes = 2;
+  static constexpr bool kDca = false;
+  int W;
+  __device__ __forceinline__ int kplane(int p) const { return p; }
+  __device__ __forceinline__ void meets(int r0, int k0, bool (&pr)[3]) const {
+    // distances i - j in the tile span [r0 - k0 - (kBN - 1), r0 + 15 - k0]
+    pr[0] = max(r0 - k0 - (kBN - 1), 0) < W;
+    pr[1] = r0 + 15 - k0 >= W;
+    pr[2] = false;
+  }
+  __device__ __forceinline__ int row_key(int i) const { return i; }
+  __device__ __forceinline__ int piece(int rk, int j) const { return rk - j < W ? 0 : 1; }
+};
+
 // Query row r of this launch has absolute index q_off + r (0 for a whole-
 // sequence prefill; the chunk start for chunked prefill against a cache).
 // Keys 0 .. Lkv-1 are read from fp16 K and bf16 V rows of pitch k_rows and
 // v_rows per sequence.
-template <int D>
+template <int D, class Rule>
 __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
     const __half* __restrict__ Qrot, const __half* __restrict__ Krot,
     const __nv_bfloat16* __restrict__ V, __nv_bfloat16* __restrict__ O, float* __restrict__ LSE,
-    int B, int L, int Hq, int Hkv, int s, int c, float scale_log2, int piece_mask,
+    int B, int L, int Hq, int Hkv, Rule rule, float scale_log2, int piece_mask,
     float* __restrict__ Of32, int q_off, int k_rows, int v_rows, int Lkv) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
+  constexpr int kNQ = Rule::kQPlanes, kNK = Rule::kKPlanes;
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK = sQ + 3 * kBM * D * 2;
-  const uint32_t sV = sK + 2 * kBN * D * 2;
+  const uint32_t sK = sQ + kNQ * kBM * D * 2;        // [stage][key plane] tiles
+  const uint32_t sV = sK + 2 * kNK * kBN * D * 2;    // [stage] tiles
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_qt = (L + kBM - 1) / kBM;
@@ -83,8 +127,8 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
   const int q0 = qt * kBM;
   const size_t plane = (size_t)B * L * Hq * D;
 
-  // Query tile, all three rotations.
-  for (int idx = tid; idx < 3 * kBM * CH; idx += kThreads) {
+  // Query tile, every rotation the rule uses.
+  for (int idx = tid; idx < kNQ * kBM * CH; idx += kThreads) {
     const int v = idx / (kBM * CH), r = (idx / CH) % kBM, ch = idx % CH;
     const int row = q0 + r;
     const bool ok = row < L;
@@ -92,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
         Qrot + v * plane + (((size_t)b * L + (ok ? row : 0)) * Hq + h) * D + ch * 8;
     cp_async_16(sQ + v * kBM * D * 2 + swz<D>(r, ch), src, ok);
   }
+  const size_t k_plane = (size_t)B * k_rows * Hkv * D;
   auto load_kv = [&](int stage, int kt) {
     for (int idx = tid; idx < kBN * CH; idx += kThreads) {
       const int r = idx / CH, ch = idx % CH;
@@ -99,8 +144,10 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
       const bool ok = row < Lkv;
       const size_t col = (size_t)hk * D + ch * 8;
       const size_t rr = ok ? row : 0;
-      cp_async_16(sK + stage * kBN * D * 2 + swz<D>(r, ch),
-                  Krot + ((size_t)b * k_rows + rr) * Hkv * D + col, ok);
+#pragma unroll
+      for (int kp = 0; kp < kNK; ++kp)
+        cp_async_16(sK + (stage * kNK + kp) * kBN * D * 2 + swz<D>(r, ch),
+                    Krot + kp * k_plane + ((size_t)b * k_rows + rr) * Hkv * D + col, ok);
       cp_async_16(sV + stage * kBN * D * 2 + swz<D>(r, ch),
                   V + ((size_t)b * v_rows + rr) * Hkv * D + col, ok);
     }
@@ -108,27 +155,30 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
   // Key tiles this CTA visits: 0 .. the last row's diagonal, narrowed to the
   // keys of the pieces in piece_mask (a single-piece pass skips the rest).
   int kt_begin = 0, kt_end = (q_off + q0 + kBM - 1) / kBN + 1;
-  if (piece_mask != 7) {
-    const int cq_lo = (q_off + q0) / s;
-    const int cq_hi = (q_off + min(q0 + kBM, L) - 1) / s;
-    int key_lo = INT_MAX, key_hi = -1;  // inclusive key range of the pieces
-    if (piece_mask & 1) {
-      key_lo = min(key_lo, cq_lo * s);
-      key_hi = max(key_hi, q_off + q0 + kBM - 1);
-    }
-    if ((piece_mask & 2) && cq_hi >= 1) {
-      key_lo = min(key_lo, max(cq_lo - 1, 0) * s);
-      key_hi = max(key_hi, cq_hi * s - 1);
-    }
-    if ((piece_mask & 4) && cq_hi >= 2) {
-      key_lo = min(key_lo, 0);
-      key_hi = max(key_hi, (cq_hi - 1) * s - 1);
-    }
-    if (key_hi < 0) {
-      kt_end = 0;
-    } else {
-      kt_begin = key_lo / kBN;
-      kt_end = min(kt_end, key_hi / kBN + 1);
+  if constexpr (Rule::kDca) {
+    if (piece_mask != 7) {
+      const int s = rule.s;
+      const int cq_lo = (q_off + q0) / s;
+      const int cq_hi = (q_off + min(q0 + kBM, L) - 1) / s;
+      int key_lo = INT_MAX, key_hi = -1;  // inclusive key range of the pieces
+      if (piece_mask & 1) {
+        key_lo = min(key_lo, cq_lo * s);
+        key_hi = max(key_hi, q_off + q0 + kBM - 1);
+      }
+      if ((piece_mask & 2) && cq_hi >= 1) {
+        key_lo = min(key_lo, max(cq_lo - 1, 0) * s);
+        key_hi = max(key_hi, cq_hi * s - 1);
+      }
+      if ((piece_mask & 4) && cq_hi >= 2) {
+        key_lo = min(key_lo, 0);
+        key_hi = max(key_hi, (cq_hi - 1) * s - 1);
+      }
+      if (key_hi < 0) {
+        kt_end = 0;
+      } else {
+        kt_begin = key_lo / kBN;
+        kt_end = min(kt_end, key_hi / kBN + 1);
+      }
     }
   }
   if (kt_begin < kt_end) load_kv(0, kt_begin);
@@ -159,15 +209,12 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
     __syncthreads();
 
     const int k0 = kt * kBN;
-    const uint32_t kb = sK + stage * kBN * D * 2;
+    const uint32_t kb = sK + stage * kNK * kBN * D * 2;
     const uint32_t vb = sV + stage * kBN * D * 2;
 
-    // Pieces this warp's rows meet in this tile (chunk differences form an
-    // interval; causal pairs have difference >= 0).
-    const int ci_lo = r0_abs / s, ci_hi = (r0_abs + 15) / s;
-    const int cj_lo = k0 / s, cj_hi = (k0 + kBN - 1) / s;
-    const int dmin = max(ci_lo - cj_hi, 0), dmax = ci_hi - cj_lo;
-    const bool present[3] = {dmin == 0, dmin <= 1 && dmax >= 1, dmax >= 2};
+    // Pieces this warp's rows meet in this tile.
+    bool present[3];
+    rule.meets(r0_abs, k0, present);
     // pieces computed in this pass (piece_mask: 1 intra, 2 successive, 4 inter)
     const bool need[3] = {present[0] && (piece_mask & 1), present[1] && (piece_mask & 2),
                           present[2] && (piece_mask & 4)};
@@ -177,27 +224,25 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
     float sacc[8][4];
     if (npieces == 1 && npresent == 1) {
       const int p = need[0] ? 0 : (need[1] ? 1 : 2);
-      compute_s<D>(sacc, sQ + p * kBM * D * 2, kb, warp, lane);
+      compute_s<D>(sacc, sQ + p * kBM * D * 2, kb + rule.kplane(p) * kBN * D * 2, warp, lane);
     } else {
       // keys of pieces not computed here stay -inf (excluded from the softmax)
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[nt][e] = -INFINITY;
-      const int ci_a = i_a / s, ci_b = i_b / s;
+      const int rk_a = rule.row_key(i_a), rk_b = rule.row_key(i_b);
 #pragma unroll 1
-      for (int p = 0; p < 3; ++p) {
+      for (int p = 0; p < Rule::kPieces; ++p) {
         if (!need[p]) continue;
         float tmp[8][4];
-        compute_s<D>(tmp, sQ + p * kBM * D * 2, kb, warp, lane);
+        compute_s<D>(tmp, sQ + p * kBM * D * 2, kb + rule.kplane(p) * kBN * D * 2, warp, lane);
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = k0 + nt * 8 + 2 * t4 + (e & 1);
-            const int d = ((e >> 1) ? ci_b : ci_a) - j / s;
-            const int pe = d <= 0 ? 0 : (d == 1 ? 1 : 2);
-            if (pe == p) sacc[nt][e] = tmp[nt][e];
+            if (rule.piece((e >> 1) ? rk_b : rk_a, j) == p) sacc[nt][e] = tmp[nt][e];
           }
       }
     }
@@ -291,12 +336,12 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
   }
 }
 
-template <int D>
+template <int D, class Rule>
 cudaError_t launch_mma(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
-                       int B, int L, int Hq, int Hkv, int s, int c, float scale, int piece_mask,
+                       int B, int L, int Hq, int Hkv, Rule rule, float scale, int piece_mask,
                        float* Of32, int q_off, int k_rows, int v_rows, cudaStream_t stream) {
-  const int smem = (3 * kBM + 4 * kBN) * D * 2;
-  auto kern = prefill_attn_mma_kernel<D>;
+  const int smem = (Rule::kQPlanes * kBM + 2 * Rule::kKPlanes * kBN + 2 * kBN) * D * 2;
+  auto kern = prefill_attn_mma_kernel<D, Rule>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((L + kBM - 1) / kBM, Hq, B);
@@ -304,7 +349,7 @@ cudaError_t launch_mma(const void* Qrot, const void* Krot, const void* V, void* 
   kern<<<grid, kThreads, smem, stream>>>(
       static_cast<const __half*>(Qrot), static_cast<const __half*>(Krot),
       static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(O), LSE, B, L, Hq, Hkv,
-      s, c, scale_log2, piece_mask, Of32, q_off, k_rows, v_rows, q_off + L);
+      rule, scale_log2, piece_mask, Of32, q_off, k_rows, v_rows, q_off + L);
   return cudaGetLastError();
 }
 
@@ -317,10 +362,11 @@ cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const vo
                                     float* Of32) {
   using namespace mma_path;
   if (L == 0 || B == 0 || Hq == 0) return cudaSuccess;
+  const DcaRule rule{s};
   if (D == 64)
-    return launch_mma<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, piece_mask, Of32, 0,
+    return launch_mma<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, scale, piece_mask, Of32, 0,
                           L, L, stream);
-  return launch_mma<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, s, c, scale, piece_mask, Of32, 0,
+  return launch_mma<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, scale, piece_mask, Of32, 0,
                          L, L, stream);
 }
 
@@ -330,11 +376,25 @@ cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, co
                                           cudaStream_t stream) {
   using namespace mma_path;
   if (Lq == 0 || B == 0 || Hq == 0) return cudaSuccess;
+  const DcaRule rule{s};
   if (D == 64)
-    return launch_mma<64>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, s, c, scale, 7, nullptr,
-                          t0, t0 + Lq, Tcap, stream);
-  return launch_mma<128>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, s, c, scale, 7, nullptr, t0,
+    return launch_mma<64>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
+                          t0 + Lq, Tcap, stream);
+  return launch_mma<128>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
                          t0 + Lq, Tcap, stream);
+}
+
+cudaError_t launch_prefill_attn_selfextend(const void* Qse, const void* Kse, const void* V,
+                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                           int D, int W, float scale, cudaStream_t stream) {
+  using namespace mma_path;
+  if (L == 0 || B == 0 || Hq == 0) return cudaSuccess;
+  const SelfExtendRule rule{W};
+  if (D == 64)
+    return launch_mma<64>(Qse, Kse, V, O, LSE, B, L, Hq, Hkv, rule, scale, 3, nullptr, 0, L, L,
+                          stream);
+  return launch_mma<128>(Qse, Kse, V, O, LSE, B, L, Hq, Hkv, rule, scale, 3, nullptr, 0, L, L,
+                         stream);
 }
 
 // Combine the three single-piece passes: O = sum_p e^{LSE_p - LSE} O_p with

@@ -311,6 +311,41 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 
+size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D) {
+  if (B < 0 || L < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
+  return align256((size_t)2 * B * L * Hq * D * 2) + align256((size_t)2 * B * L * Hkv * D * 2);
+}
+
+dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const void* V, void* O,
+                                         float* LSE, int B, int L, int Hq, int Hkv, int D, int G,
+                                         int W, float base, float scale, void* workspace,
+                                         size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_prefill_selfextend";
+  dca_status_t st = check_heads(fn, B, L, Hq, Hkv, D);
+  if (st != DCA_OK) return st;
+  if (G < 1 || W < 1)
+    return fail(DCA_ERR_INVALID_ARG, "%s: need group size G >= 1 and window W >= 1 (G=%d W=%d)",
+                fn, G, W);
+  if (!(base > 1.f)) return fail(DCA_ERR_INVALID_ARG, "%s: RoPE base must be > 1", fn);
+  if ((long long)B * L == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = dca_selfextend_workspace(B, L, Hq, Hkv, D);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
+  void* kse = static_cast<char*>(workspace) + align256((size_t)2 * B * L * Hq * D * 2);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_selfextend_rope(Q, K, workspace, kse, B, L, Hq, Hkv, D, G, W, base, strm);
+  if (e == cudaSuccess)
+    e = launch_prefill_attn_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc, strm);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 size_t dca_attn_decode_workspace(int B, int Hq, int D, int Tcap) {
   if (B < 0 || Hq < 1 || (D != 64 && D != 128) || Tcap < 1) return 0;
   return decode_workspace_bytes(B, Hq, D, Tcap);

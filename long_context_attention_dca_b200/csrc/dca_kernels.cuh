@@ -34,6 +34,16 @@ cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, co
                                           int D, int s, int c, float scale, int t0, int Tcap,
                                           cudaStream_t stream);
 
+// SelfExtend (prior-art position map): Qse [2][B][L][Hq][D] and Kse
+// [2][B][L][Hkv][D] fp16 (neighbour, grouped rotations), then the general
+// kernel with the neighbour / grouped rule.
+cudaError_t launch_selfextend_rope(const void* Q, const void* K, void* Qse, void* Kse, int B,
+                                   int L, int Hq, int Hkv, int D, int G, int W, float base,
+                                   cudaStream_t stream);
+cudaError_t launch_prefill_attn_selfextend(const void* Qse, const void* Kse, const void* V,
+                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                           int D, int W, float scale, cudaStream_t stream);
+
 // General prefill attention (warp MMA; any s, D in {64, 128}).  piece_mask
 // selects the pieces the softmax covers (1 intra, 2 successive, 4 inter; 7 =
 // DCA); with Of32 set, the normalised O is written there in fp32 instead.

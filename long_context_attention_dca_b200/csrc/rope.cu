@@ -296,6 +296,44 @@ __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restric
   }
 }
 
+// SelfExtend rotations, fp16: query planes [2][B][L][Hq][D] at i (neighbour)
+// and floor(i/G) + W - floor(W/G) (grouped); key planes [2][B][L][Hkv][D] at
+// j and floor(j/G).  One thread per (row, head, 16-byte pair group).
+template <int D>
+__global__ void __launch_bounds__(256) selfextend_rope_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+    __half* __restrict__ Qse, __half* __restrict__ Kse, int B, int L, int Hq, int Hkv, int G,
+    int W, double log2_base) {
+  constexpr int kGroups = D / 16;
+  const int heads = Hq + Hkv;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)B * L * heads * kGroups) return;
+  const int g = (int)(gid % kGroups);
+  const int hh = (int)((gid / kGroups) % heads);
+  const long long row = gid / ((long long)kGroups * heads);
+  const int i = (int)(row % L);
+  const bool is_k = hh < Hkv;
+  const int h = is_k ? hh : hh - Hkv;
+  const int H = is_k ? Hkv : Hq;
+  const size_t off = ((size_t)row * H + h) * D + g * 8;
+  const size_t plane = (size_t)B * L * H * D;
+  const __nv_bfloat16* src = is_k ? K : Q;
+  __half* dst = is_k ? Kse : Qse;
+  const uint4 lo = __ldg(reinterpret_cast<const uint4*>(src + off));
+  const uint4 hi = __ldg(reinterpret_cast<const uint4*>(src + off + D / 2));
+  const int grouped = is_k ? i / G : i / G + W - W / G;
+  CosSin8 cs;
+  uint4 olo, ohi;
+  cos_sin_group(i, g * 8, D, log2_base, cs);
+  rotate8<true>(lo, hi, cs, olo, ohi);
+  *reinterpret_cast<uint4*>(dst + off) = olo;
+  *reinterpret_cast<uint4*>(dst + off + D / 2) = ohi;
+  cos_sin_group(grouped, g * 8, D, log2_base, cs);
+  rotate8<true>(lo, hi, cs, olo, ohi);
+  *reinterpret_cast<uint4*>(dst + plane + off) = olo;
+  *reinterpret_cast<uint4*>(dst + plane + off + D / 2) = ohi;
+}
+
 }  // namespace rope_path
 
 
@@ -380,6 +418,26 @@ cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, 
   keys_to_f16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(Kcache),
                                                  static_cast<uint4*>(Kf16), rows, Tcap,
                                                  out_rows, gpr, total);
+  return cudaGetLastError();
+}
+}  // namespace dca
+
+namespace dca {
+cudaError_t launch_selfextend_rope(const void* Q, const void* K, void* Qse, void* Kse, int B,
+                                   int L, int Hq, int Hkv, int D, int G, int W, float base,
+                                   cudaStream_t stream) {
+  using namespace rope_path;
+  const long long total = (long long)B * L * (Hq + Hkv) * (D / 16);
+  if (total == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((total + 255) / 256);
+  auto args = [&](auto kern) {
+    kern<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(Q),
+                                     static_cast<const __nv_bfloat16*>(K),
+                                     static_cast<__half*>(Qse), static_cast<__half*>(Kse), B, L,
+                                     Hq, Hkv, G, W, log2((double)base));
+  };
+  if (D == 64) args(selfextend_rope_kernel<64>);
+  else args(selfextend_rope_kernel<128>);
   return cudaGetLastError();
 }
 }  // namespace dca

@@ -59,6 +59,9 @@ def test_workspace_queries(lib):
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, 50) == (
         up(3 * 2 * 100 * 8 * 128 * 2) + up(2 * 150 * 2 * 128 * 2))
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, -1) == 0
+    # SelfExtend: neighbour + grouped rotations of Q and K, fp16
+    assert dca.dca_selfextend_workspace(1, 100, 4, 2, 64) == (up(2 * 100 * 4 * 64 * 2) +
+                                                              up(2 * 100 * 2 * 64 * 2))
 
 
 def test_prefill_path_selection(lib):
@@ -126,6 +129,14 @@ def test_argument_errors_return_codes(lib):
                                             0.0, ws, 1 << 30, None)) == 1
     assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, 64, 128, 16, 32, 1e4,
                                             0.0, ws, 64, None)) == 5
+    # SelfExtend: G < 1, W < 1, short workspace
+    sargs = (fake,) * 5
+    assert _code(lib.dca_attn_prefill_selfextend(*sargs, 1, 64, 4, 2, 128, 0, 8, 1e4, 0.0, ws,
+                                                 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_selfextend(*sargs, 1, 64, 4, 2, 128, 2, 0, 1e4, 0.0, ws,
+                                                 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_selfextend(*sargs, 1, 64, 4, 2, 128, 2, 8, 1e4, 0.0, ws,
+                                                 64, None)) == 5
     # wait self-test: deadline out of range
     assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
     assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1

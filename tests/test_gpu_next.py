@@ -295,3 +295,52 @@ def test_chunked_prefill_workload_sampled():
                                     pu.F64View(V[:, a:e]), model[:, :a], pu.F64View(V[:, :a]),
                                     a, s, c, rows=rows, heads=heads)
         _check_chunk(outs[k][0], outs[k][1], ref, f"7B chunk [{a}, {e})")
+
+
+# ---------------------------------------------------------------------------
+# SelfExtend position map (prior art) on the same general kernel
+# ---------------------------------------------------------------------------
+
+SE_CASES = [
+    # B, L, Hq, Hkv, D, G, W
+    (1, 300, 4, 2, 128, 2, 3),
+    (2, 333, 4, 4, 64, 3, 40),
+    (1, 700, 8, 2, 128, 8, 100),
+    (1, 517, 2, 1, 64, 4, 64),
+    (1, 129, 2, 2, 128, 1, 5),      # G = 1: plain RoPE attention
+    (1, 200, 2, 1, 128, 5, 1000),   # W >= L: plain RoPE attention
+    (1, 1, 2, 1, 64, 3, 2),
+]
+
+
+@pytest.mark.parametrize("case", SE_CASES, ids=str)
+def test_selfextend_matches_oracle(case):
+    B, L, Hq, Hkv, D, G, Wn = case
+    Q, K, V = W.make_prefill_inputs(dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=L + G)
+    O, LSE = dca.dca_attn_prefill_selfextend(Q.cuda(), K.cuda(), V.cuda(), G, Wn)
+    dca.dca_sync_status()
+    ref = orc.selfextend_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), G, Wn)
+    mx, mean, lse = pu.compare_rows(O.cpu(), LSE.cpu(), ref)
+    print(f"selfextend {case}: O max {mx:.3e} mean {mean:.3e} LSE rel {lse:.3e}")
+    pu.assert_close(mx, mean, lse, f"selfextend {case}")
+    if G == 1 or Wn >= L:
+        # the library's own plain path: DCA with one chunk covering the sequence
+        O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), L, L)
+        assert (O.float() - O1.float()).abs().max().item() < 2e-2
+        assert (LSE - L1).abs().max().item() < 1e-3
+
+
+def test_selfextend_workload_sampled():
+    # the 16k-token 7B workload with G = 8, W = 1024 (largest distance 2943 < 4096)
+    cfg = W.CONFIGS["llama2_7b_16k"]
+    G, Wn = 8, 1024
+    Q, K, V = W.make_prefill_inputs(cfg)
+    O, LSE = dca.dca_attn_prefill_selfextend(Q.cuda(), K.cuda(), V.cuda(), G, Wn)
+    dca.dca_sync_status()
+    L = cfg["L"]
+    rows = sorted(set(pu.sample_rows(L, 1024, 2048, n_random=24)) | {1023, 1024, 1025, L - 1})
+    ref = orc.selfextend_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), G, Wn,
+                                      rows=rows, heads=[0, cfg["Hq"] - 1])
+    mx, mean, lse = pu.compare_rows(O.cpu(), LSE.cpu(), ref)
+    print(f"selfextend 7B: O max {mx:.3e} mean {mean:.3e} LSE rel {lse:.3e}")
+    pu.assert_close(mx, mean, lse, "selfextend 7B")
