@@ -322,7 +322,9 @@ def run_ours(args, rank, world, dev):
             tf, n_rows, n_heads, dt = oracle_sample(args.cpu_seconds, name=args.workload)
             cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                    "sample": f"{n_rows} random query rows x {n_heads} head of the {args.workload} "
-                             f"prefill workload, fp64 oracle, {dt:.1f} s"}
+                             f"prefill workload, fp64 oracle, {dt:.1f} s",
+                   "rows_per_s": n_rows * n_heads / dt,
+                   "extrapolated_full_prefill_s": flops / (tf * 1e12) if tf > 0 else None}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -338,8 +340,11 @@ def run_ours(args, rank, world, dev):
                              "3.2 GB); no flush"},
             "prefill": {"tflops_rope_plus_attn": value / world, "attn_tflops": attn_tflops,
                         "attn_ms": attn_sum / args.steps, "rope_ms": rope_sum / args.steps,
+                        "attn_ms_median": statistics.median(attn_ms),
+                        "rope_ms_median": statistics.median(rope_ms),
                         "rope_gbs": rope_gbs, "frac_of_peak": attn_tflops / tpk},
             "decode": {"value": dec_gbs, "unit": "GB/s", "ms": dec_sum / args.steps,
+                       "ms_median": statistics.median(dec_ms),
                        "bytes_per_step": dec_bytes, "frac_of_hbm_peak": dec_gbs / world / hbm},
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpk,
                          "unit": "TFLOP/s", "frac": attn_tflops / tpk,
