@@ -199,6 +199,36 @@ dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const voi
                                          int W, float base, float scale, void* workspace,
                                          size_t ws_bytes, void* stream);
 
+/* Device workspace bytes for dca_attn_prefill_host with chunks of chunk_rows
+ * rows: the whole sequence's rotated keys (fp16) and values, plus two
+ * chunk-sized sets of staging and output buffers.  Returns 0 for unsupported
+ * arguments. */
+size_t dca_attn_prefill_host_workspace(int B, int L, int Hq, int Hkv, int D, int chunk_rows);
+
+/* dca_attn_prefill with HOST buffers: Q, K, V are read from and O, LSE
+ * written to host memory (same layouts as dca_attn_prefill), with the PCIe
+ * copies overlapped with the attention.  The sequence is processed in chunks
+ * of chunk_rows rows; chunk k is the chunked prefill of rows k*chunk_rows ..
+ * against the keys before it (the index rule depends only on absolute
+ * indices), so the results equal dca_attn_prefill's.  Copies of chunk k+1 in,
+ * the kernels of chunk k and the copies of chunk k-1's results out run
+ * concurrently; this serves DCA as a drop-in wrapper on a host-fed pipeline
+ * (Guide, "Strategic Recommendations", item 1).
+ *   - Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister):
+ *     with pageable memory the copies serialise.
+ *   - Kernels run on `stream`; the call creates two copy streams and its
+ *     events and releases them before returning (they are freed once the
+ *     queued work is done), so it cannot be captured into a CUDA graph.
+ *     Work queued on `stream` after the call runs after the last copy out.
+ *   - The tcgen05 path is used when D == 128, s % 256 == 0 and chunk_rows is
+ *     a multiple of 256 or covers the sequence; otherwise the warp-MMA path.
+ *   - `workspace`: dca_attn_prefill_host_workspace bytes of device memory.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_host(const void* Q, const void* K, const void* V, void* O,
+                                   float* LSE, int B, int L, int Hq, int Hkv, int D, int s, int c,
+                                   float base, float scale, int chunk_rows, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 /* Which prefill path DCA_PATH_AUTO takes for these sizes (1 general,
  * 2 tcgen05), or 0 for unsupported arguments. */
 int dca_prefill_path(int L, int D, int s, int c);

@@ -26,6 +26,7 @@ __all__ = [
     "dca_attn_prefill_3pass_workspace", "dca_attn_prefill_3pass",
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
+    "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
     "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
     "dca_debug_index_map", "dca_debug_wait_timeout",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
@@ -51,6 +52,9 @@ _SIGS = {
     "dca_attn_prefill_3pass_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "dca_selfextend_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_attn_prefill_host_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "dca_attn_prefill_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I,
+                                   _P, _Z, _P]),
     "dca_attn_prefill_selfextend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F,
                                          _P, _Z, _P]),
     "dca_attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
@@ -267,6 +271,40 @@ def dca_attn_prefill_selfextend(Q, K, V, G, W, base=10000.0, scale=0.0):
     _check(lib().dca_attn_prefill_selfextend(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L,
                                              Hq, Hkv, D, int(G), int(W), base, scale, _ptr(ws),
                                              ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_host_workspace(B: int, L: int, Hq: int, Hkv: int, D: int,
+                                    chunk_rows: int) -> int:
+    return int(lib().dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, chunk_rows))
+
+
+def dca_attn_prefill_host(Q, K, V, s, c, base=10000.0, scale=0.0, chunk_rows=2048,
+                          workspace=None, O=None, LSE=None, device=None):
+    """DCA prefill with host (CPU) tensors in and out, copies overlapped with
+    the kernels.  Q, K, V: contiguous bf16 CPU tensors (pinned for overlap);
+    returns CPU (O, LSE), written into O / LSE when given.  `workspace` is a
+    device uint8 tensor (allocated when None) on `device`.  Asynchronous on
+    the device's current stream: synchronise before reading O and LSE."""
+    for t, name in ((Q, "Q"), (K, "K"), (V, "V")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 \
+                or t.dim() != 4 or not t.is_contiguous():
+            raise DcaError(1, f"{name} must be a contiguous 4-d bf16 CPU tensor")
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else \
+        torch.device(device)
+    if workspace is None:
+        workspace = _workspace(dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, chunk_rows), dev)
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if LSE is None:
+        LSE = torch.empty((B, Hq, L), dtype=torch.float32, pin_memory=True)
+    with torch.cuda.device(dev):
+        strm = torch.cuda.current_stream(dev).cuda_stream
+        _check(lib().dca_attn_prefill_host(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L,
+                                           Hq, Hkv, D, s, c, base, scale, int(chunk_rows),
+                                           _ptr(workspace), workspace.numel(), strm))
     return O, LSE
 
 

@@ -370,18 +370,18 @@ cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const vo
                          L, L, stream);
 }
 
-cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* Vcache,
+cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* V,
                                           void* O, float* LSE, int B, int Lq, int Hq, int Hkv,
-                                          int D, int s, int c, float scale, int t0, int Tcap,
-                                          cudaStream_t stream) {
+                                          int D, int s, int c, float scale, int t0, int k_rows,
+                                          int v_rows, cudaStream_t stream) {
   using namespace mma_path;
   if (Lq == 0 || B == 0 || Hq == 0) return cudaSuccess;
   const DcaRule rule{s};
   if (D == 64)
-    return launch_mma<64>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
-                          t0 + Lq, Tcap, stream);
-  return launch_mma<128>(Qrot, Kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
-                         t0 + Lq, Tcap, stream);
+    return launch_mma<64>(Qrot, Kf16, V, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
+                          k_rows, v_rows, stream);
+  return launch_mma<128>(Qrot, Kf16, V, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
+                         k_rows, v_rows, stream);
 }
 
 cudaError_t launch_prefill_attn_selfextend(const void* Qse, const void* Kse, const void* V,

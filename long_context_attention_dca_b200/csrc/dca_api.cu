@@ -299,7 +299,7 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
   // keys are rotated here and rounded once, to fp16, like a one-shot prefill.
   void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * B * Lq * Hq * D * 2);
   cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, B, Lq, Hq, Hkv, D,
-                                    t0, Tcap, s, c, base, strm);
+                                    t0, Tcap, t0 + Lq, s, c, base, strm);
   if (e == cudaSuccess) e = launch_keys_to_f16(Kcache, kf16, B, t0, Tcap, t0 + Lq, Hkv, D, strm);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   if (auto_path(D, s) == DCA_PATH_TCGEN05 && s % 256 == 0 && t0 % 256 == 0)
@@ -307,7 +307,7 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
                                      strm, t0, t0 + Lq, Tcap);
   else
     e = launch_prefill_attn_mma_chunk(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, c, sc,
-                                      t0, Tcap, strm);
+                                      t0, t0 + Lq, Tcap, strm);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 

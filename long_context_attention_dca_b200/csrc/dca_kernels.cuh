@@ -21,18 +21,19 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
                                 cudaStream_t stream);
 
 // Chunk of Lq rows at absolute positions t0 .. t0+Lq-1: Qrot [3][B][Lq][Hq][D]
-// fp16; rotated keys go in bf16 to cache rows t0 + r (pitch Tcap) and in fp16
-// to rows t0 + r of Kf16 [B][t0+Lq][Hkv][D]; values to cache rows t0 + r.
+// fp16; rotated keys go in bf16 to cache rows t0 + r (pitch Tcap; skipped when
+// Kcache is null) and in fp16 to rows t0 + r of Kf16 (kh_rows rows per
+// sequence); values to cache rows t0 + r (skipped when Vcache is null).
 cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
-                              int Hkv, int D, int t0, int Tcap, int s, int c, float base,
-                              cudaStream_t stream);
-// Attention of that chunk over keys 0 .. t0+Lq-1 of Kf16 and the value cache
-// (general path).
-cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* Vcache,
+                              int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
+                              float base, cudaStream_t stream);
+// Attention of that chunk over keys 0 .. t0+Lq-1 of Kf16 (k_rows rows per
+// sequence) and V (v_rows rows per sequence) (general path).
+cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* V,
                                           void* O, float* LSE, int B, int Lq, int Hq, int Hkv,
-                                          int D, int s, int c, float scale, int t0, int Tcap,
-                                          cudaStream_t stream);
+                                          int D, int s, int c, float scale, int t0, int k_rows,
+                                          int v_rows, cudaStream_t stream);
 
 // SelfExtend (prior-art position map): Qse [2][B][L][Hq][D] and Kse
 // [2][B][L][Hkv][D] fp16 (neighbour, grouped rotations), then the general

@@ -9,3 +9,4 @@
 #include "attn_prefill_sm100_pp.cu"
 #include "attn_decode.cu"
 #include "decode_noalloc.cu"
+#include "prefill_host.cu"

@@ -125,14 +125,15 @@ constexpr int kRopeThreads = 256;
 // absolute index q_off + r.  Whole-sequence prefill (kChunk false, q_off 0)
 // writes the rotated keys to the fp16 workspace Kout laid out like K.  A chunk
 // against a cache (kChunk true) writes them in bf16 to cache rows q_off + r of
-// pitch Tcap (Kout) and in fp16 to rows q_off + r of Kh (pitch q_off + L), and
-// copies the chunk's values into the value cache.
+// pitch Tcap (Kout, unless null) and in fp16 to rows q_off + r of Kh (kh_rows
+// rows per sequence), and copies the chunk's values into the value cache
+// (unless Vc is null).
 template <int D, bool kChunk>
 __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
     __half* __restrict__ Qrot, void* __restrict__ Kout, int B, int L, int Hq, int Hkv, int s,
     int c, double log2_base, int q_off, int Tcap, const __nv_bfloat16* __restrict__ Vsrc,
-    __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh) {
+    __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh, int kh_rows) {
   constexpr int kHalf = D / 2;
   constexpr int kGroups = D / 16;
   __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   __syncthreads();
   const size_t plane = (size_t)B * L * Hq * D;
   const int heads = Hq + (kChunk ? 2 : 1) * Hkv;  // [keys | (values) | queries]
+  const bool write_kc = Kout != nullptr, write_v = Vc != nullptr;
   const int items = nrows * heads * kGroups;
 #pragma unroll 2
   for (int it = threadIdx.x; it < items; it += kRopeThreads) {
@@ -164,6 +166,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
       const long long seq = row / L;
       const size_t cache_row = (size_t)(seq * Tcap + (row % L) + q_off);
       if (hh >= Hkv && hh < 2 * Hkv) {  // value copy
+        if (!write_v) continue;
         const size_t src = (size_t)row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
         const size_t dst = cache_row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
         *reinterpret_cast<uint4*>(Vc + dst) = __ldg(reinterpret_cast<const uint4*>(Vsrc + src));
@@ -184,12 +187,14 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
           cs.s[e] = v.y;
         }
         uint4 olo, ohi;
-        rotate8<false>(lo, hi, cs, olo, ohi);
-        __nv_bfloat16* Kc = static_cast<__nv_bfloat16*>(Kout);
-        *reinterpret_cast<uint4*>(Kc + dst) = olo;
-        *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
+        if (write_kc) {
+          rotate8<false>(lo, hi, cs, olo, ohi);
+          __nv_bfloat16* Kc = static_cast<__nv_bfloat16*>(Kout);
+          *reinterpret_cast<uint4*>(Kc + dst) = olo;
+          *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
+        }
         rotate8<true>(lo, hi, cs, olo, ohi);
-        const size_t hdst = ((size_t)(seq * (q_off + L) + (row % L) + q_off) * Hkv + hh) * D + g * 8;
+        const size_t hdst = ((size_t)(seq * kh_rows + (row % L) + q_off) * Hkv + hh) * D + g * 8;
         *reinterpret_cast<uint4*>(Kh + hdst) = olo;
         *reinterpret_cast<uint4*>(Kh + hdst + kHalf) = ohi;
         continue;
@@ -362,7 +367,7 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
     kern<<<blocks, kRopeThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Krot, B, L, Hq, Hkv, s, c, log2((double)base), 0, L,
-        nullptr, nullptr, nullptr);
+        nullptr, nullptr, nullptr, 0);
   };
   if (D == 64) args(prefill_rope_kernel<64, false>);
   else args(prefill_rope_kernel<128, false>);
@@ -371,8 +376,8 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
 
 cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
-                              int Hkv, int D, int t0, int Tcap, int s, int c, float base,
-                              cudaStream_t stream) {
+                              int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
+                              float base, cudaStream_t stream) {
   using namespace rope_path;
   const long long rows = (long long)B * Lq;
   if (rows == 0) return cudaSuccess;
@@ -382,7 +387,7 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Kcache, B, Lq, Hq, Hkv, s, c, log2((double)base), t0, Tcap,
         static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(Vcache),
-        static_cast<__half*>(Kf16));
+        static_cast<__half*>(Kf16), kh_rows);
   };
   if (D == 64) args(prefill_rope_kernel<64, true>);
   else args(prefill_rope_kernel<128, true>);

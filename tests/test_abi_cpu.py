@@ -59,6 +59,14 @@ def test_workspace_queries(lib):
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, 50) == (
         up(3 * 2 * 100 * 8 * 128 * 2) + up(2 * 150 * 2 * 128 * 2))
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, -1) == 0
+    # host prefill: whole-sequence fp16 keys and values + two chunk-sized sets
+    # of staging (Q, K), outputs (O, LSE) and one chunk's three query rotations
+    B, L, Hq, Hkv, D, C = 2, 1000, 8, 2, 64, 300
+    want = 2 * up(B * L * Hkv * D * 2) + 2 * (up(B * C * Hq * D * 2) + up(B * C * Hkv * D * 2) +
+                                              up(B * C * Hq * D * 2) + up(B * Hq * C * 4)) + \
+        up(3 * B * C * Hq * D * 2)
+    assert dca.dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, C) == want
+    assert dca.dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, 0) == 0
     # SelfExtend: neighbour + grouped rotations of Q and K, fp16
     assert dca.dca_selfextend_workspace(1, 100, 4, 2, 64) == (up(2 * 100 * 4 * 64 * 2) +
                                                               up(2 * 100 * 2 * 64 * 2))
@@ -129,6 +137,14 @@ def test_argument_errors_return_codes(lib):
                                             0.0, ws, 1 << 30, None)) == 1
     assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, 64, 128, 16, 32, 1e4,
                                             0.0, ws, 64, None)) == 5
+    # host prefill: chunk_rows < 1, null host buffer, short workspace
+    hargs = (fake,) * 5
+    assert _code(lib.dca_attn_prefill_host(*hargs, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, 0, ws,
+                                           1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_host(None, fake, fake, fake, fake, 1, 64, 4, 2, 128, 16, 32,
+                                           1e4, 0.0, 32, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_host(*hargs, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, 32, ws, 64,
+                                           None)) == 5
     # SelfExtend: G < 1, W < 1, short workspace
     sargs = (fake,) * 5
     assert _code(lib.dca_attn_prefill_selfextend(*sargs, 1, 64, 4, 2, 128, 0, 8, 1e4, 0.0, ws,

@@ -344,3 +344,47 @@ def test_selfextend_workload_sampled():
     mx, mean, lse = pu.compare_rows(O.cpu(), LSE.cpu(), ref)
     print(f"selfextend 7B: O max {mx:.3e} mean {mean:.3e} LSE rel {lse:.3e}")
     pu.assert_close(mx, mean, lse, "selfextend 7B")
+
+
+# ---------------------------------------------------------------------------
+# host-buffer prefill with copies overlapped (chunked internally)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [
+    # B, L, Hq, Hkv, D, s, c, chunk_rows
+    (2, 1100, 8, 2, 128, 512, 640, 256),   # tcgen05 path, ragged last chunk
+    (1, 777, 4, 4, 64, 100, 150, 300),     # warp-MMA path, chunks off the 64-row tiles
+    (1, 500, 2, 1, 128, 256, 384, 4096),   # one chunk
+], ids=str)
+def test_host_prefill_matches_device_prefill_and_oracle(case):
+    B, L, Hq, Hkv, D, s, c, C = case
+    Q, K, V = W.make_prefill_inputs(dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D), seed=L + C)
+    Qp, Kp, Vp = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    O, LSE = dca.dca_attn_prefill_host(Qp, Kp, Vp, s, c, chunk_rows=C)
+    torch.cuda.synchronize()
+    dca.dca_sync_status()
+    O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), s, c)
+    dca.dca_sync_status()
+    d = (O.float() - O1.cpu().float()).abs().max().item()
+    dl = (LSE - L1.cpu()).abs().max().item()
+    print(f"host prefill {case}: vs device O max {d:.3e} LSE max {dl:.3e}")
+    if C % 64 == 0:  # same tiles as the one-shot launch: identical arithmetic
+        assert d == 0.0 and dl == 0.0
+    else:
+        assert d < 2e-2 and dl < 1e-3
+    rows = pu.sample_rows(L, s, c, n_random=24)
+    ref = orc.dca_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), s, c, rows=rows,
+                               heads=pu.sample_heads(Hq, Hkv))
+    mx, mean, lse = pu.compare_rows(O, LSE, ref)
+    pu.assert_close(mx, mean, lse, f"host prefill {case}")
+
+
+def test_host_prefill_workload_equals_device_prefill():
+    cfg = W.CONFIGS["llama2_7b_16k"]
+    Q, K, V = W.make_prefill_inputs(cfg)
+    O, LSE = dca.dca_attn_prefill_host(Q.pin_memory(), K.pin_memory(), V.pin_memory(),
+                                       cfg["s"], cfg["c"], chunk_rows=2048)
+    torch.cuda.synchronize()
+    O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), cfg["s"], cfg["c"])
+    dca.dca_sync_status()
+    assert torch.equal(O, O1.cpu()) and torch.equal(LSE, L1.cpu())
