@@ -426,6 +426,10 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
     with CUDA events, after one untimed call:
       prefill_chunk  the prefill workload as four equal chunks against a cache
                      (dca_attn_prefill_chunk, chunk starts 0, L/4, L/2, 3L/4);
+      prefill_general_path  the attention of the prefill workload forced onto
+                     the general warp-MMA kernel (dca_prefill_attention);
+      prefill_unaligned_s  the prefill workload's attention with s = 3000 (tiles
+                     straddle chunk boundaries; dca_prefill_attention, auto path);
       prefill_3pass  the prefill workload as three single-piece passes merged
                      by LSE (dca_attn_prefill_3pass);
       prefill_selfextend  the prefill workload under the SelfExtend position
@@ -485,6 +489,50 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                             "path": "tcgen05/TMEM/TMA" if tc else "general (warp MMA)",
                             "launches_per_call": 3 if tc else 2}
     del Kcache, Vcache, cws, Oc, Lc, Ob, Lb, Qs, Ks, Vs
+
+    # the general (warp-MMA) kernel on the same workload: the path of every
+    # chunking the tcgen05 kernels do not cover (straddling tiles, per-element
+    # piece selection)
+    gws = dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+    gbuf = torch.empty(gws, dtype=torch.uint8, device=dev)
+    Og = torch.empty_like(Q)
+    Lg = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s, c, base,
+                              P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+    if st != 0:
+        raise dca.DcaError(st, dca.dca_last_error_string())
+
+    def general():
+        st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
+                                       Hq, Hkv, D, s, c, 0.0, dca.DCA_PATH_GENERAL,
+                                       P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(general)
+    out["prefill_general_path"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                   "ms": ms, "path": "general (warp MMA), attention only",
+                                   "launches_per_call": 1}
+
+    # a chunk size that is not a multiple of the 128-row tiles (s = 3000):
+    # tiles straddle chunk boundaries, the per-row-interval tcgen05 kernel
+    s_u = 3000
+    st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s_u, c, base,
+                              P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+    if st != 0:
+        raise dca.DcaError(st, dca.dca_last_error_string())
+
+    def unaligned():
+        st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
+                                       Hq, Hkv, D, s_u, c, 0.0, dca.DCA_PATH_AUTO,
+                                       P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(unaligned)
+    out["prefill_unaligned_s"] = {
+        "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms, "s": s_u, "c": c,
+        "path": {1: "general (warp MMA)", 2: "tcgen05 per-row intervals"}.get(
+            dca.dca_prefill_path(L, D, s_u, c)), "launches_per_call": 1}
+    del gbuf, Og, Lg
 
     # three passes + LSE merge
     wsz = dca.dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D)

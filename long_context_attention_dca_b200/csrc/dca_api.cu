@@ -76,13 +76,12 @@ PrefillWs prefill_ws_layout(void* base, int B, int L, int Hq, int Hkv, int D) {
   return PrefillWs{p, p ? p + qbytes : nullptr, qbytes + kbytes};
 }
 
-int auto_path(int D, int s) { return (kHaveTcgen05 && D == 128 && s % 128 == 0) ? DCA_PATH_TCGEN05 : DCA_PATH_GENERAL; }
-
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return n;
+// tcgen05 kernels at D = 128 for every chunk size: the two-tile ping-pong
+// kernel when s % 256 == 0 (no tile straddles a chunk), the per-row-interval
+// kernel otherwise; the warp-MMA kernel for D = 64.
+int auto_path(int D, int s) {
+  (void)s;
+  return (kHaveTcgen05 && D == 128) ? DCA_PATH_TCGEN05 : DCA_PATH_GENERAL;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -190,8 +189,8 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   if (path < DCA_PATH_AUTO || path > DCA_PATH_TCGEN05)
     return fail(DCA_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
   if (path == DCA_PATH_AUTO) path = auto_path(D, s);
-  if (path == DCA_PATH_TCGEN05 && auto_path(D, s) != DCA_PATH_TCGEN05)
-    return fail(DCA_ERR_UNSUPPORTED, "%s: tcgen05 path needs D == 128 and s %% 128 == 0", fn);
+  if (path == DCA_PATH_TCGEN05 && !(kHaveTcgen05 && D == 128))
+    return fail(DCA_ERR_UNSUPPORTED, "%s: tcgen05 path needs D == 128", fn);
   if ((long long)B * L == 0) return DCA_OK;
   DCA_CHECK_PTR(V);
   DCA_CHECK_PTR(O);
@@ -206,9 +205,8 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   cudaError_t e;
   if (path == DCA_PATH_TCGEN05 && s % 256 == 0)
     e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
-  else if (path == DCA_PATH_TCGEN05)
-    e = launch_prefill_attn_sm100(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, c, sc,
-                                  sm_count(), strm);
+  else if (path == DCA_PATH_TCGEN05)  // tiles or tile pairs straddle chunk boundaries
+    e = launch_prefill_attn_sm100_gen(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
   else
     e = launch_prefill_attn_mma(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, c, sc, strm);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
@@ -305,6 +303,9 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
   if (auto_path(D, s) == DCA_PATH_TCGEN05 && s % 256 == 0 && t0 % 256 == 0)
     e = launch_prefill_attn_sm100_pp(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
                                      strm, t0, t0 + Lq, Tcap);
+  else if (auto_path(D, s) == DCA_PATH_TCGEN05)
+    e = launch_prefill_attn_sm100_gen(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
+                                      strm, t0, t0 + Lq, Tcap);
   else
     e = launch_prefill_attn_mma_chunk(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, c, sc,
                                       t0, t0 + Lq, Tcap, strm);

@@ -56,11 +56,6 @@ cudaError_t launch_prefill_attn_mma(const void* Qrot, const void* Krot, const vo
 cudaError_t launch_merge3(const float* Op, const float* LSEp, void* O, float* LSE, int B, int L,
                           int Hq, int D, cudaStream_t stream);
 
-// tcgen05/TMEM/TMA prefill attention (D = 128, s % 128 == 0).
-cudaError_t launch_prefill_attn_sm100(const void* Qrot, const void* Krot, const void* V, void* O,
-                                      float* LSE, int B, int L, int Hq, int Hkv, int D, int s,
-                                      int c, float scale, int num_sms, cudaStream_t stream);
-
 // tcgen05 ping-pong variant: two query tiles per CTA (D = 128, s % 256 == 0).
 // Chunk form: query rows q_off .. q_off+L-1 (q_off % 256 == 0) against keys
 // 0 .. q_off+L-1 held with k_rows / v_rows rows per sequence (0: q_off + L).
@@ -68,6 +63,12 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
                                          int q_off = 0, int k_rows = 0, int v_rows = 0);
+// tcgen05 prefill attention for any chunk size (D = 128): per-row key
+// intervals per piece, straddling tiles visited once per piece they hold.
+cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
+                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                          int D, int s, float scale, cudaStream_t stream,
+                                          int q_off = 0, int k_rows = 0, int v_rows = 0);
 // Rows 0 .. rows-1 of a bf16 key cache [B][Tcap][Hkv][D] -> the same rows of
 // fp16 [B][out_rows][Hkv][D].
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,

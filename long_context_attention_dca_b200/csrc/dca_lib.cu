@@ -5,8 +5,8 @@
 #include "rope.cu"
 #include "index_map.cu"
 #include "attn_prefill_mma.cu"
-#include "attn_prefill_sm100.cu"
 #include "attn_prefill_sm100_pp.cu"
+#include "attn_prefill_sm100_gen.cu"
 #include "attn_decode.cu"
 #include "decode_noalloc.cu"
 #include "prefill_host.cu"

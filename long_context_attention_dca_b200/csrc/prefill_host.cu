@@ -90,9 +90,11 @@ extern "C" dca_status_t dca_attn_prefill_host(const void* Q, const void* K, cons
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int n_chunks = (L + C - 1) / C;
-  // tcgen05 kernel when every chunk start is a multiple of its 256-row pairs
-  const bool tc =
-      auto_path(D, s) == DCA_PATH_TCGEN05 && s % 256 == 0 && (C % 256 == 0 || n_chunks == 1);
+  // the two-tile kernel when every chunk start is a multiple of its 256-row
+  // pairs and no tile straddles a chunk; the per-row-interval tcgen05 kernel
+  // for any other chunking at D = 128
+  const bool tc = auto_path(D, s) == DCA_PATH_TCGEN05;
+  const bool pp = tc && s % 256 == 0 && (C % 256 == 0 || n_chunks == 1);
 
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t* ev = nullptr;  // [3][n_chunks]: copied in, computed, copied out
@@ -143,9 +145,12 @@ extern "C" dca_status_t dca_attn_prefill_host(const void* Q, const void* K, cons
       e = launch_chunk_rope(w.qin[slot], w.kin[slot], nullptr, w.qrot, nullptr, nullptr, w.kh,
                             B, Lq, Hq, Hkv, D, a, L, L, s, c, base, cs);
     if (e == cudaSuccess) {
-      if (tc)
+      if (pp)
         e = launch_prefill_attn_sm100_pp(w.qrot, w.kh, w.vd, w.oc[slot], w.lc[slot], B, Lq, Hq,
                                          Hkv, D, s, sc, cs, a, L, L);
+      else if (tc)
+        e = launch_prefill_attn_sm100_gen(w.qrot, w.kh, w.vd, w.oc[slot], w.lc[slot], B, Lq, Hq,
+                                          Hkv, D, s, sc, cs, a, L, L);
       else
         e = launch_prefill_attn_mma_chunk(w.qrot, w.kh, w.vd, w.oc[slot], w.lc[slot], B, Lq, Hq,
                                           Hkv, D, s, c, sc, a, L, L, cs);

@@ -44,7 +44,8 @@ def _prefill_gpu(Q, K, V, s, c, path, base=10000.0):
 
 
 def _path_ok(path, D, s):
-    return path == dca.DCA_PATH_GENERAL or dca.dca_prefill_path(1, D, s, s) == path
+    # the tcgen05 path takes every chunk size at D = 128 (straddling tiles masked)
+    return path == dca.DCA_PATH_GENERAL or D == 128
 
 
 # ---------------------------------------------------------------------------
@@ -147,6 +148,13 @@ SMALL = [  # (B, L, Hq, Hkv, D, s, c)
     (1, 1300, 2, 2, 128, 256, 4096),   # w > s
     (1, 129, 2, 2, 128, 256, 300),
     (1, 2200, 4, 1, 128, 512, 640),
+    # D = 128, s not a multiple of 128: tiles straddle chunk boundaries
+    (1, 1000, 2, 1, 128, 192, 256),
+    (2, 777, 4, 2, 128, 100, 150),
+    (1, 600, 2, 2, 128, 3, 5),         # many chunks per tile
+    (1, 1500, 4, 4, 128, 300, 400),
+    (1, 900, 2, 1, 128, 160, 1000),    # w > s
+    (1, 1100, 2, 1, 128, 1000, 1000),  # w = 0
 ]
 
 
