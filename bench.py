@@ -203,6 +203,8 @@ def run_ours(args, rank, world, dev):
     P = ctypes.c_void_p
 
     pc = W.CONFIGS[args.workload]
+    if args.override_s:  # profiling runs of the straddling-tile kernel
+        pc = dict(pc, s=args.override_s)
     dc = W.CONFIGS[DECODE]
     Q, K, V = W.make_prefill_inputs(pc, device=dev)
     B, L, Hq, D = Q.shape
@@ -569,7 +571,9 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
     ms = timed(selfextend)
     out["prefill_selfextend"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                                  "ms": ms, "G": G_se, "W": W_se,
-                                 "path": "RoPE (2 planes) + general (warp MMA)",
+                                 "path": "RoPE (2 planes) + " + (
+                                     "tcgen05 per-row intervals" if D == 128
+                                     else "general (warp MMA)"),
                                  "launches_per_call": 2}
     del sws, Ose, Lse
 
@@ -647,6 +651,9 @@ def main():
     ap.add_argument("--next-rows", action=argparse.BooleanOptionalAction, default=True,
                     help="also time chunked prefill, the 3-pass variant and KV append "
                          "(outside the timed step)")
+    ap.add_argument("--override-s", type=int, default=0,
+                    help="profiling runs: chunk size s of the prefill workload (e.g. 3000, "
+                         "whose tiles straddle chunk boundaries)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default=PREFILL, choices=sorted(

@@ -193,8 +193,11 @@ size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D);
  * grouped distance >= W, above all neighbour distances.  G = 1 or W >= L is
  * plain RoPE attention.  Same tensors and conventions as dca_attn_prefill
  * (Q, K unrotated bf16; O bf16; LSE fp32 [B][Hq][L]); any G >= 1, W >= 1,
- * D in {64, 128}; warp-MMA kernel.  `workspace`: dca_selfextend_workspace
- * bytes, 256-byte aligned, scratch for the call.
+ * D in {64, 128}.  Kernels: at D == 128 the per-row-interval tcgen05 kernel
+ * (each row's neighbour keys [i-W+1, i] and grouped keys [0, i-W] are two
+ * intervals, visited with their own query and key rotations); the warp-MMA
+ * kernel at D == 64.  `workspace`: dca_selfextend_workspace bytes, 256-byte
+ * aligned, scratch for the call.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const void* V, void* O,
                                          float* LSE, int B, int L, int Hq, int Hkv, int D, int G,

@@ -59,21 +59,54 @@ static_assert(kSmTotal <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
-// Key interval [lo, hi] of piece p (0 intra, 1 successive, 2 inter) for
-// absolute query row i; lo > hi when the piece is empty for the row.
-__device__ __forceinline__ void piece_keys(int p, int i, int s, int& lo, int& hi) {
-  const int ci = i / s;
-  if (p == kIntra) {
-    lo = ci * s;
-    hi = i;
-  } else if (p == kSucc) {
-    lo = ci >= 1 ? (ci - 1) * s : 1;
-    hi = ci >= 1 ? ci * s - 1 : 0;
-  } else {
-    lo = 0;
-    hi = ci >= 2 ? (ci - 1) * s - 1 : -1;
+// Position rules.  For query row i the keys of each piece form one interval
+// [lo, hi] (lo > hi: none); pieces are walked in increasing key order; a
+// piece reads query plane `piece` and key plane kplane(piece).
+struct DcaIntervals {
+  // pieces 0 intra, 1 successive, 2 inter; one key plane (keys at j mod s)
+  static constexpr int kPieces = 3, kKPlanes = 1;
+  int s;
+  __device__ __forceinline__ int walk(int k) const { return 2 - k; }  // inter, succ, intra
+  __device__ __forceinline__ int kplane(int) const { return 0; }
+  __device__ __forceinline__ void keys(int p, int i, int& lo, int& hi) const {
+    const int ci = i / s;
+    if (p == kIntra) {
+      lo = ci * s;
+      hi = i;
+    } else if (p == kSucc) {
+      lo = ci >= 1 ? (ci - 1) * s : 1;
+      hi = ci >= 1 ? ci * s - 1 : 0;
+    } else {
+      lo = 0;
+      hi = ci >= 2 ? (ci - 1) * s - 1 : -1;
+    }
   }
-}
+  // first row >= r0 whose interval for p is nonempty (they form a suffix)
+  __device__ __forceinline__ int first_row(int p, int r0) const {
+    return p == kIntra ? r0 : max(r0, (p == kSucc ? 1 : 2) * s);
+  }
+};
+
+struct SelfExtendIntervals {
+  // pieces 0 neighbour (i - j < W: keys [i-W+1, i]), 1 grouped (keys
+  // [0, i-W]); query plane p with key plane p
+  static constexpr int kPieces = 2, kKPlanes = 2;
+  int W;
+  __device__ __forceinline__ int walk(int k) const { return 1 - k; }  // grouped, neighbour
+  __device__ __forceinline__ int kplane(int p) const { return p; }
+  __device__ __forceinline__ void keys(int p, int i, int& lo, int& hi) const {
+    if (p == 0) {
+      lo = max(i - W + 1, 0);
+      hi = i;
+    } else {
+      lo = 0;
+      hi = i - W;
+    }
+  }
+  __device__ __forceinline__ int first_row(int p, int r0) const {
+    return p == 0 ? r0 : max(r0, W);
+  }
+};
 
 // The visits of one CTA, computed identically by every role: phase k walks
 // piece pc[k] over key tiles ulo[k] .. uhi[k]; tile X takes part in the
@@ -85,11 +118,13 @@ struct Plan {  // lives in shared memory, written by thread 0 before the CTA bar
 };
 
 // rows_lo[X] .. rows_hi[X]: absolute rows of tile X that exist (lo > hi: none)
-__device__ __forceinline__ Plan make_plan(const int (&rows_lo)[2], const int (&rows_hi)[2],
-                                          int s) {
+template <class Rule>
+__device__ __forceinline__ Plan make_plan(const Rule& rule, const int (&rows_lo)[2],
+                                          const int (&rows_hi)[2]) {
   Plan pl;
   pl.n_ph = 0;
-  for (int p = kInter; p >= kIntra; --p) {
+  for (int w = 0; w < Rule::kPieces; ++w) {
+    const int p = rule.walk(w);
     int lo_t[2], hi_t[2];
     bool any = false;
     for (int x = 0; x < 2; ++x) {
@@ -97,12 +132,12 @@ __device__ __forceinline__ Plan make_plan(const int (&rows_lo)[2], const int (&r
       hi_t[x] = 0;
       const int r0 = rows_lo[x], r1 = rows_hi[x];
       if (r0 > r1) continue;
-      // rows with a nonempty interval are a suffix of the tile's rows
-      const int first = p == kIntra ? r0 : max(r0, (p == kSucc ? 1 : 2) * s);
+      const int first = rule.first_row(p, r0);
       if (first > r1) continue;
+      // both interval ends are nondecreasing in the row
       int lo, hi, lo1, hi1;
-      piece_keys(p, first, s, lo, hi);
-      piece_keys(p, r1, s, lo1, hi1);
+      rule.keys(p, first, lo, hi);
+      rule.keys(p, r1, lo1, hi1);
       lo_t[x] = lo / kTile;
       hi_t[x] = hi1 / kTile;
       any = true;
@@ -145,10 +180,11 @@ __device__ __forceinline__ float row_max_range(uint32_t (&v)[4][32], int clo, in
   return row_max(v);
 }
 
+template <class Rule>
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-    float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2,
+    float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
     int q_off) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -174,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const Plan& pl = *reinterpret_cast<const Plan*>(smem + kSmPlan);
 
   if (tid == 0) {
-    *reinterpret_cast<Plan*>(smem + kSmPlan) = make_plan(rows_lo, rows_hi, s);
+    *reinterpret_cast<Plan*>(smem + kSmPlan) = make_plan(rule, rows_lo, rows_hi);
     for (int i = 0; i < kNumQSlots; ++i) {
       mbar_init(bar(kQFull + i), 1);
       mbar_init(bar(kQEmpty + i), 1);
@@ -238,8 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
             break;
           mbar_arrive_expect_tx(bar(kKFull + sg), kTileBytes);
           const uint32_t kd = sbase + kSmK + sg * kTileBytes;
-          tma_load_4d(kd, &tmK, bar(kKFull + sg), 0, hk, t * kTile, b);
-          tma_load_4d(kd + kBox, &tmK, bar(kKFull + sg), 64, hk, t * kTile, b);
+          const int kb = rule.kplane(pl.pc[k]) * B + b;  // key plane of the piece
+          tma_load_4d(kd, &tmK, bar(kKFull + sg), 0, hk, t * kTile, kb);
+          tma_load_4d(kd + kBox, &tmK, bar(kKFull + sg), 64, hk, t * kTile, kb);
           k_last[sg] = st;
           if (first && !(ok = load_q(2 * k + 1, pl.pc[k]))) break;
           if (st >= 2 &&
@@ -366,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     int j = 0;  // visits of this tile so far
     for (int k = 0; k < pl.n_ph && ok; ++k) {
       int klo, khi;  // this row's key interval for the phase's piece
-      piece_keys(pl.pc[k], i_abs, s, klo, khi);
+      rule.keys(pl.pc[k], i_abs, klo, khi);
       for (int t = pl.ulo[k]; t <= pl.uhi[k]; ++t) {
         if (!takes_part(pl, x, k, t)) continue;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(kSFull + x), j & 1, abort_flag, 497));
@@ -454,15 +491,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
 
 }  // namespace gen_path
 
-// tcgen05 prefill attention for any chunk size (D = 128).  Query rows q_off ..
-// q_off+L-1 against keys 0 .. q_off+L-1 held with k_rows / v_rows rows per
-// sequence (0: q_off + L).
-cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
-                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
-                                          int D, int s, float scale, cudaStream_t stream,
-                                          int q_off, int k_rows, int v_rows) {
-  using namespace gen_path;
-  if (D != kHD || s < 1 || q_off < 0) return cudaErrorInvalidValue;
+namespace gen_path {
+
+// Tensor maps and launch: Qrot [nq planes][B][L][Hq][D] and Krot [kKPlanes]
+// [B][k_rows][Hkv][D] fp16, V [B][v_rows][Hkv][D] bf16.
+template <class Rule>
+cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
+                       int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
+                       cudaStream_t stream, int q_off, int k_rows, int v_rows) {
+  if (D != kHD || q_off < 0) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
   const int Lkv = q_off + L;
   if (k_rows == 0) k_rows = Lkv;
@@ -470,7 +507,7 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
   CUtensorMap tmQ, tmK, tmV;
   const uint32_t box[4] = {64, 1, (uint32_t)kTile, 1};
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)L, (uint64_t)3 * B};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)L, (uint64_t)nq * B};
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hq * D * 2,
                                  (uint64_t)L * Hq * D * 2};
     if (!encode_tensor_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Qrot, 4, dims, strides, box,
@@ -478,27 +515,55 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)B};
+    const uint64_t kdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv,
+                               (uint64_t)Rule::kKPlanes * B};
+    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)B};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
     const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)v_rows * Hkv * D * 2};
-    if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, dims, ks, box,
+    if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, kdims, ks, box,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, dims, vs, box,
+        !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, vdims, vs, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  auto kern = prefill_attn_gen_kernel;
+  auto kern = prefill_attn_gen_kernel<Rule>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
   if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
   dim3 grid((num_qt + 1) / 2, Hq, B);
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
-                                             B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
+                                             B, L, Hq, Hkv, rule, scale * 1.4426950408889634f,
                                              q_off);
   return cudaGetLastError();
+}
+
+}  // namespace gen_path
+
+// tcgen05 prefill attention for any chunk size (D = 128).  Query rows q_off ..
+// q_off+L-1 against keys 0 .. q_off+L-1 held with k_rows / v_rows rows per
+// sequence (0: q_off + L).
+cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
+                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
+                                          int D, int s, float scale, cudaStream_t stream,
+                                          int q_off, int k_rows, int v_rows) {
+  if (s < 1) return cudaErrorInvalidValue;
+  return gen_path::launch_gen(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, D,
+                              gen_path::DcaIntervals{s}, 3, scale, stream, q_off, k_rows,
+                              v_rows);
+}
+
+// SelfExtend on the same kernel: Qse, Kse [2][B][L][H][D] fp16 (neighbour,
+// grouped rotations).
+cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
+                                                 const void* V, void* O, float* LSE, int B,
+                                                 int L, int Hq, int Hkv, int D, int W,
+                                                 float scale, cudaStream_t stream) {
+  if (W < 1) return cudaErrorInvalidValue;
+  return gen_path::launch_gen(Qse, Kse, V, O, LSE, B, L, Hq, Hkv, D,
+                              gen_path::SelfExtendIntervals{W}, 2, scale, stream, 0, 0, 0);
 }
 
 }  // namespace dca

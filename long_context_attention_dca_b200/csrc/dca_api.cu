@@ -342,8 +342,14 @@ dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const voi
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_selfextend_rope(Q, K, workspace, kse, B, L, Hq, Hkv, D, G, W, base, strm);
-  if (e == cudaSuccess)
-    e = launch_prefill_attn_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc, strm);
+  if (e == cudaSuccess) {
+    if (auto_path(D, W) == DCA_PATH_TCGEN05)
+      e = launch_prefill_attn_sm100_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc,
+                                               strm);
+    else
+      e = launch_prefill_attn_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc,
+                                         strm);
+  }
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 

@@ -69,6 +69,11 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off = 0, int k_rows = 0, int v_rows = 0);
+// SelfExtend on the per-row-interval tcgen05 kernel (D = 128).
+cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
+                                                 const void* V, void* O, float* LSE, int B,
+                                                 int L, int Hq, int Hkv, int D, int W,
+                                                 float scale, cudaStream_t stream);
 // Rows 0 .. rows-1 of a bf16 key cache [B][Tcap][Hkv][D] -> the same rows of
 // fp16 [B][out_rows][Hkv][D].
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
