@@ -59,11 +59,6 @@ constexpr int kSmTotal = kSmMisc + 16 + 1024;
 static_assert(kSmTotal <= 232448, "shared memory budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-// Of every 8 column pairs of an off-diagonal tile, this many could be
-// exponentiated on the FMA pipe instead of the special-function unit; measured
-// on B200 the softmax here is latency-bound, not exponent-throughput-bound
-// (1 of 8: no change, 2-3 of 8: slower), so none are.
-constexpr int kPolyPairs = 0;
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
