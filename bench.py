@@ -436,6 +436,8 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                      by LSE (dca_attn_prefill_3pass);
       prefill_selfextend  the prefill workload under the SelfExtend position
                      map, G = 8, W = 1024 (dca_attn_prefill_selfextend);
+      decode_paged   the decode workload over a paged copy of its caches
+                     (dca_attn_decode_paged, 256-row blocks in random order);
       kv_append      one decoded token appended per sequence of the decode
                      batch (dca_kv_append), 100 calls back to back."""
     import ctypes
@@ -576,6 +578,38 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                                      else "general (warp MMA)"),
                                  "launches_per_call": 2}
     del sws, Ose, Lse
+
+    # decode over a paged cache: the decode workload's caches scattered into
+    # 256-row blocks in a seeded random physical order
+    Bd, Tcap, Hkvd, Dd = Kc.shape
+    rows = 256
+    nb = Tcap // rows
+    gperm = torch.Generator().manual_seed(0)
+    perm = torch.randperm(Bd * nb, generator=gperm).to(dev)
+    Kp = torch.empty(Bd * nb, rows, Hkvd, Dd, dtype=Kc.dtype, device=dev)
+    Vp = torch.empty_like(Kp)
+    Kp[perm] = Kc.view(Bd * nb, rows, Hkvd, Dd)
+    Vp[perm] = Vc.view(Bd * nb, rows, Hkvd, Dd)
+    table = perm.view(Bd, nb).to(torch.int32)
+    qd = torch.randn(Bd, dc["Hq"], Dd, device=dev).to(torch.bfloat16)
+    pws = torch.empty(dca.dca_attn_decode_workspace(Bd, dc["Hq"], Dd, Tcap), dtype=torch.uint8,
+                      device=dev)
+    Opg = torch.empty_like(qd)
+    Lpg = torch.empty(Bd, dc["Hq"], dtype=torch.float32, device=dev)
+
+    def paged():
+        st = lib.dca_attn_decode_paged(P(qd.data_ptr()), P(Kp.data_ptr()), P(Vp.data_ptr()),
+                                       P(table.data_ptr()), nb, rows, Bd * nb,
+                                       P(t_dec.data_ptr()), P(Opg.data_ptr()), P(Lpg.data_ptr()),
+                                       Bd, dc["Hq"], Hkvd, Dd, dc["s"], dc["c"], dc["base"], 0.0,
+                                       P(pws.data_ptr()), pws.numel(), P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(paged, 10)
+    dbytes = W.decode_bytes(dc, t_dec.cpu().tolist())
+    out["decode_paged"] = {"value": dbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms": ms,
+                           "block_rows": rows, "launches_per_call": 2}
+    del Kp, Vp, pws
 
     # decode-time append of one token per sequence (positions t_dec + 1 < Tcap)
     Bd, Tcap, Hkvd, Dd = Kc.shape

@@ -271,6 +271,37 @@ dca_status_t dca_kv_append(const void* k_new, const void* v_new, void* Kcache, v
                            const int* t, int B, int Hkv, int D, int Tcap, int s, int c,
                            float base, void* stream);
 
+/* dca_attn_decode over a PAGED cache: keys and values live in pools
+ * Kpool, Vpool [num_blocks][block_rows][Hkv][D] bf16 (keys already rotated at
+ * j mod s), and sequence b's token j is row j % block_rows of physical block
+ * block_table[b * max_blocks + j / block_rows] (block_table int32 on the
+ * device, [B][max_blocks]).  block_rows must be a multiple of 64.  Same
+ * q, t, O, LSE, s, c, base, scale conventions as dca_attn_decode; the
+ * workspace is dca_attn_decode_workspace(B, Hq, D, max_blocks * block_rows)
+ * bytes.  A table entry outside [0, num_blocks) for a block the sequence
+ * reads is reported by dca_sync_status (INVALID_ARG) and read as zeros.
+ * Source: FlashDecoding over the cache (Guide, "Strategic Recommendations",
+ * item 3), with the cache in fixed-size blocks so a serving stack can grow
+ * and share sequences without copying.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_decode_paged(const void* q, const void* Kpool, const void* Vpool,
+                                   const int* block_table, int max_blocks, int block_rows,
+                                   int num_blocks, const int* t, void* O, float* LSE, int B,
+                                   int Hq, int Hkv, int D, int s, int c, float base, float scale,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* dca_kv_append into a paged cache: the new token of sequence b (unrotated
+ * key, value [B][Hkv][D]) is rotated at t[b] mod s and written to row
+ * t[b] % block_rows of block block_table[b * max_blocks + t[b] / block_rows]
+ * of Kpool / Vpool.  A t[b] outside [0, max_blocks * block_rows) or a table
+ * entry outside [0, num_blocks) is skipped and reported by dca_sync_status
+ * (INVALID_ARG).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+dca_status_t dca_kv_append_paged(const void* k_new, const void* v_new, void* Kpool, void* Vpool,
+                                 const int* block_table, int max_blocks, int block_rows,
+                                 int num_blocks, const int* t, int B, int Hkv, int D, int s,
+                                 int c, float base, void* stream);
+
 /* dca_attn_decode for callers that cannot allocate device memory (e.g. a
  * plugin inside a serving framework whose allocator owns the GPU's memory, or
  * a decode loop that must avoid cudaMalloc's implicit synchronisation).  Same

@@ -27,6 +27,7 @@ __all__ = [
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
+    "dca_attn_decode_paged", "dca_kv_append_paged",
     "dca_attn_decode_workspace", "dca_attn_decode", "dca_attn_decode_noalloc", "dca_kv_append",
     "dca_debug_index_map", "dca_debug_wait_timeout",
     "dca_sync_status", "dca_last_error_string", "EXPORTED_SYMBOLS",
@@ -53,6 +54,10 @@ _SIGS = {
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "dca_selfextend_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "dca_attn_prefill_host_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "dca_attn_decode_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _I, _I, _I, _I,
+                                   _I, _F, _F, _P, _Z, _P]),
+    "dca_kv_append_paged": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I, _I, _F,
+                                 _P]),
     "dca_attn_prefill_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I,
                                    _P, _Z, _P]),
     "dca_attn_prefill_selfextend": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F,
@@ -342,6 +347,45 @@ def dca_kv_append(k_new, v_new, Kcache, Vcache, t, s, c, base=10000.0):
     B, Hkv, D = k_new.shape
     _check(lib().dca_kv_append(_ptr(k_new), _ptr(v_new), _ptr(Kcache), _ptr(Vcache), _ptr(t), B,
                                Hkv, D, Kcache.shape[1], s, c, base, _stream(k_new)))
+
+
+def dca_attn_decode_paged(q, Kpool, Vpool, block_table, t, s, c, base=10000.0, scale=0.0,
+                          workspace=None):
+    """Decode over paged pools Kpool, Vpool [num_blocks][block_rows][Hkv][D] with
+    block_table int32 [B][max_blocks] (device)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(Kpool, "Kpool", torch.bfloat16, 4)
+    _need(Vpool, "Vpool", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(t, "t", torch.int32, 1)
+    B, Hq, D = q.shape
+    num_blocks, block_rows, Hkv = Kpool.shape[0], Kpool.shape[1], Kpool.shape[2]
+    max_blocks = block_table.shape[1]
+    if workspace is None:
+        workspace = _workspace(dca_attn_decode_workspace(B, Hq, D, max_blocks * block_rows),
+                               q.device)
+    O = torch.empty_like(q)
+    LSE = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check(lib().dca_attn_decode_paged(_ptr(q), _ptr(Kpool), _ptr(Vpool), _ptr(block_table),
+                                       max_blocks, block_rows, num_blocks, _ptr(t), _ptr(O),
+                                       _ptr(LSE), B, Hq, Hkv, D, s, c, base, scale,
+                                       _ptr(workspace), workspace.numel(), _stream(q)))
+    return O, LSE
+
+
+def dca_kv_append_paged(k_new, v_new, Kpool, Vpool, block_table, t, s, c, base=10000.0):
+    """Append one token per sequence into paged pools (in place)."""
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(Kpool, "Kpool", torch.bfloat16, 4)
+    _need(Vpool, "Vpool", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(t, "t", torch.int32, 1)
+    B, Hkv, D = k_new.shape
+    _check(lib().dca_kv_append_paged(_ptr(k_new), _ptr(v_new), _ptr(Kpool), _ptr(Vpool),
+                                     _ptr(block_table), block_table.shape[1], Kpool.shape[1],
+                                     Kpool.shape[0], _ptr(t), B, Hkv, D, s, c, base,
+                                     _stream(k_new)))
 
 
 def dca_attn_decode_noalloc(q, Kcache, Vcache, t, s, c, base=10000.0, scale=0.0, O=None,

@@ -54,7 +54,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __nv_bfloat16* __restrict__ q, const int* __restrict__ t, float* __restrict__ Opart,
     float* __restrict__ MLpart, int Hq, int Hkv, int Tcap, int s, int c, double log2_base,
-    float scale_log2, int nsplit_max, int n_hg) {
+    float scale_log2, int nsplit_max, int n_hg, const int* __restrict__ block_table,
+    int max_blocks, int block_rows, int num_blocks) {
   using SM = DecSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -149,10 +150,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         mbar_arrive_expect_tx(fb, SM::kStageBytes);
         const uint32_t dst = ring + st * SM::kStageBytes;
         const int key0 = k_begin + it * kDecKeys;
+        // contiguous cache: (row key0, sequence b); paged cache: the tile lies
+        // in one block (block_rows % 64 == 0), fetched from its physical slot
+        int row = key0, z = b;
+        if (block_table != nullptr) {
+          row = key0 % block_rows;
+          z = block_table[(size_t)b * max_blocks + key0 / block_rows];
+          if (z < 0 || z >= num_blocks) {  // reported; TMA fills the tile with zeros
+            report_error(kDevBadArg, 103);
+            z = num_blocks;
+          }
+        }
 #pragma unroll
         for (int hf = 0; hf < SM::kHalves; ++hf) {
-          tma_load_4d(dst + hf * kBoxBytes, &tmK, fb, hf * 64, hk, key0, b);
-          tma_load_4d(dst + (SM::kHalves + hf) * kBoxBytes, &tmV, fb, hf * 64, hk, key0, b);
+          tma_load_4d(dst + hf * kBoxBytes, &tmK, fb, hf * 64, hk, row, z);
+          tma_load_4d(dst + (SM::kHalves + hf) * kBoxBytes, &tmV, fb, hf * 64, hk, row, z);
         }
       }
     }
@@ -343,14 +355,21 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const float* __restrict
   if (d == 0) LSE[(size_t)b * Hq + h] = (M + log2f(lsum)) * 0.69314718055994530942f;
 }
 
+// Contiguous caches [B][Tcap][Hkv][D] (block_table null), or paged pools
+// [num_blocks][block_rows][Hkv][D] addressed through block_table [B][max_blocks]
+// (Tcap = max_blocks * block_rows).
 template <int D>
 cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const int* t, void* O,
                             float* LSE, int B, int Hq, int Hkv, int Tcap, int s, int c,
-                            float base, float scale, void* workspace, cudaStream_t stream) {
+                            float base, float scale, void* workspace, cudaStream_t stream,
+                            const int* block_table, int max_blocks, int block_rows,
+                            int num_blocks) {
   CUtensorMap tmK, tmV;
-  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Tcap, (uint64_t)B};
-  const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
-                               (uint64_t)Tcap * Hkv * D * 2};
+  const bool paged = block_table != nullptr;
+  const uint64_t rows = paged ? (uint64_t)block_rows : (uint64_t)Tcap;
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, rows,
+                            paged ? (uint64_t)num_blocks : (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2, rows * Hkv * D * 2};
   const uint32_t box[4] = {64, 1, kDecKeys, 1};
   if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Kc, 4, dims, strides, box,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -370,7 +389,8 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
   kern<<<grid, kDecThreads, smem, stream>>>(tmK, tmV, static_cast<const __nv_bfloat16*>(q), t,
                                             Opart, MLpart, Hq, Hkv, Tcap, s, c,
                                             log2((double)base),
-                                            scale * 1.4426950408889634f, nsplit, n_hg);
+                                            scale * 1.4426950408889634f, nsplit, n_hg,
+                                            block_table, max_blocks, block_rows, num_blocks);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<D><<<dim3(Hq, B), D, 0, stream>>>(
@@ -394,9 +414,26 @@ cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const i
   if (B == 0 || Hq == 0) return cudaSuccess;
   if (D == 64)
     return launch_decode_t<64>(q, Kc, Vc, t, O, LSE, B, Hq, Hkv, Tcap, s, c, base, scale,
-                               workspace, stream);
+                               workspace, stream, nullptr, 0, 0, 0);
   return launch_decode_t<128>(q, Kc, Vc, t, O, LSE, B, Hq, Hkv, Tcap, s, c, base, scale,
-                              workspace, stream);
+                              workspace, stream, nullptr, 0, 0, 0);
+}
+
+cudaError_t launch_decode_paged(const void* q, const void* Kpool, const void* Vpool,
+                                const int* block_table, int max_blocks, int block_rows,
+                                int num_blocks, const int* t, void* O, float* LSE, int B, int Hq,
+                                int Hkv, int D, int s, int c, float base, float scale,
+                                void* workspace, cudaStream_t stream) {
+  using namespace dec_path;
+  if (B == 0 || Hq == 0) return cudaSuccess;
+  const int Tcap = max_blocks * block_rows;
+  if (D == 64)
+    return launch_decode_t<64>(q, Kpool, Vpool, t, O, LSE, B, Hq, Hkv, Tcap, s, c, base, scale,
+                               workspace, stream, block_table, max_blocks, block_rows,
+                               num_blocks);
+  return launch_decode_t<128>(q, Kpool, Vpool, t, O, LSE, B, Hq, Hkv, Tcap, s, c, base, scale,
+                              workspace, stream, block_table, max_blocks, block_rows,
+                              num_blocks);
 }
 
 }  // namespace dca

@@ -121,8 +121,8 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_attn_mma_kernel(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_qt = (L + kBM - 1) / kBM;
-  const int qt = num_qt - 1 - (int)blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int qt = num_qt - 1 - (int)blockIdx.z;  // longest rows of every head first
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0 = qt * kBM;
   const size_t plane = (size_t)B * L * Hq * D;
@@ -344,7 +344,7 @@ cudaError_t launch_mma(const void* Qrot, const void* Krot, const void* V, void* 
   auto kern = prefill_attn_mma_kernel<D, Rule>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((L + kBM - 1) / kBM, Hq, B);
+  dim3 grid(Hq, B, (L + kBM - 1) / kBM);
   const float scale_log2 = scale * 1.4426950408889634f;
   kern<<<grid, kThreads, smem, stream>>>(
       static_cast<const __half*>(Qrot), static_cast<const __half*>(Krot),

@@ -197,8 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_qt = (L + kTile - 1) / kTile;
   const int num_pairs = (num_qt + 1) / 2;
-  const int m = num_pairs - 1 - (int)blockIdx.x;  // longest pairs first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // pairs are the slowest grid dimension: the longest pairs of every (head,
+  // sequence) are dispatched first
+  const int m = num_pairs - 1 - (int)blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0_loc = m * 2 * kTile;          // row of this call
   const int last_row = q_off + L - 1;        // absolute
@@ -533,7 +535,7 @@ cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* 
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
   if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
-  dim3 grid((num_qt + 1) / 2, Hq, B);
+  dim3 grid(Hq, B, (num_qt + 1) / 2);
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, rule, scale * 1.4426950408889634f,
                                              q_off);

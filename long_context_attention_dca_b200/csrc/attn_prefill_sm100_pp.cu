@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   // Pair m covers absolute rows m*256 .. m*256+255; the call's query row r
   // has absolute index pair_off*256 + r (pair_off > 0 for a chunk appended to
   // a cache).
-  const int m = num_pairs - 1 - (int)blockIdx.x + pair_off;  // longest pairs first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // pairs are the slowest grid dimension: the longest pairs of every (head,
+  // sequence) are dispatched first
+  const int m = num_pairs - 1 - (int)blockIdx.z + pair_off;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int hk = h / (Hq / Hkv);
   const int q0 = m * 2 * kTile;              // absolute
   const int q0_loc = q0 - pair_off * 2 * kTile;
@@ -385,7 +387,7 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
   if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
-  dim3 grid((num_qt + 1) / 2, Hq, B);
+  dim3 grid(Hq, B, (num_qt + 1) / 2);
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
                                              q_off / (2 * kTile));

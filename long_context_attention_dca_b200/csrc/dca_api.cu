@@ -58,6 +58,10 @@ dca_status_t check_heads(const char* fn, int B, int L, int Hq, int Hkv, int D) {
   if (Hq % Hkv != 0)
     return fail(DCA_ERR_UNSUPPORTED, "%s: Hq=%d is not a multiple of Hkv=%d", fn, Hq, Hkv);
   if (D != 64 && D != 128) return fail(DCA_ERR_UNSUPPORTED, "%s: D=%d (need 64 or 128)", fn, D);
+  // grid limits of the prefill launches: sequences on grid y, 64-row query
+  // tiles on grid z (both at most 65535)
+  if (B > 65535 || L > 65535 * 64)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: B=%d or L=%d beyond the launch grid", fn, B, L);
   return DCA_OK;
 }
 
@@ -401,6 +405,73 @@ dca_status_t dca_kv_append(const void* k_new, const void* v_new, void* Kcache, v
   if (t == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: t is null", fn);
   cudaError_t e = launch_kv_append(k_new, v_new, Kcache, Vcache, t, B, Hkv, D, Tcap, s, base,
                                    static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+namespace {
+dca_status_t check_paged(const char* fn, const int* block_table, int max_blocks, int block_rows,
+                         int num_blocks) {
+  if (block_table == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: block_table is null", fn);
+  if (max_blocks < 1 || num_blocks < 1)
+    return fail(DCA_ERR_INVALID_ARG, "%s: max_blocks=%d num_blocks=%d", fn, max_blocks,
+                num_blocks);
+  if (block_rows < 64 || block_rows % 64 != 0)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: block_rows=%d (need a multiple of 64)", fn,
+                block_rows);
+  if ((long long)max_blocks * block_rows > (1ll << 30))
+    return fail(DCA_ERR_INVALID_ARG, "%s: max_blocks * block_rows too large", fn);
+  return DCA_OK;
+}
+}  // namespace
+
+dca_status_t dca_attn_decode_paged(const void* q, const void* Kpool, const void* Vpool,
+                                   const int* block_table, int max_blocks, int block_rows,
+                                   int num_blocks, const int* t, void* O, float* LSE, int B,
+                                   int Hq, int Hkv, int D, int s, int c, float base, float scale,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_decode_paged";
+  dca_status_t st = check_heads(fn, B, 1, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st == DCA_OK) st = check_paged(fn, block_table, max_blocks, block_rows, num_blocks);
+  if (st != DCA_OK) return st;
+  if (B == 0) return DCA_OK;
+  DCA_CHECK_PTR(q);
+  DCA_CHECK_PTR(Kpool);
+  DCA_CHECK_PTR(Vpool);
+  if (t == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: t is null", fn);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = decode_workspace_bytes(B, Hq, D, max_blocks * block_rows);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes,
+                need);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaError_t e = launch_decode_paged(q, Kpool, Vpool, block_table, max_blocks, block_rows,
+                                      num_blocks, t, O, LSE, B, Hq, Hkv, D, s, c, base, sc,
+                                      workspace, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+dca_status_t dca_kv_append_paged(const void* k_new, const void* v_new, void* Kpool, void* Vpool,
+                                 const int* block_table, int max_blocks, int block_rows,
+                                 int num_blocks, const int* t, int B, int Hkv, int D, int s,
+                                 int c, float base, void* stream) {
+  const char* fn = "dca_kv_append_paged";
+  dca_status_t st = check_heads(fn, B, 1, Hkv, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st == DCA_OK) st = check_paged(fn, block_table, max_blocks, block_rows, num_blocks);
+  if (st != DCA_OK) return st;
+  if (B == 0) return DCA_OK;
+  DCA_CHECK_PTR(k_new);
+  DCA_CHECK_PTR(v_new);
+  DCA_CHECK_PTR(Kpool);
+  DCA_CHECK_PTR(Vpool);
+  if (t == nullptr) return fail(DCA_ERR_INVALID_ARG, "%s: t is null", fn);
+  cudaError_t e = launch_kv_append(k_new, v_new, Kpool, Vpool, t, B, Hkv, D,
+                                   max_blocks * block_rows, s, base,
+                                   static_cast<cudaStream_t>(stream), block_table, max_blocks,
+                                   block_rows, num_blocks);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 

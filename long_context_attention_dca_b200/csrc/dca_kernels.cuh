@@ -79,16 +79,27 @@ cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Ks
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
                                int out_rows, int Hkv, int D, cudaStream_t stream);
 
-// Decode-time append of one token per sequence into pre-rotated caches.
+// Decode-time append of one token per sequence into pre-rotated caches:
+// contiguous [B][Tcap][Hkv][D] (block_table null) or a paged pool
+// [num_blocks][block_rows][Hkv][D] through block_table [B][max_blocks]
+// (Tcap = max_blocks * block_rows).
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, void* Vc,
                              const int* t, int B, int Hkv, int D, int Tcap, int s, float base,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const int* block_table = nullptr,
+                             int max_blocks = 0, int block_rows = 0, int num_blocks = 0);
 
 // Split-KV decode + LSE merge.
 size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap);
 cudaError_t launch_decode(const void* q, const void* Kc, const void* Vc, const int* t, void* O,
                           float* LSE, int B, int Hq, int Hkv, int D, int Tcap, int s, int c,
                           float base, float scale, void* workspace, cudaStream_t stream);
+// Decode over paged pools [num_blocks][block_rows][Hkv][D] (block_rows % 64 ==
+// 0) through block_table [B][max_blocks].
+cudaError_t launch_decode_paged(const void* q, const void* Kpool, const void* Vpool,
+                                const int* block_table, int max_blocks, int block_rows,
+                                int num_blocks, const int* t, void* O, float* LSE, int B, int Hq,
+                                int Hkv, int D, int s, int c, float base, float scale,
+                                void* workspace, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout(int deadline_us, cudaStream_t stream);
 

@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
 __global__ void __launch_bounds__(256) kv_append_kernel(
     const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
     __nv_bfloat16* __restrict__ Kc, __nv_bfloat16* __restrict__ Vc, const int* __restrict__ t,
-    int B, int Hkv, int D, int Tcap, int s, double log2_base) {
+    int B, int Hkv, int D, int Tcap, int s, double log2_base, const int* __restrict__ block_table,
+    int max_blocks, int block_rows, int num_blocks) {
   const int groups = D / 16;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)B * Hkv * groups) return;
@@ -266,10 +267,21 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
     if (g == 0 && h == 0) report_error(kDevBadArg, 202);
     return;
   }
+  // physical row: sequence b's row tb, or row tb % block_rows of the block the
+  // table maps block tb / block_rows to
+  size_t prow = (size_t)b * Tcap + tb;
+  if (block_table != nullptr) {
+    const int blk = block_table[(size_t)b * max_blocks + tb / block_rows];
+    if (blk < 0 || blk >= num_blocks) {
+      if (g == 0 && h == 0) report_error(kDevBadArg, 203);
+      return;
+    }
+    prow = (size_t)blk * block_rows + tb % block_rows;
+  }
   CosSin8 cs;
   cos_sin_group(tb % s, g * 8, D, log2_base, cs);
   const size_t src = ((size_t)b * Hkv + h) * D + g * 8;
-  const size_t dst = (((size_t)b * Tcap + tb) * Hkv + h) * D + g * 8;
+  const size_t dst = (prow * Hkv + h) * D + g * 8;
   const uint4 lo = *reinterpret_cast<const uint4*>(k_new + src);
   const uint4 hi = *reinterpret_cast<const uint4*>(k_new + src + D / 2);
   uint4 olo, ohi;
@@ -399,14 +411,15 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
 namespace dca {
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, void* Vc,
                              const int* t, int B, int Hkv, int D, int Tcap, int s, float base,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const int* block_table, int max_blocks,
+                             int block_rows, int num_blocks) {
   using namespace rope_path;
   const long long total = (long long)B * Hkv * (D / 16);
   if (total == 0) return cudaSuccess;
   kv_append_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), t, B, Hkv, D, Tcap, s,
-      log2((double)base));
+      log2((double)base), block_table, max_blocks, block_rows, num_blocks);
   return cudaGetLastError();
 }
 }  // namespace dca

@@ -137,6 +137,15 @@ def test_argument_errors_return_codes(lib):
                                             0.0, ws, 1 << 30, None)) == 1
     assert _code(lib.dca_attn_prefill_chunk(*cargs, 1, 64, 4, 2, 128, 64, 128, 16, 32, 1e4,
                                             0.0, ws, 64, None)) == 5
+    # paged decode / append: null table, block_rows not a multiple of 64
+    assert _code(lib.dca_attn_decode_paged(fake, fake, fake, None, 4, 64, 8, fake, fake, fake, 2,
+                                           8, 1, 128, 64, 96, 1e4, 0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_decode_paged(fake, fake, fake, fake, 4, 96, 8, fake, fake, fake, 2,
+                                           8, 1, 128, 64, 96, 1e4, 0.0, ws, 1 << 30, None)) == 2
+    assert _code(lib.dca_attn_decode_paged(fake, fake, fake, fake, 4, 64, 8, fake, fake, fake, 2,
+                                           8, 1, 128, 64, 96, 1e4, 0.0, ws, 8, None)) == 5
+    assert _code(lib.dca_kv_append_paged(fake, fake, fake, fake, fake, 4, 100, 8, fake, 2, 1,
+                                         128, 64, 96, 1e4, None)) == 2
     # host prefill: chunk_rows < 1, null host buffer, short workspace
     hargs = (fake,) * 5
     assert _code(lib.dca_attn_prefill_host(*hargs, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, 0, ws,

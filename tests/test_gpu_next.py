@@ -388,3 +388,79 @@ def test_host_prefill_workload_equals_device_prefill():
     O1, L1 = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), cfg["s"], cfg["c"])
     dca.dca_sync_status()
     assert torch.equal(O, O1.cpu()) and torch.equal(LSE, L1.cpu())
+
+
+# ---------------------------------------------------------------------------
+# paged KV cache: decode and append through a block table
+# ---------------------------------------------------------------------------
+
+def _to_pool(Kc, block_rows, extra, seed):
+    """Scatter a contiguous cache [B][Tcap][H][D] into a pool of blocks in a
+    random physical order; returns (pool, block_table int32 [B][Tcap/block_rows])."""
+    B, Tcap, H, D = Kc.shape
+    nb = Tcap // block_rows
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(B * nb + extra, generator=g)[:B * nb].view(B, nb).to(torch.int32)
+    pool = torch.zeros(B * nb + extra, block_rows, H, D, dtype=Kc.dtype, device=Kc.device)
+    for b in range(B):
+        for k in range(nb):
+            pool[int(perm[b, k])] = Kc[b, k * block_rows:(k + 1) * block_rows]
+    return pool, perm.to(Kc.device)
+
+
+@pytest.mark.parametrize("block_rows", [64, 256])
+def test_paged_decode_equals_contiguous_decode(block_rows):
+    dc = W.scaled(W.CONFIGS["decode_b16"], B=3, Tcap=4096, t_lo=100, t_hi=4096)
+    t, q, Kc, Vc = W.make_decode_inputs(dc, device="cuda")
+    s, c = dc["s"], dc["c"]
+    Kp, table = _to_pool(Kc, block_rows, 7, 1)
+    Vp, _ = _to_pool(Vc, block_rows, 7, 1)
+    O1, L1 = dca.dca_attn_decode(q, Kc, Vc, t, s, c)
+    O2, L2 = dca.dca_attn_decode_paged(q, Kp, Vp, table, t, s, c)
+    dca.dca_sync_status()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+def test_paged_append_then_decode_matches_contiguous():
+    B, Hq, Hkv, D, T, s, c, rows = 2, 16, 2, 128, 1024, 256, 384, 128
+    gen = torch.Generator().manual_seed(17)
+    K = torch.randn(B, T, Hkv, D, generator=gen).to(torch.bfloat16).cuda()
+    V = torch.randn(B, T, Hkv, D, generator=gen).to(torch.bfloat16).cuda()
+    Q = torch.randn(B, T, Hq, D, generator=gen).to(torch.bfloat16).cuda()
+    Kc = torch.zeros(B, T, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    Vc = torch.zeros_like(Kc)
+    Kp, table = _to_pool(Kc, rows, 3, 2)
+    Vp = torch.zeros_like(Kp)
+    for tt in range(0, 700):
+        t = torch.full((B,), tt, dtype=torch.int32, device="cuda")
+        dca.dca_kv_append(K[:, tt].contiguous(), V[:, tt].contiguous(), Kc, Vc, t, s, c)
+        dca.dca_kv_append_paged(K[:, tt].contiguous(), V[:, tt].contiguous(), Kp, Vp, table, t,
+                                s, c)
+    t = torch.tensor([699, 450], dtype=torch.int32, device="cuda")
+    O1, L1 = dca.dca_attn_decode(Q[:, 699].contiguous(), Kc, Vc, t, s, c)
+    O2, L2 = dca.dca_attn_decode_paged(Q[:, 699].contiguous(), Kp, Vp, table, t, s, c)
+    dca.dca_sync_status()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+    # every appended row sits in its mapped block
+    for b in range(B):
+        for tt in (0, 127, 128, 699):
+            blk = int(table[b, tt // rows])
+            assert torch.equal(Kp[blk, tt % rows], Kc[b, tt])
+
+
+def test_paged_table_out_of_range_is_reported():
+    B, Hq, Hkv, D, rows = 1, 8, 1, 128, 64
+    Kp = torch.zeros(4, rows, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    Vp = torch.zeros_like(Kp)
+    table = torch.tensor([[0, 9]], dtype=torch.int32, device="cuda")  # block 9 does not exist
+    q = torch.ones(B, Hq, D, dtype=torch.bfloat16, device="cuda")
+    t = torch.tensor([100], dtype=torch.int32, device="cuda")
+    dca.dca_attn_decode_paged(q, Kp, Vp, table, t, 64, 96)
+    with pytest.raises(dca.DcaError) as ei:
+        dca.dca_sync_status()
+    assert ei.value.status == 1
+    dca.dca_sync_status()  # cleared; the context keeps working
+    t = torch.tensor([50], dtype=torch.int32, device="cuda")
+    O, L = dca.dca_attn_decode_paged(q, Kp, Vp, table, t, 64, 96)
+    dca.dca_sync_status()
+    assert torch.isfinite(L).all()
