@@ -69,10 +69,10 @@ typedef enum dca_pos_rule {
 } dca_pos_rule_t;
 
 typedef enum dca_prefill_path {
-  DCA_PATH_AUTO = 0,    /* tcgen05 path when D == 128, else warp MMA        */
+  DCA_PATH_AUTO = 0,    /* the tcgen05 path                                  */
   DCA_PATH_GENERAL = 1, /* warp-MMA path: any s, D 64 or 128                */
-  DCA_PATH_TCGEN05 = 2  /* tcgen05/TMEM/TMA path: D == 128 (any s; tiles that
-                           straddle chunk boundaries are masked per row)    */
+  DCA_PATH_TCGEN05 = 2  /* tcgen05/TMEM/TMA path: D 64 or 128, any s (tiles
+                           straddling chunk boundaries are masked per row) */
 } dca_prefill_path_t;
 
 /* Rotate x [B][L][H][D] (bf16) into out (same shape; may equal x) with
@@ -166,10 +166,9 @@ size_t dca_attn_prefill_chunk_workspace(int B, int Lq, int Hq, int Hkv, int D, i
  *   O [B][Lq][Hq][D] bf16 and LSE [B][Hq][Lq] fp32: results for the chunk.
  *   t0 (host int) is the same for every sequence; 0 <= t0, t0 + Lq <= Tcap.
  * The call owns no memory; `workspace` (dca_attn_prefill_chunk_workspace
- * bytes, 256-byte aligned) is scratch for the call's duration.  Kernels: at
- * D == 128 a tcgen05 kernel with the query offset (the two-tile kernel when
- * s % 256 == 0 and t0 % 256 == 0, the per-row-interval kernel otherwise); the
- * warp-MMA kernel at D == 64.
+ * bytes, 256-byte aligned) is scratch for the call's duration.  Kernels: a
+ * tcgen05 kernel with the query offset (the two-tile kernel when D == 128,
+ * s % 256 == 0 and t0 % 256 == 0, the per-row-interval kernel otherwise).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V, void* Kcache,
                                     void* Vcache, void* O, float* LSE, int B, int Lq, int Hq,
@@ -193,10 +192,9 @@ size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D);
  * grouped distance >= W, above all neighbour distances.  G = 1 or W >= L is
  * plain RoPE attention.  Same tensors and conventions as dca_attn_prefill
  * (Q, K unrotated bf16; O bf16; LSE fp32 [B][Hq][L]); any G >= 1, W >= 1,
- * D in {64, 128}.  Kernels: at D == 128 the per-row-interval tcgen05 kernel
- * (each row's neighbour keys [i-W+1, i] and grouped keys [0, i-W] are two
- * intervals, visited with their own query and key rotations); the warp-MMA
- * kernel at D == 64.  `workspace`: dca_selfextend_workspace bytes, 256-byte
+ * D in {64, 128}.  Kernel: the per-row-interval tcgen05 kernel (each row's
+ * neighbour keys [i-W+1, i] and grouped keys [0, i-W] are two intervals,
+ * visited with their own query and key rotations).  `workspace`: dca_selfextend_workspace bytes, 256-byte
  * aligned, scratch for the call.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const void* V, void* O,
@@ -225,9 +223,9 @@ size_t dca_attn_prefill_host_workspace(int B, int L, int Hq, int Hkv, int D, int
  *     events and releases them before returning (they are freed once the
  *     queued work is done), so it cannot be captured into a CUDA graph.
  *     Work queued on `stream` after the call runs after the last copy out.
- *   - Kernels: tcgen05 at D == 128 (the two-tile kernel when s % 256 == 0
- *     and chunk_rows is a multiple of 256 or covers the sequence, the
- *     per-row-interval kernel otherwise); the warp-MMA kernel at D == 64.
+ *   - Kernels: tcgen05 (the two-tile kernel when D == 128, s % 256 == 0 and
+ *     chunk_rows is a multiple of 256 or covers the sequence, the
+ *     per-row-interval kernel otherwise).
  *   - `workspace`: dca_attn_prefill_host_workspace bytes of device memory.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_attn_prefill_host(const void* Q, const void* K, const void* V, void* O,

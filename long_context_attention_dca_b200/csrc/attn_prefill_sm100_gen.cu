@@ -34,9 +34,7 @@ namespace dca {
 namespace gen_path {
 
 constexpr int kTile = 128;
-constexpr int kHD = 128;
 constexpr int kBox = kTile * 64 * 2;   // [128 rows x 64 cols] 16-bit = 16 KB
-constexpr int kTileBytes = 2 * kBox;   // 32 KB
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 216;
@@ -44,18 +42,28 @@ constexpr int kControlRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allotment");
 constexpr int kNumQSlots = 3;
-constexpr int kSmQ = 0;
-constexpr int kSmK = kNumQSlots * kTileBytes;
-constexpr int kSmV = kSmK + 2 * kTileBytes;
-constexpr int kSmBar = kSmV + 2 * kTileBytes;
+// Shared-memory layout for head dimension D (64 or 128): a Q, K or V tile is
+// D/64 boxes of [128 rows x 64 columns].
+template <int D>
+struct Lay {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kHalves * kBox;
+  static constexpr int kSmQ = 0;
+  static constexpr int kSmK = kNumQSlots * kTileBytes;
+  static constexpr int kSmV = kSmK + 2 * kTileBytes;
+  static constexpr int kSmBar = kSmV + 2 * kTileBytes;
+};
 enum Bar {
   kQFull = 0, kQEmpty = 3, kKFull = 6, kKEmpty = 8, kVFull = 10, kVEmpty = 12,
   kSFull = 14, kPFull = 16, kODone = 18, kMmaEnd = 20, kNumBars = 21
 };
-constexpr int kSmMisc = kSmBar + kNumBars * 8;   // TMEM base, abort flag
-constexpr int kSmPlan = kSmMisc + 16;             // the CTA's visit plan
-constexpr int kSmTotal = kSmPlan + 128 + 1024;
-static_assert(kSmTotal <= 232448, "shared memory budget");
+template <int D>
+struct Lay2 {
+  static constexpr int kSmMisc = Lay<D>::kSmBar + kNumBars * 8;  // TMEM base, abort flag
+  static constexpr int kSmPlan = kSmMisc + 16;                    // the CTA's visit plan
+  static constexpr int kSmTotal = kSmPlan + 128 + 1024;
+  static_assert(kSmTotal <= 232448, "shared memory budget");
+};
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -180,12 +188,17 @@ __device__ __forceinline__ float row_max_range(uint32_t (&v)[4][32], int clo, in
   return row_max(v);
 }
 
-template <class Rule>
+template <int D, class Rule>
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
-    int q_off) {
+    int q_off, int group_units) {
+  using LD = Lay<D>;
+  constexpr int kHalves = LD::kHalves, kTileBytes = LD::kTileBytes;
+  constexpr int kSmQ = LD::kSmQ, kSmK = LD::kSmK, kSmV = LD::kSmV, kSmBar = LD::kSmBar;
+  constexpr int kSmMisc = Lay2<D>::kSmMisc, kSmPlan = Lay2<D>::kSmPlan;
+  constexpr uint32_t kOCols = (uint32_t)D;  // O accumulator columns per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -197,10 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int num_qt = (L + kTile - 1) / kTile;
   const int num_pairs = (num_qt + 1) / 2;
-  // pairs are the slowest grid dimension: the longest pairs of every (head,
-  // sequence) are dispatched first
-  const int m = num_pairs - 1 - (int)blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
+  // longest pairs first over all (sequence, kv head) units (one group: with
+  // L2-sized groups the longer, uneven visits of this kernel left a tail)
+  const PairOrder po = pair_order((int)blockIdx.x, num_pairs, Hq, Hkv, B, group_units);
+  const int m = num_pairs - 1 - po.m_rank;
+  const int h = po.h, b = po.b;
   const int hk = h / (Hq / Hkv);
   const int q0_loc = m * 2 * kTile;          // row of this call
   const int last_row = q_off + L - 1;        // absolute
@@ -259,8 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
         mbar_arrive_expect_tx(fb, kTileBytes);
         const uint32_t dst = sbase + kSmQ + slot * kTileBytes;
         const int row = q0_loc + x * kTile;
-        tma_load_4d(dst, &tmQ, fb, 0, h, row, piece * B + b);
-        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, piece * B + b);
+#pragma unroll
+        for (int hf = 0; hf < kHalves; ++hf)
+          tma_load_4d(dst + hf * kBox, &tmQ, fb, hf * 64, h, row, piece * B + b);
         q_last[slot] = n;
         return true;
       };
@@ -277,8 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
           mbar_arrive_expect_tx(bar(kKFull + sg), kTileBytes);
           const uint32_t kd = sbase + kSmK + sg * kTileBytes;
           const int kb = rule.kplane(pl.pc[k]) * B + b;  // key plane of the piece
-          tma_load_4d(kd, &tmK, bar(kKFull + sg), 0, hk, t * kTile, kb);
-          tma_load_4d(kd + kBox, &tmK, bar(kKFull + sg), 64, hk, t * kTile, kb);
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_4d(kd + hf * kBox, &tmK, bar(kKFull + sg), hf * 64, hk, t * kTile, kb);
           k_last[sg] = st;
           if (first && !(ok = load_q(2 * k + 1, pl.pc[k]))) break;
           if (st >= 2 &&
@@ -286,8 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
             break;
           mbar_arrive_expect_tx(bar(kVFull + sg), kTileBytes);
           const uint32_t vd = sbase + kSmV + sg * kTileBytes;
-          tma_load_4d(vd, &tmV, bar(kVFull + sg), 0, hk, t * kTile, b);
-          tma_load_4d(vd + kBox, &tmV, bar(kVFull + sg), 64, hk, t * kTile, b);
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk, t * kTile, b);
           v_last[sg] = st;
         }
       }
@@ -304,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc(128, 128, /*bf16=*/false, 0, 0);  // fp16 Q, K
-      const uint32_t idesc_o = umma_idesc(128, 128, /*bf16=*/true, 0, 1);   // bf16 P, V
+      const uint32_t idesc_o = umma_idesc(128, D, /*bf16=*/true, 0, 1);     // bf16 P, V
       const uint64_t dq0 = smem_desc_sw128(sbase + kSmQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + kSmK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + kSmV, kBox, 1024);
@@ -319,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
         const uint64_t dk = dk0 + (uint64_t)(st & 1) * kTileU;
         const uint32_t d = tmem + 128u * (uint32_t)x;
 #pragma unroll
-        for (int kk = 0; kk < kHD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
           umma_ss(d, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
@@ -433,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
           const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
           l_run *= alpha;
 #pragma unroll 1
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < (int)kOCols / 32; ++q) {
             uint32_t o[32];
             tmem_ld32(o_addr + 32u * q, o);
             tmem_wait_ld();
@@ -460,9 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
       tc_fence_after();
       const bool valid = i_row < L;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = O + (((size_t)b * L + (valid ? i_row : 0)) * Hq + h) * kHD;
+      __nv_bfloat16* orow = O + (((size_t)b * L + (valid ? i_row : 0)) * Hq + h) * D;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < (int)kOCols / 32; ++q) {
         uint32_t o[32];
         tmem_ld32(o_addr + 32u * q, o);
         tmem_wait_ld();
@@ -497,11 +514,11 @@ namespace gen_path {
 
 // Tensor maps and launch: Qrot [nq planes][B][L][Hq][D] and Krot [kKPlanes]
 // [B][k_rows][Hkv][D] fp16, V [B][v_rows][Hkv][D] bf16.
-template <class Rule>
-cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
-                       int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
-                       cudaStream_t stream, int q_off, int k_rows, int v_rows) {
-  if (D != kHD || q_off < 0) return cudaErrorInvalidValue;
+template <int D, class Rule>
+cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
+                         int B, int L, int Hq, int Hkv, Rule rule, int nq, float scale,
+                         cudaStream_t stream, int q_off, int k_rows, int v_rows) {
+  if (q_off < 0) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
   const int Lkv = q_off + L;
   if (k_rows == 0) k_rows = Lkv;
@@ -530,16 +547,30 @@ cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* 
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  auto kern = prefill_attn_gen_kernel<Rule>;
+  constexpr int kSmTotal = Lay2<D>::kSmTotal;
+  auto kern = prefill_attn_gen_kernel<D, Rule>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
   if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
-  dim3 grid(Hq, B, (num_qt + 1) / 2);
+  dim3 grid((unsigned)(((num_qt + 1) / 2) * Hq * B));
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, rule, scale * 1.4426950408889634f,
-                                             q_off);
+                                             q_off, B * Hkv);  // one group: longest first
   return cudaGetLastError();
+}
+
+template <class Rule>
+cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
+                       int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
+                       cudaStream_t stream, int q_off, int k_rows, int v_rows) {
+  if (D == 64)
+    return launch_gen_d<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream, q_off,
+                            k_rows, v_rows);
+  if (D == 128)
+    return launch_gen_d<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream,
+                             q_off, k_rows, v_rows);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace gen_path

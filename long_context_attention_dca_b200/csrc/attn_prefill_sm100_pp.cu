@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2,
-    int pair_off) {
+    int pair_off, int group_units) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -79,10 +79,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   // Pair m covers absolute rows m*256 .. m*256+255; the call's query row r
   // has absolute index pair_off*256 + r (pair_off > 0 for a chunk appended to
   // a cache).
-  // pairs are the slowest grid dimension: the longest pairs of every (head,
-  // sequence) are dispatched first
-  const int m = num_pairs - 1 - (int)blockIdx.z + pair_off;
-  const int h = blockIdx.x, b = blockIdx.y;
+  // longest pairs first within L2-sized groups of (sequence, kv head) units
+  const PairOrder po = pair_order((int)blockIdx.x, num_pairs, Hq, Hkv, B, group_units);
+  const int m = num_pairs - 1 - po.m_rank + pair_off;
+  const int h = po.h, b = po.b;
   const int hk = h / (Hq / Hkv);
   const int q0 = m * 2 * kTile;              // absolute
   const int q0_loc = q0 - pair_off * 2 * kTile;
@@ -387,10 +387,11 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
   if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
-  dim3 grid(Hq, B, (num_qt + 1) / 2);
+  dim3 grid((unsigned)(((num_qt + 1) / 2) * Hq * B));
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
-                                             q_off / (2 * kTile));
+                                             q_off / (2 * kTile),
+                                             pair_group_units(B, Hkv, Lkv, D));
   return cudaGetLastError();
 }
 

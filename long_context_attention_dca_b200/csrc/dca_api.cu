@@ -80,12 +80,12 @@ PrefillWs prefill_ws_layout(void* base, int B, int L, int Hq, int Hkv, int D) {
   return PrefillWs{p, p ? p + qbytes : nullptr, qbytes + kbytes};
 }
 
-// tcgen05 kernels at D = 128 for every chunk size: the two-tile ping-pong
-// kernel when s % 256 == 0 (no tile straddles a chunk), the per-row-interval
-// kernel otherwise; the warp-MMA kernel for D = 64.
+// tcgen05 kernels for every chunk size and head dimension: the two-tile
+// ping-pong kernel when D == 128 and s % 256 == 0 (no tile straddles a chunk),
+// the per-row-interval kernel otherwise.
 int auto_path(int D, int s) {
   (void)s;
-  return (kHaveTcgen05 && D == 128) ? DCA_PATH_TCGEN05 : DCA_PATH_GENERAL;
+  return (kHaveTcgen05 && (D == 64 || D == 128)) ? DCA_PATH_TCGEN05 : DCA_PATH_GENERAL;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -193,8 +193,8 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   if (path < DCA_PATH_AUTO || path > DCA_PATH_TCGEN05)
     return fail(DCA_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
   if (path == DCA_PATH_AUTO) path = auto_path(D, s);
-  if (path == DCA_PATH_TCGEN05 && !(kHaveTcgen05 && D == 128))
-    return fail(DCA_ERR_UNSUPPORTED, "%s: tcgen05 path needs D == 128", fn);
+  if (path == DCA_PATH_TCGEN05 && !kHaveTcgen05)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: library built without the tcgen05 path", fn);
   if ((long long)B * L == 0) return DCA_OK;
   DCA_CHECK_PTR(V);
   DCA_CHECK_PTR(O);
@@ -207,7 +207,7 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (path == DCA_PATH_TCGEN05 && s % 256 == 0)
+  if (path == DCA_PATH_TCGEN05 && D == 128 && s % 256 == 0)
     e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
   else if (path == DCA_PATH_TCGEN05)  // tiles or tile pairs straddle chunk boundaries
     e = launch_prefill_attn_sm100_gen(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
@@ -304,7 +304,7 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
                                     t0, Tcap, t0 + Lq, s, c, base, strm);
   if (e == cudaSuccess) e = launch_keys_to_f16(Kcache, kf16, B, t0, Tcap, t0 + Lq, Hkv, D, strm);
   if (e != cudaSuccess) return cuda_fail(e, fn);
-  if (auto_path(D, s) == DCA_PATH_TCGEN05 && s % 256 == 0 && t0 % 256 == 0)
+  if (auto_path(D, s) == DCA_PATH_TCGEN05 && D == 128 && s % 256 == 0 && t0 % 256 == 0)
     e = launch_prefill_attn_sm100_pp(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
                                      strm, t0, t0 + Lq, Tcap);
   else if (auto_path(D, s) == DCA_PATH_TCGEN05)

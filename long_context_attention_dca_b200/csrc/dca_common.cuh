@@ -103,7 +103,47 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
-// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
+// Dispatch order of the two-tile prefill kernels' (query-tile pair, head,
+// sequence) work items, from a 1-D block index: the (sequence, kv head) units
+// are taken in groups of `k`, one group after another; within a group the
+// longest pairs come first (over all its q heads).  Longest-first keeps the
+// tail of the launch short; the groups keep the keys and values in flight
+// small enough to stay in L2.
+struct PairOrder {
+  int m_rank;  // 0 = the longest pair
+  int h, b;
+};
+__device__ __forceinline__ PairOrder pair_order(int idx, int num_pairs, int Hq, int Hkv, int B,
+                                                int k) {
+  const int G = Hq / Hkv, U = B * Hkv;
+  const int per_group = num_pairs * k * G;
+  const int n_groups = (U + k - 1) / k;
+  int gi = idx / per_group;
+  if (gi > n_groups - 1) gi = n_groups - 1;
+  const int kk = gi == n_groups - 1 ? U - gi * k : k;
+  const int off = idx - gi * per_group;
+  const int m_rank = off / (kk * G);
+  const int rem = off - m_rank * kk * G;
+  const int unit = gi * k + rem / G;
+  PairOrder o;
+  o.m_rank = m_rank;
+  o.b = unit / Hkv;
+  o.h = (unit % Hkv) * G + rem % G;
+  return o;
+}
+
+// Units per group so that one group's keys and values (fp16 + bf16, 4 bytes
+// per key and head dimension) take about half of the 126 MB L2.
+inline int pair_group_units(int B, int Hkv, int Lkv, int D) {
+  const long long per_unit = 4ll * Lkv * D;
+  long long k = (64ll << 20) / (per_unit > 0 ? per_unit : 1);
+  const long long U = (long long)B * Hkv;
+  if (k < 1) k = 1;
+  if (k > U) k = U;
+  return (int)k;
+}
+
+// Per-warpgroup register reallocation// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
 // the same one).  The counts used by a kernel must sum, over its warpgroups,
 // to no more than the registers the block was launched with.
 template <int N>

@@ -94,7 +94,7 @@ extern "C" dca_status_t dca_attn_prefill_host(const void* Q, const void* K, cons
   // pairs and no tile straddles a chunk; the per-row-interval tcgen05 kernel
   // for any other chunking at D = 128
   const bool tc = auto_path(D, s) == DCA_PATH_TCGEN05;
-  const bool pp = tc && s % 256 == 0 && (C % 256 == 0 || n_chunks == 1);
+  const bool pp = tc && D == 128 && s % 256 == 0 && (C % 256 == 0 || n_chunks == 1);
 
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t* ev = nullptr;  // [3][n_chunks]: copied in, computed, copied out

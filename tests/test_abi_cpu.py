@@ -75,7 +75,7 @@ def test_workspace_queries(lib):
 def test_prefill_path_selection(lib):
     assert dca.dca_prefill_path(16384, 128, 3072, 4096) in (dca.DCA_PATH_GENERAL,
                                                               dca.DCA_PATH_TCGEN05)
-    assert dca.dca_prefill_path(1024, 64, 192, 256) == dca.DCA_PATH_GENERAL
+    assert dca.dca_prefill_path(1024, 64, 192, 256) == dca.DCA_PATH_TCGEN05
     assert dca.dca_prefill_path(1024, 128, 192, 256) == dca.DCA_PATH_TCGEN05
     assert dca.dca_prefill_path(1024, 128, 300, 256) == 0  # s > c
     assert dca.dca_prefill_path(1024, 96, 128, 256) == 0
@@ -115,8 +115,8 @@ def test_argument_errors_return_codes(lib):
     assert "workspace" in dca.dca_last_error_string()
     assert _code(lib.dca_attn_prefill(*args, 1, 64, 4, 2, 128, 16, 32, 1e4, 0.0, None, 1 << 30,
                                       None)) == 1
-    # tcgen05 path on a head dimension it does not cover
-    assert _code(lib.dca_prefill_attention(fake, fake, fake, 1, 64, 4, 2, 64, 96, 128, 0.0,
+    # a head dimension no path covers
+    assert _code(lib.dca_prefill_attention(fake, fake, fake, 1, 64, 4, 2, 96, 96, 128, 0.0,
                                            2, ws, 1 << 30, None)) == 2
     assert _code(lib.dca_prefill_attention(fake, fake, fake, 1, 64, 4, 2, 128, 96, 128, 0.0,
                                            7, ws, 1 << 30, None)) == 1

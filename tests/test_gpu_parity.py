@@ -44,8 +44,8 @@ def _prefill_gpu(Q, K, V, s, c, path, base=10000.0):
 
 
 def _path_ok(path, D, s):
-    # the tcgen05 path takes every chunk size at D = 128 (straddling tiles masked)
-    return path == dca.DCA_PATH_GENERAL or D == 128
+    # the tcgen05 path takes every chunk size and both head dimensions
+    return path in (dca.DCA_PATH_GENERAL, dca.DCA_PATH_TCGEN05)
 
 
 # ---------------------------------------------------------------------------
@@ -119,15 +119,17 @@ def test_prefill_rope_workspace_planes():
 # prefill, small cases, every output
 # ---------------------------------------------------------------------------
 
-def test_prefill_tiny_workload_full():
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_tiny_workload_full(path):
     cfg = W.CONFIGS["tiny"]
     Q, K, V = W.make_prefill_inputs(cfg)
-    O, LSE = _prefill_gpu(Q, K, V, cfg["s"], cfg["c"], dca.DCA_PATH_GENERAL)
+    O, LSE = _prefill_gpu(Q, K, V, cfg["s"], cfg["c"], path)
     O_ref, LSE_ref = orc.dca_prefill(Q.float().numpy(), K.float().numpy(), V.float().numpy(),
                                      cfg["s"], cfg["c"], cfg["base"])
     err = np.abs(O.double().numpy() - O_ref)
     lse_rel = np.abs(LSE.double().numpy() - LSE_ref) / np.maximum(np.abs(LSE_ref), 1.0)
-    print(f"tiny: O max {err.max():.3e} mean {err.mean():.3e} LSE rel {lse_rel.max():.3e}")
+    print(f"tiny path {path}: O max {err.max():.3e} mean {err.mean():.3e} "
+          f"LSE rel {lse_rel.max():.3e}")
     pu.assert_close(err.max(), err.mean(), lse_rel.max(), "tiny")
 
 
