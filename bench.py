@@ -385,7 +385,7 @@ def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
     hOd = torch.empty(q_dec.shape, dtype=torch.bfloat16).pin_memory()
     hLd = torch.empty(q_dec.shape[:2], dtype=torch.float32).pin_memory()
     s, c = pc["s"], pc["c"]
-    chunk = 2048
+    chunk = args.e2e_chunk
     ws = torch.empty(dca.dca_attn_prefill_host_workspace(*Q.shape[:3], K.shape[2], Q.shape[3],
                                                          chunk), dtype=torch.uint8, device=dev)
     dws = torch.empty(dca.dca_attn_decode_workspace(*q_dec.shape[:2], q_dec.shape[2],
@@ -688,6 +688,8 @@ def main():
     ap.add_argument("--override-s", type=int, default=0,
                     help="profiling runs: chunk size s of the prefill workload (e.g. 3000, "
                          "whose tiles straddle chunk boundaries)")
+    ap.add_argument("--e2e-chunk", type=int, default=2048,
+                    help="rows per chunk of the host-buffer prefill in the e2e leg")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default=PREFILL, choices=sorted(
