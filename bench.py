@@ -194,7 +194,9 @@ def _cfg_summary(cfg):
 def run_ours(args, rank, world, dev):
     import long_context_attention_dca_b200 as dca
     from long_context_attention_dca_b200 import build
-    build.build()
+    if rank == 0:
+        build.build()  # (re)built once; the other ranks load it after the barrier
+    _barrier(world)
     lib = dca.lib()
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)

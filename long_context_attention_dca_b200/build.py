@@ -52,7 +52,7 @@ def up_to_date() -> bool:
 def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+    tmp = f"{LIB_PATH}.{os.getpid()}.tmp"  # concurrent builders never share a file
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, os.path.join(CSRC, "dca_lib.cu")]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
