@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
       const uint64_t dk0 = smem_desc_sw128(sbase + kSmK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + kSmV, kBox, 1024);
       constexpr uint64_t kTileU = kTileBytes >> 4;
-      int j_s[2] = {0, 0}, j_p[2] = {0, 0};  // S and PV issued per tile
+      int jp_a = 0, jp_b = 0;  // PV MMAs issued for tiles A and B
       // S_X of visit st (ring position st) with the query in slot q_slot
       auto issue_s = [&](int x, int st, int q_slot, bool wait_k) -> bool {
         if (wait_k && !mbar_wait(bar(kKFull + (st & 1)), (st >> 1) & 1, abort_flag, 491))
@@ -341,23 +341,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
           umma_ss(d, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(kSFull + x));
-        ++j_s[x];
         return true;
       };
       auto issue_pv = [&](int x, int st, bool wait_v) -> bool {
-        if (!mbar_wait(bar(kPFull + x), j_p[x] & 1, abort_flag, 492)) return false;
+        const int jp = x ? jp_b : jp_a;
+        if (!mbar_wait(bar(kPFull + x), jp & 1, abort_flag, 492)) return false;
         if (wait_v && !mbar_wait(bar(kVFull + (st & 1)), (st >> 1) & 1, abort_flag, 493))
           return false;
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)(st & 1) * kTileU;
         const uint32_t pa = tmem + 128u * (uint32_t)x;
         const uint32_t od = tmem + 256u + 128u * (uint32_t)x;
-        umma_ts(od, pa, dv, idesc_o, j_p[x] > 0 ? 1u : 0u);
+        umma_ts(od, pa, dv, idesc_o, jp > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < kTile / 16; ++kk)
           umma_ts(od, pa + 8u * (uint32_t)kk, dv + (uint64_t)((kk * 2048) >> 4), idesc_o, 1u);
         umma_commit(bar(kODone + x));
-        ++j_p[x];
+        if (x) ++jp_b;
+        else ++jp_a;
         return true;
       };
       bool ok = true;
