@@ -438,6 +438,8 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                      by LSE (dca_attn_prefill_3pass);
       prefill_selfextend  the prefill workload under the SelfExtend position
                      map, G = 8, W = 1024 (dca_attn_prefill_selfextend);
+      prefill_varlen a packed batch of eight Llama-2 7B prompts of mixed length
+                     (dca_attn_prefill_varlen, RoPE included);
       decode_paged   the decode workload over a paged copy of its caches
                      (dca_attn_decode_paged, 256-row blocks in random order);
       kv_append      one decoded token appended per sequence of the decode
@@ -580,6 +582,35 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                                      else "general (warp MMA)"),
                                  "launches_per_call": 2}
     del sws, Ose, Lse
+
+    # packed variable-length batch: Llama-2 7B heads, eight prompts of seeded
+    # lengths in [512, 16384] back to back (RoPE + attention in one call)
+    vc = W.CONFIGS["varlen_7b_mix"]
+    Qv, Kv, Vv, cu, lens = W.make_varlen_inputs(vc, device=dev)
+    cu_d = cu.to(dev)
+    Tv, Hqv, Dv = Qv.shape
+    Hkvv = Kv.shape[1]
+    wsz = dca.dca_attn_prefill_varlen_workspace(Tv, Hqv, Hkvv, Dv)
+    vws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    Ov = torch.empty_like(Qv)
+    Lv = torch.empty(Hqv, Tv, dtype=torch.float32, device=dev)
+
+    def varlen():
+        st = lib.dca_attn_prefill_varlen(P(Qv.data_ptr()), P(Kv.data_ptr()), P(Vv.data_ptr()),
+                                         P(Ov.data_ptr()), P(Lv.data_ptr()), P(cu_d.data_ptr()),
+                                         len(lens), max(lens), Tv, Hqv, Hkvv, Dv, vc["s"],
+                                         vc["c"], vc["base"], 0.0, P(vws.data_ptr()), wsz,
+                                         P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(varlen)
+    out["prefill_varlen"] = {
+        "value": W.varlen_flops(lens, Hqv, Dv) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "ms": ms, "workload": "varlen_7b_mix", "lens": lens, "T": Tv,
+        "path": "RoPE + tcgen05 " + ("two-tile" if Dv == 128 and vc["s"] % 256 == 0
+                                     else "per-row intervals"),
+        "launches_per_call": 2}
+    del Qv, Kv, Vv, vws, Ov, Lv
 
     # decode over a paged cache: the decode workload's caches scattered into
     # 256-row blocks in a seeded random physical order

@@ -121,6 +121,42 @@ dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void*
                               int B, int L, int Hq, int Hkv, int D, int s, int c, float base,
                               float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/* Workspace bytes for dca_attn_prefill_varlen over T packed rows: the fp16
+ * query rotations [3][T][Hq][D] and rotated keys [T][Hkv][D], each rounded up
+ * to 256 bytes (dca_attn_prefill_workspace(1, T, Hq, Hkv, D)).
+ * Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_varlen_workspace(int T, int Hq, int Hkv, int D);
+
+/* Variable-length batched prefill: B independent sequences of different
+ * lengths packed one after another, each a whole DCA prefill of its own
+ * (chunks counted from its first token, causal over its own keys only).  The
+ * batch a serving stack prefills at once when prompts differ in length
+ * (Guide, "Strategic Recommendations", item 1: DCA as a drop-in inference
+ * wrapper); no padding rows are stored or computed.
+ *   Q [T][Hq][D], K, V [T][Hkv][D]: UNROTATED queries and keys and the
+ *     values, bf16, dense; sequence b owns rows cu_seqlens[b] ..
+ *     cu_seqlens[b+1]-1 and its local row r is query index r.
+ *   cu_seqlens: DEVICE int32 [B+1], non-decreasing, cu_seqlens[0] >= 0,
+ *     cu_seqlens[B] <= T; max_seqlen (host) >= every sequence's length.
+ *   O [T][Hq][D] bf16, LSE [Hq][T] fp32 (natural log, scale included); rows
+ *     that belong to no sequence are left untouched.
+ *   V must be finite everywhere: the last key tile of a sequence reaches into
+ *     the next one's rows, which the causal mask weights by exactly 0.
+ * Kernels: the fused RoPE kernel over the packed rows, then the tcgen05
+ * attention kernels (two-tile kernel when D == 128 and s % 256 == 0, the
+ * per-row-interval kernel otherwise); work is issued longest query tiles
+ * first over all sequences.  Offsets that break the rules above are not read
+ * on the host: the kernels skip such a sequence and set the device error word
+ * (DCA_ERR_INVALID_ARG at the next dca_sync_status).
+ * The call owns no memory; `workspace` (dca_attn_prefill_varlen_workspace
+ * bytes) is the caller's.  D in {64, 128}.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
+                                     float* LSE, const int* cu_seqlens, int B, int max_seqlen,
+                                     int T, int Hq, int Hkv, int D, int s, int c, float base,
+                                     float scale, void* workspace, size_t ws_bytes,
+                                     void* stream);
+
 /* Workspace bytes for dca_attn_prefill_3pass: the prefill workspace plus, for
  * each of the three pieces, an fp32 output [B][L][Hq][D] and an fp32 LSE
  * [B][Hq][L].  Returns 0 for unsupported arguments. */

@@ -25,6 +25,7 @@ __all__ = [
     "dca_prefill_attention", "dca_attn_prefill", "dca_prefill_path",
     "dca_attn_prefill_3pass_workspace", "dca_attn_prefill_3pass",
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
+    "dca_attn_prefill_varlen_workspace", "dca_attn_prefill_varlen",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
     "dca_attn_decode_paged", "dca_kv_append_paged",
@@ -51,6 +52,9 @@ _SIGS = {
                               _P]),
     "dca_prefill_path": (_I, [_I, _I, _I, _I]),
     "dca_attn_prefill_3pass_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_attn_prefill_varlen_workspace": (_Z, [_I, _I, _I, _I]),
+    "dca_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                     _F, _P, _Z, _P]),
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "dca_selfextend_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "dca_attn_prefill_host_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -209,6 +213,36 @@ def dca_attn_prefill(Q, K, V, s, c, base=10000.0, scale=0.0, workspace=None, O=N
     _need(LSE, "LSE", torch.float32, 3)
     _check(lib().dca_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, L, Hq, Hkv,
                                   D, s, c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_varlen_workspace(T: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(lib().dca_attn_prefill_varlen_workspace(T, Hq, Hkv, D))
+
+
+def dca_attn_prefill_varlen(Q, K, V, cu_seqlens, max_seqlen, s, c, base=10000.0, scale=0.0,
+                            workspace=None, O=None, LSE=None):
+    """Packed variable-length prefill.  Q [T, Hq, D], K, V [T, Hkv, D] bf16;
+    cu_seqlens int32 [B+1] on the device (sequence b owns rows cu_seqlens[b]
+    .. cu_seqlens[b+1]-1); max_seqlen (int) bounds every sequence's length.
+    Returns (O [T, Hq, D] bf16, LSE [Hq, T] fp32); rows of no sequence are left
+    as allocated."""
+    _need(Q, "Q", torch.bfloat16, 3)
+    _need(K, "K", torch.bfloat16, 3)
+    _need(V, "V", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    nbytes = dca_attn_prefill_varlen_workspace(T, Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    O = torch.empty_like(Q) if O is None else O
+    LSE = torch.empty((Hq, T), dtype=torch.float32, device=Q.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 3)
+    _need(LSE, "LSE", torch.float32, 2)
+    _check(lib().dca_attn_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                         _ptr(cu_seqlens), B, int(max_seqlen), T, Hq, Hkv, D, s,
+                                         c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
     return O, LSE
 
 

@@ -61,7 +61,8 @@ template <int D>
 struct Lay2 {
   static constexpr int kSmMisc = Lay<D>::kSmBar + kNumBars * 8;  // TMEM base, abort flag
   static constexpr int kSmPlan = kSmMisc + 16;                    // the CTA's visit plan
-  static constexpr int kSmTotal = kSmPlan + 128 + 1024;
+  static constexpr int kSmSeq = kSmPlan + 128;                    // its sequence's rows
+  static constexpr int kSmTotal = kSmSeq + 32 + 1024;
   static_assert(kSmTotal <= 232448, "shared memory budget");
 };
 constexpr uint32_t kTmemCols = 512;
@@ -193,11 +194,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
-    int q_off, int group_units) {
+    int q_off, int group_units, const int* __restrict__ cu_seqlens, int T) {
   using LD = Lay<D>;
   constexpr int kHalves = LD::kHalves, kTileBytes = LD::kTileBytes;
   constexpr int kSmQ = LD::kSmQ, kSmK = LD::kSmK, kSmV = LD::kSmV, kSmBar = LD::kSmBar;
-  constexpr int kSmMisc = Lay2<D>::kSmMisc, kSmPlan = Lay2<D>::kSmPlan;
+  constexpr int kSmMisc = Lay2<D>::kSmMisc, kSmPlan = Lay2<D>::kSmPlan, kSmSeq = Lay2<D>::kSmSeq;
+  static_assert(sizeof(Plan) <= 128 && sizeof(SeqSpan) <= 32, "plan / span slots");
   constexpr uint32_t kOCols = (uint32_t)D;  // O accumulator columns per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -217,16 +219,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const int h = po.h, b = po.b;
   const int hk = h / (Hq / Hkv);
   const int q0_loc = m * 2 * kTile;          // row of this call
-  const int last_row = q_off + L - 1;        // absolute
+  SeqSpan sq0;
+  if (!seq_span(cu_seqlens, b, B, L, T, sq0)) {  // reported, no work
+    if (tid == 0) report_error(kDevBadArg, 312);
+    return;
+  }
+  if (q0_loc >= sq0.n) return;  // the pair lies past a shorter sequence's end
+  const int last_row = q_off + sq0.n - 1;    // absolute
   int rows_lo[2], rows_hi[2];
   for (int x = 0; x < 2; ++x) {
     rows_lo[x] = q_off + q0_loc + x * kTile;
     rows_hi[x] = min(rows_lo[x] + kTile - 1, last_row);
   }
   const Plan& pl = *reinterpret_cast<const Plan*>(smem + kSmPlan);
+  // read from shared memory where used (fewer live registers)
+  const SeqSpan& sq = *reinterpret_cast<const SeqSpan*>(smem + kSmSeq);
 
   if (tid == 0) {
     *reinterpret_cast<Plan*>(smem + kSmPlan) = make_plan(rule, rows_lo, rows_hi);
+    *reinterpret_cast<SeqSpan*>(smem + kSmSeq) = sq0;
     for (int i = 0; i < kNumQSlots; ++i) {
       mbar_init(bar(kQFull + i), 1);
       mbar_init(bar(kQEmpty + i), 1);
@@ -275,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
         const int row = q0_loc + x * kTile;
 #pragma unroll
         for (int hf = 0; hf < kHalves; ++hf)
-          tma_load_4d(dst + hf * kBox, &tmQ, fb, hf * 64, h, row, piece * B + b);
+          tma_load_4d(dst + hf * kBox, &tmQ, fb, hf * 64, h, sq.row0 + row,
+                      piece * sq.nb + sq.bt);
         q_last[slot] = n;
         return true;
       };
@@ -291,10 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
             break;
           mbar_arrive_expect_tx(bar(kKFull + sg), kTileBytes);
           const uint32_t kd = sbase + kSmK + sg * kTileBytes;
-          const int kb = rule.kplane(pl.pc[k]) * B + b;  // key plane of the piece
+          const int kb = rule.kplane(pl.pc[k]) * sq.nb + sq.bt;  // key plane of the piece
 #pragma unroll
           for (int hf = 0; hf < kHalves; ++hf)
-            tma_load_4d(kd + hf * kBox, &tmK, bar(kKFull + sg), hf * 64, hk, t * kTile, kb);
+            tma_load_4d(kd + hf * kBox, &tmK, bar(kKFull + sg), hf * 64, hk,
+                        sq.row0 + t * kTile, kb);
           k_last[sg] = st;
           if (first && !(ok = load_q(2 * k + 1, pl.pc[k]))) break;
           if (st >= 2 &&
@@ -304,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
           const uint32_t vd = sbase + kSmV + sg * kTileBytes;
 #pragma unroll
           for (int hf = 0; hf < kHalves; ++hf)
-            tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk, t * kTile, b);
+            tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk,
+                        sq.row0 + t * kTile, sq.bt);
           v_last[sg] = st;
         }
       }
@@ -476,9 +490,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kODone + x), (j - 1) & 1, abort_flag, 499));
     if (ok && j > 0) {
       tc_fence_after();
-      const bool valid = i_row < L;
+      const bool valid = i_row < sq.n;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = O + (((size_t)b * L + (valid ? i_row : 0)) * Hq + h) * D;
+      const size_t o_row = (size_t)sq.bt * sq.rows + sq.row0 + (valid ? i_row : 0);
+      __nv_bfloat16* orow = O + (o_row * Hq + h) * D;
 #pragma unroll 1
       for (int q = 0; q < (int)kOCols / 32; ++q) {
         uint32_t o[32];
@@ -497,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
         }
       }
       if (valid)
-        LSE[((size_t)b * Hq + h) * L + i_row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+        LSE[((size_t)sq.bt * Hq + h) * sq.rows + sq.row0 + i_row] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
     }
   }
 
@@ -514,30 +530,36 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
 namespace gen_path {
 
 // Tensor maps and launch: Qrot [nq planes][B][L][Hq][D] and Krot [kKPlanes]
-// [B][k_rows][Hkv][D] fp16, V [B][v_rows][Hkv][D] bf16.
+// [B][k_rows][Hkv][D] fp16, V [B][v_rows][Hkv][D] bf16.  With cu_seqlens
+// (device [B+1], q_off == 0) each tensor is one packed batch of T rows
+// holding B sequences of at most L rows.
 template <int D, class Rule>
 cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
                          int B, int L, int Hq, int Hkv, Rule rule, int nq, float scale,
-                         cudaStream_t stream, int q_off, int k_rows, int v_rows) {
+                         cudaStream_t stream, int q_off, int k_rows, int v_rows,
+                         const int* cu_seqlens, int T) {
   if (q_off < 0) return cudaErrorInvalidValue;
+  if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
-  const int Lkv = q_off + L;
+  const int Bm = cu_seqlens ? 1 : B;       // tensor batch extent
+  const int Lrows = cu_seqlens ? T : L;    // tensor query rows per batch entry
+  const int Lkv = cu_seqlens ? T : q_off + L;
   if (k_rows == 0) k_rows = Lkv;
   if (v_rows == 0) v_rows = Lkv;
   CUtensorMap tmQ, tmK, tmV;
   const uint32_t box[4] = {64, 1, (uint32_t)kTile, 1};
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)L, (uint64_t)nq * B};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Lrows, (uint64_t)nq * Bm};
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hq * D * 2,
-                                 (uint64_t)L * Hq * D * 2};
+                                 (uint64_t)Lrows * Hq * D * 2};
     if (!encode_tensor_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Qrot, 4, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   {
     const uint64_t kdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv,
-                               (uint64_t)Rule::kKPlanes * B};
-    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)B};
+                               (uint64_t)Rule::kKPlanes * Bm};
+    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)Bm};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
     const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
@@ -557,36 +579,39 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
   dim3 grid((unsigned)(((num_qt + 1) / 2) * Hq * B));
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, rule, scale * 1.4426950408889634f,
-                                             q_off, B * Hkv);  // one group: longest first
+                                             q_off, B * Hkv,  // one group: longest first
+                                             cu_seqlens, T);
   return cudaGetLastError();
 }
 
 template <class Rule>
 cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
                        int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
-                       cudaStream_t stream, int q_off, int k_rows, int v_rows) {
+                       cudaStream_t stream, int q_off, int k_rows, int v_rows,
+                       const int* cu_seqlens = nullptr, int T = 0) {
   if (D == 64)
     return launch_gen_d<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream, q_off,
-                            k_rows, v_rows);
+                            k_rows, v_rows, cu_seqlens, T);
   if (D == 128)
     return launch_gen_d<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream,
-                             q_off, k_rows, v_rows);
+                             q_off, k_rows, v_rows, cu_seqlens, T);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace gen_path
 
-// tcgen05 prefill attention for any chunk size (D = 128).  Query rows q_off ..
-// q_off+L-1 against keys 0 .. q_off+L-1 held with k_rows / v_rows rows per
-// sequence (0: q_off + L).
+// tcgen05 prefill attention for any chunk size (D = 64 or 128).  Query rows
+// q_off .. q_off+L-1 against keys 0 .. q_off+L-1 held with k_rows / v_rows
+// rows per sequence (0: q_off + L); or, with cu_seqlens, a packed batch.
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
-                                          int q_off, int k_rows, int v_rows) {
+                                          int q_off, int k_rows, int v_rows,
+                                          const int* cu_seqlens, int T) {
   if (s < 1) return cudaErrorInvalidValue;
   return gen_path::launch_gen(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, D,
                               gen_path::DcaIntervals{s}, 3, scale, stream, q_off, k_rows,
-                              v_rows);
+                              v_rows, cu_seqlens, T);
 }
 
 // SelfExtend on the same kernel: Qse, Kse [2][B][L][H][D] fp16 (neighbour,

@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2,
-    int pair_off, int group_units) {
+    int pair_off, int group_units, const int* __restrict__ cu_seqlens, int T) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -86,6 +86,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   const int hk = h / (Hq / Hkv);
   const int q0 = m * 2 * kTile;              // absolute
   const int q0_loc = q0 - pair_off * 2 * kTile;
+  SeqSpan sq;
+  if (!seq_span(cu_seqlens, b, B, L, T, sq)) {  // reported, no work
+    if (tid == 0) report_error(kDevBadArg, 311);
+    return;
+  }
+  if (q0_loc >= sq.n) return;  // the pair lies past a shorter sequence's end
   const int tpc = s / kTile;
   // DCA pieces met by this query-tile pair, in walk order: phase p uses Qrot
   // plane n_ph - 1 - p (inter = 2, successive = 1, intra = 0) and starts at key
@@ -146,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         const uint32_t dst = sbase + kSmQ + slot * kTileBytes;
         const int row = q0_loc + x * kTile;
         const int plane = n_ph - 1 - p;
-        tma_load_4d(dst, &tmQ, fb, 0, h, row, plane * B + b);
-        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, row, plane * B + b);
+        tma_load_4d(dst, &tmQ, fb, 0, h, sq.row0 + row, plane * sq.nb + sq.bt);
+        tma_load_4d(dst + kBox, &tmQ, fb, 64, h, sq.row0 + row, plane * sq.nb + sq.bt);
         q_last[slot] = n;
         return true;
       };
@@ -162,16 +168,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
           break;
         mbar_arrive_expect_tx(bar(kKFull + st), kTileBytes);
         const uint32_t kd = sbase + kSmK + st * kTileBytes;
-        tma_load_4d(kd, &tmK, bar(kKFull + st), 0, hk, i * kTile, b);
-        tma_load_4d(kd + kBox, &tmK, bar(kKFull + st), 64, hk, i * kTile, b);
+        tma_load_4d(kd, &tmK, bar(kKFull + st), 0, hk, sq.row0 + i * kTile, sq.bt);
+        tma_load_4d(kd + kBox, &tmK, bar(kKFull + st), 64, hk, sq.row0 + i * kTile, sq.bt);
         k_last[st] = i;
         if (boundary && !(ok = load_q(2 * p + 1))) break;
         if (i >= 2 && !(ok = mbar_wait(bar(kVEmpty + st), ((i >> 1) + 1) & 1, abort_flag, 403)))
           break;
         mbar_arrive_expect_tx(bar(kVFull + st), kTileBytes);
         const uint32_t vd = sbase + kSmV + st * kTileBytes;
-        tma_load_4d(vd, &tmV, bar(kVFull + st), 0, hk, i * kTile, b);
-        tma_load_4d(vd + kBox, &tmV, bar(kVFull + st), 64, hk, i * kTile, b);
+        tma_load_4d(vd, &tmV, bar(kVFull + st), 0, hk, sq.row0 + i * kTile, sq.bt);
+        tma_load_4d(vd + kBox, &tmV, bar(kVFull + st), 64, hk, sq.row0 + i * kTile, sq.bt);
         v_last[st] = i;
       }
       // drain: every issued copy has landed before shared memory is released
@@ -313,8 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      const bool valid = i_row < L;
-      __nv_bfloat16* orow = O + (((size_t)b * L + (valid ? i_row : 0)) * Hq + h) * kHD;
+      const bool valid = i_row < sq.n;
+      const size_t o_row = (size_t)sq.bt * sq.rows + sq.row0 + (valid ? i_row : 0);
+      __nv_bfloat16* orow = O + (o_row * Hq + h) * kHD;
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
@@ -333,7 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         }
       }
       if (valid)
-        LSE[((size_t)b * Hq + h) * L + i_row] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+        LSE[((size_t)sq.bt * Hq + h) * sq.rows + sq.row0 + i_row] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
     }
   }
 
@@ -349,29 +357,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
 
 // Ping-pong tcgen05 prefill attention (D = 128, s % 256 == 0).  Query rows
 // are q_off .. q_off+L-1 (q_off % 256 == 0) of sequences whose keys 0 ..
-// q_off+L-1 sit in Krot / V with kv_rows rows per sequence.
+// q_off+L-1 sit in Krot / V with kv_rows rows per sequence.  With cu_seqlens
+// (device [B+1], q_off == 0) the tensors are one packed batch of T rows
+// holding B sequences of at most L rows each.
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
-                                         int q_off, int k_rows, int v_rows) {
+                                         int q_off, int k_rows, int v_rows,
+                                         const int* cu_seqlens, int T) {
   using namespace pp_path;
   if (D != kHD || s % (2 * kTile) != 0 || q_off % (2 * kTile) != 0) return cudaErrorInvalidValue;
+  if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
-  const int Lkv = q_off + L;
+  const int Bm = cu_seqlens ? 1 : B;       // tensor batch extent
+  const int Lrows = cu_seqlens ? T : L;    // tensor query rows per batch entry
+  const int Lkv = cu_seqlens ? T : q_off + L;
   if (k_rows == 0) k_rows = Lkv;
   if (v_rows == 0) v_rows = Lkv;
   CUtensorMap tmQ, tmK, tmV;
   const uint32_t box[4] = {64, 1, (uint32_t)kTile, 1};
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)L, (uint64_t)3 * B};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Lrows, (uint64_t)3 * Bm};
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hq * D * 2,
-                                 (uint64_t)L * Hq * D * 2};
+                                 (uint64_t)Lrows * Hq * D * 2};
     if (!encode_tensor_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Qrot, 4, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)B};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)Bm};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
     const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
@@ -391,7 +405,8 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
   kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
                                              B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
                                              q_off / (2 * kTile),
-                                             pair_group_units(B, Hkv, Lkv, D));
+                                             pair_group_units(B, Hkv, cu_seqlens ? L : Lkv, D),
+                                             cu_seqlens, T);
   return cudaGetLastError();
 }
 

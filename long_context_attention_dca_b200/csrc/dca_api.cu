@@ -226,6 +226,50 @@ dca_status_t dca_attn_prefill(const void* Q, const void* K, const void* V, void*
                                workspace, ws_bytes, stream);
 }
 
+size_t dca_attn_prefill_varlen_workspace(int T, int Hq, int Hkv, int D) {
+  return dca_attn_prefill_workspace(1, T, Hq, Hkv, D);
+}
+
+dca_status_t dca_attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
+                                     float* LSE, const int* cu_seqlens, int B, int max_seqlen,
+                                     int T, int Hq, int Hkv, int D, int s, int c, float base,
+                                     float scale, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+  const char* fn = "dca_attn_prefill_varlen";
+  dca_status_t st = check_heads(fn, B, max_seqlen, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (T < 0) return fail(DCA_ERR_INVALID_ARG, "%s: T=%d", fn, T);
+  if (auto_path(D, s) != DCA_PATH_TCGEN05)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: library built without the tcgen05 path", fn);
+  if ((long long)B * max_seqlen == 0 || T == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(DCA_ERR_INVALID_ARG, "%s: cu_seqlens is null or not 4-byte aligned", fn);
+  DCA_CHECK_PTR(workspace);
+  PrefillWs ws = prefill_ws_layout(workspace, 1, T, Hq, Hkv, D);
+  if (ws_bytes < ws.bytes)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes,
+                ws.bytes);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_prefill_rope(Q, K, ws.qrot, ws.krot, 1, T, Hq, Hkv, D, s, c, base, strm,
+                                      cu_seqlens, B);
+  if (e == cudaSuccess) {
+    if (D == 128 && s % 256 == 0)
+      e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, max_seqlen, Hq, Hkv, D, s,
+                                       sc, strm, 0, 0, 0, cu_seqlens, T);
+    else
+      e = launch_prefill_attn_sm100_gen(ws.qrot, ws.krot, V, O, LSE, B, max_seqlen, Hq, Hkv, D, s,
+                                        sc, strm, 0, 0, 0, cu_seqlens, T);
+  }
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 size_t dca_attn_prefill_3pass_workspace(int B, int L, int Hq, int Hkv, int D) {
   const size_t base = dca_attn_prefill_workspace(B, L, Hq, Hkv, D);
   if (base == 0 && !(B == 0 || L == 0)) return 0;

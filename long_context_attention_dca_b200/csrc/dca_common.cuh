@@ -103,6 +103,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Where sequence b's rows sit in the prefill tensors.  A padded batch holds
+// sequence b at tensor batch coordinate b, rows 0 .. L-1.  A packed batch
+// (cu_seqlens != null) is one tensor of T rows; sequence b owns rows
+// cu_seqlens[b] .. cu_seqlens[b+1]-1, at most L (the longest sequence), and
+// its local row r is query index r of its own prefill.
+struct SeqSpan {
+  int row0;  // tensor row of local row 0
+  int n;     // rows of the sequence
+  int bt;    // tensor batch coordinate
+  int nb;    // tensor batch extent
+  int rows;  // tensor rows per batch entry (the O / LSE row stride)
+};
+// False when the packed offsets of sequence b are not a valid span of at
+// most L rows inside [0, T).
+__device__ __forceinline__ bool seq_span(const int* cu_seqlens, int b, int B, int L, int T,
+                                         SeqSpan& sq) {
+  if (cu_seqlens == nullptr) {
+    sq = SeqSpan{0, L, b, B, L};
+    return true;
+  }
+  const int a = __ldg(cu_seqlens + b), e = __ldg(cu_seqlens + b + 1);
+  sq = SeqSpan{a, e - a, 0, 1, T};
+  return a >= 0 && e >= a && e - a <= L && e <= T;
+}
+
 // Dispatch order of the two-tile prefill kernels' (query-tile pair, head,
 // sequence) work items, from a 1-D block index: the (sequence, kv head) units
 // are taken in groups of `k`, one group after another; within a group the
@@ -143,7 +168,7 @@ inline int pair_group_units(int B, int Hkv, int Lkv, int D) {
   return (int)k;
 }
 
-// Per-warpgroup register reallocation// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
+// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
 // the same one).  The counts used by a kernel must sum, over its warpgroups,
 // to no more than the registers the block was launched with.
 template <int N>

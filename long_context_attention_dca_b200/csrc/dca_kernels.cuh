@@ -18,7 +18,8 @@ cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, in
 // Writes Krot [B][L][Hkv][D] and Qrot [3][B][L][Hq][D] (intra, succ, inter), fp16.
 cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const int* cu_seqlens = nullptr,
+                                int n_seq = 0);
 
 // Chunk of Lq rows at absolute positions t0 .. t0+Lq-1: Qrot [3][B][Lq][Hq][D]
 // fp16; rotated keys go in bf16 to cache rows t0 + r (pitch Tcap; skipped when
@@ -62,13 +63,15 @@ cudaError_t launch_merge3(const float* Op, const float* LSEp, void* O, float* LS
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
-                                         int q_off = 0, int k_rows = 0, int v_rows = 0);
+                                         int q_off = 0, int k_rows = 0, int v_rows = 0,
+                                         const int* cu_seqlens = nullptr, int T = 0);
 // tcgen05 prefill attention for any chunk size (D = 128): per-row key
 // intervals per piece, straddling tiles visited once per piece they hold.
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
-                                          int q_off = 0, int k_rows = 0, int v_rows = 0);
+                                          int q_off = 0, int k_rows = 0, int v_rows = 0,
+                                          const int* cu_seqlens = nullptr, int T = 0);
 // SelfExtend on the per-row-interval tcgen05 kernel (D = 128).
 cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
                                                  const void* V, void* O, float* LSE, int B,

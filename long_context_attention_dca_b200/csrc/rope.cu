@@ -127,23 +127,47 @@ constexpr int kRopeThreads = 256;
 // against a cache (kChunk true) writes them in bf16 to cache rows q_off + r of
 // pitch Tcap (Kout, unless null) and in fp16 to rows q_off + r of Kh (kh_rows
 // rows per sequence), and copies the chunk's values into the value cache
-// (unless Vc is null).
+// (unless Vc is null).  A packed batch (cu_seqlens != null, B = 1, L = T rows,
+// kChunk false) holds n_seq sequences, sequence b at rows cu_seqlens[b] ..
+// cu_seqlens[b+1]-1; a row's index is counted from its sequence's first row.
 template <int D, bool kChunk>
 __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
     __half* __restrict__ Qrot, void* __restrict__ Kout, int B, int L, int Hq, int Hkv, int s,
     int c, double log2_base, int q_off, int Tcap, const __nv_bfloat16* __restrict__ Vsrc,
-    __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh, int kh_rows) {
+    __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh, int kh_rows,
+    const int* __restrict__ cu_seqlens, int n_seq) {
   constexpr int kHalf = D / 2;
   constexpr int kGroups = D / 16;
   __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
+  __shared__ int im_s[kRopeRows];               // row index mod s
   const long long total_rows = (long long)B * L;
   const long long row0 = (long long)blockIdx.x * kRopeRows;
   const int nrows = (int)min((long long)kRopeRows, total_rows - row0);
   constexpr double kTwoPi = 6.283185307179586476925286766559;
+  if (threadIdx.x < nrows) {
+    const long long row = row0 + threadIdx.x;
+    int im;
+    if (cu_seqlens == nullptr) {
+      im = (int)(((row % L) + q_off) % s);
+    } else {
+      // last sequence starting at or before the row (rows of no sequence
+      // are rotated as if they continued the last one; nothing reads them)
+      const int r = (int)row;
+      int lo = 0, hi = n_seq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(cu_seqlens + mid) <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      im = max(r - __ldg(cu_seqlens + lo), 0) % s;
+    }
+    im_s[threadIdx.x] = im;
+  }
+  __syncthreads();
   for (int idx = threadIdx.x; idx < nrows * 3 * kHalf; idx += kRopeThreads) {
     const int r = idx / (3 * kHalf), kind = (idx / kHalf) % 3, k = idx % kHalf;
-    const int im = (int)((((row0 + r) % L) + q_off) % s);
+    const int im = im_s[r];
     const int pos = kind == 0 ? im : (kind == 1 ? query_pos_for_piece(kSucc, im, s, c) : c - 1);
     const double theta = exp2(-(2.0 * (double)k / (double)D) * log2_base);
     const double a = (double)pos * theta;
@@ -233,8 +257,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     rotate8<true>(lo, hi, cs, olo, ohi);  // inter plane (c - 1)
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = olo;
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + kHalf) = ohi;
-    const int im = (int)(((row % L) + q_off) % s);
-    if (query_pos_for_piece(kSucc, im, s, c) != c - 1) {
+    if (query_pos_for_piece(kSucc, im_s[r], s, c) != c - 1) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float2 v = cs_s[r][1][g * 8 + e];
@@ -370,7 +393,7 @@ cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, in
 
 cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const int* cu_seqlens, int n_seq) {
   using namespace rope_path;
   const long long rows = (long long)B * L;
   if (rows == 0) return cudaSuccess;
@@ -379,7 +402,7 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
     kern<<<blocks, kRopeThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Krot, B, L, Hq, Hkv, s, c, log2((double)base), 0, L,
-        nullptr, nullptr, nullptr, 0);
+        nullptr, nullptr, nullptr, 0, cu_seqlens, n_seq);
   };
   if (D == 64) args(prefill_rope_kernel<64, false>);
   else args(prefill_rope_kernel<128, false>);
@@ -399,7 +422,7 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Kcache, B, Lq, Hq, Hkv, s, c, log2((double)base), t0, Tcap,
         static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(Vcache),
-        static_cast<__half*>(Kf16), kh_rows);
+        static_cast<__half*>(Kf16), kh_rows, nullptr, 0);
   };
   if (D == 64) args(prefill_rope_kernel<64, true>);
   else args(prefill_rope_kernel<128, true>);

@@ -10,6 +10,9 @@ Recipe (every config, seed 0 unless stated):
   * "K x2 on 1% of positions": n = floor(frac * L) token positions from a
     ``randperm(L)`` drawn after V; K is doubled at those positions for every
     batch entry and kv head (exact in bf16);
+  * packed variable-length batch: lengths [B] uniform integers in
+    [len_lo, len_hi] drawn first (or given), cu_seqlens their running sums
+    from 0, then Q [T, Hq, D], K [T, Hkv, D], V [T, Hkv, D] as for prefill;
   * decode: t [B] uniform integers in [t_lo, t_hi) drawn first, then q
     [B, Hq, D], then the K cache entry by entry (K[b] = [Tcap, Hkv, D] for
     b = 0 .. B-1), then the V cache the same way.  The K cache stands for keys
@@ -38,6 +41,9 @@ CONFIGS = {
                          c=4096, s=3072, base=10000.0, k_boost_frac=0.0),
     "decode_b16": dict(kind="decode", B=16, Hq=64, Hkv=8, D=128, Tcap=65536,
                        c=4096, s=3072, base=10000.0, t_lo=32768, t_hi=65536),
+    # packed batch of prompts of mixed length (serving-style prefill)
+    "varlen_7b_mix": dict(kind="varlen", B=8, Hq=32, Hkv=32, D=128, c=4096, s=3072,
+                          base=10000.0, len_lo=512, len_hi=16384),
 }
 
 
@@ -60,6 +66,25 @@ def make_prefill_inputs(cfg: dict, device="cpu", seed: int = 0):
         pos = torch.randperm(L, generator=gen, device=device)[:n]
         K[:, pos] = K[:, pos] * 2
     return Q, K, V
+
+
+def make_varlen_inputs(cfg: dict, device="cpu", seed: int = 0, lens=None):
+    """Return (Q [T,Hq,D], K, V [T,Hkv,D] bf16 on ``device``, cu_seqlens int32
+    [B+1] on the CPU, lens list) for a packed batch of mixed-length prompts."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    if lens is None:
+        lens = torch.randint(cfg["len_lo"], cfg["len_hi"] + 1, (cfg["B"],), generator=gen,
+                             device=device, dtype=torch.int64).tolist()
+    lens = [int(n) for n in lens]
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+    T = int(cu[-1])
+    Hq, Hkv, D = cfg["Hq"], cfg["Hkv"], cfg["D"]
+    Q = _normal_bf16((T, Hq, D), gen, device)
+    K = _normal_bf16((T, Hkv, D), gen, device)
+    V = _normal_bf16((T, Hkv, D), gen, device)
+    return Q, K, V, cu, lens
 
 
 def boosted_positions(cfg: dict, seed: int = 0):
@@ -103,6 +128,11 @@ def prefill_flops(cfg: dict) -> float:
     """Algorithmic FLOPs of causal attention: 4 * D * Hq * B * L(L+1)/2."""
     L = cfg["L"]
     return 4.0 * cfg["D"] * cfg["Hq"] * cfg["B"] * L * (L + 1) / 2
+
+
+def varlen_flops(lens, Hq: int, D: int) -> float:
+    """Algorithmic FLOPs of a packed batch: causal attention per sequence."""
+    return sum(4.0 * D * Hq * n * (n + 1) / 2 for n in lens)
 
 
 def decode_bytes(cfg: dict, t) -> float:

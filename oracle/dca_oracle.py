@@ -29,6 +29,8 @@ fusion or reordering:
   l = sum exp(z - m),  O_i = sum exp(z_j - m) v_j / l,  LSE_i = m + ln l.
 * Chunked prefill (dca_prefill_chunk): rows t0 .. t0+Lq-1 of the same
   definition with keys 0 .. t0-1 read, already rotated, from a cache.
+* Variable-length batch (dca_prefill_varlen_rows): sequences packed one after
+  another, each its own prefill (chunks from its first token, own keys only).
 * SelfExtend (prior art; LLM Maybe LongLM: Self-Extend LLM Context Window
   Without Tuning, abstract): neighbour pairs (i - j < W) at positions (i, j),
   grouped pairs at (floor(i/G) + W - floor(W/G), floor(j/G)), one softmax.
@@ -39,7 +41,8 @@ Every function is fp64 end to end; nothing is rounded to bf16.
 Pins that hold this module to something other than itself live in
 ``tests/test_oracle_pins.py`` (worked index table, closed-form piece counts,
 reduction to plain RoPE attention, Q = 0 and constant-V closed forms, RoPE
-relativity, decode = prefill row, chunk = whole-sequence rows, hand-worked
+relativity, decode = prefill row, chunk = whole-sequence rows, packed batch =
+padded batch and its Q = 0 closed form, hand-worked
 SelfExtend distance tables and its reductions to plain RoPE attention) and
 ``tests/test_oracle_mutations.py``
 (plausible mistakes planted here must each fail a pin).
@@ -306,6 +309,34 @@ def dca_prefill_chunk(Qc, Kc, Vc, k_cache_rot, v_cache, t0: int, s: int, c: int,
                     i = t0 + r
                     q = np.asarray(Qc[b, r, h, :], np.float64)
                     out[(b, h, r)] = dca_row(q, k_rot[:i + 1], v[:i + 1], i, s, c, base, sc)
+    return out
+
+
+def dca_prefill_varlen_rows(Q, K, V, cu_seqlens, s: int, c: int, base: float = 10000.0,
+                            scale: float = 0.0, rows=None, heads=None):
+    """Packed variable-length batch of independent DCA prefills.
+
+    Q: [T, Hq, D]; K, V: [T, Hkv, D] (unrotated).  Sequence b owns packed rows
+    cu_seqlens[b] .. cu_seqlens[b+1]-1; its row at packed index t is query
+    index t - cu_seqlens[b] of a prefill over that sequence alone: chunks are
+    counted from the sequence's first token and only its own keys are
+    attended.  rows: packed indices to evaluate (default: every row of every
+    sequence).  Returns {(h, t): (O [D], LSE)} keyed by packed row.
+    """
+    cu = [int(x) for x in cu_seqlens]
+    want = None if rows is None else {int(r) for r in rows}
+    out = {}
+    for b in range(len(cu) - 1):
+        a, e = cu[b], cu[b + 1]
+        if e <= a:
+            continue
+        local = [t - a for t in range(a, e) if want is None or t in want]
+        if not local:
+            continue
+        res = dca_prefill_rows(Q[None, a:e], K[None, a:e], V[None, a:e], s, c, base, scale,
+                               rows=local, heads=heads)
+        for (_, h, r), val in res.items():
+            out[(h, a + r)] = val
     return out
 
 

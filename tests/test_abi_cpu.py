@@ -70,6 +70,10 @@ def test_workspace_queries(lib):
     # SelfExtend: neighbour + grouped rotations of Q and K, fp16
     assert dca.dca_selfextend_workspace(1, 100, 4, 2, 64) == (up(2 * 100 * 4 * 64 * 2) +
                                                               up(2 * 100 * 2 * 64 * 2))
+    # packed variable-length batch: the prefill workspace of one T-row sequence
+    assert dca.dca_attn_prefill_varlen_workspace(777, 8, 2, 128) == (
+        up(3 * 777 * 8 * 128 * 2) + up(777 * 2 * 128 * 2))
+    assert dca.dca_attn_prefill_varlen_workspace(777, 8, 3, 128) == 0
 
 
 def test_prefill_path_selection(lib):
@@ -162,6 +166,22 @@ def test_argument_errors_return_codes(lib):
                                                  1 << 30, None)) == 1
     assert _code(lib.dca_attn_prefill_selfextend(*sargs, 1, 64, 4, 2, 128, 2, 8, 1e4, 0.0, ws,
                                                  64, None)) == 5
+    # packed batch: null or misaligned offsets, negative T, short workspace, s > c
+    vargs = (fake,) * 5
+    assert _code(lib.dca_attn_prefill_varlen(*vargs, None, 3, 64, 100, 4, 2, 128, 16, 32, 1e4,
+                                             0.0, ws, 1 << 30, None)) == 1
+    assert "cu_seqlens" in dca.dca_last_error_string()
+    assert _code(lib.dca_attn_prefill_varlen(*vargs, P(0x10002), 3, 64, 100, 4, 2, 128, 16, 32,
+                                             1e4, 0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_varlen(*vargs, fake, 3, 64, -1, 4, 2, 128, 16, 32, 1e4,
+                                             0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_varlen(*vargs, fake, 3, 64, 100, 4, 2, 128, 16, 32, 1e4,
+                                             0.0, ws, 64, None)) == 5
+    assert _code(lib.dca_attn_prefill_varlen(*vargs, fake, 3, 64, 100, 4, 2, 128, 64, 32, 1e4,
+                                             0.0, ws, 1 << 30, None)) == 2
+    # empty batches are no-ops even with null pointers
+    assert _code(lib.dca_attn_prefill_varlen(None, None, None, None, None, None, 0, 64, 100, 4,
+                                             2, 128, 16, 32, 1e4, 0.0, None, 0, None)) == 0
     # wait self-test: deadline out of range
     assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
     assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1

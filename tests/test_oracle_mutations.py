@@ -5,8 +5,10 @@ with a version carrying a typical slip: an off-by-one in the successive rule,
 a dropped modulo, interleaved instead of half-split RoPE pairing, a flipped
 sign, a wrong frequency exponent, a missing softmax scale, a log2 LSE, a
 causal off-by-one, a wrong GQA mapping, a shifted chunk origin, a broken
-partial merge, a decode that reads one key too few, or a chunked prefill
-that ignores or misaligns its cache.  The pins of
+partial merge, a decode that reads one key too few, a chunked prefill
+that ignores or misaligns its cache, or a packed variable-length batch that
+leaks across sequences, counts positions from the packed start or reports
+local rows.  The pins of
 ``test_oracle_pins`` must reject each one.
 """
 
@@ -154,6 +156,49 @@ def _chunk_start_early(Qc, Kc, Vc, k_cache_rot, v_cache, t0, s, c, *args, **kw):
     t = max(t0 - 1, 0)
     return _ORIG_CHUNK(Qc, Kc, Vc, k_cache_rot[:, :t], v_cache[:, :t], t, s, c, *args, **kw)
 
+_ORIG_VARLEN = orc.dca_prefill_varlen_rows
+
+
+def _varlen_whole_pack(Q, K, V, cu_seqlens, s, c, base=10000.0, scale=0.0, rows=None,
+                       heads=None):
+    # the packed tensor treated as one sequence: earlier sequences attended,
+    # chunks counted from the packed start
+    cu = [int(x) for x in cu_seqlens]
+    want = [t for t in range(cu[0], cu[-1]) if rows is None or t in set(rows)]
+    res = orc.dca_prefill_rows(Q[None], K[None], V[None], s, c, base, scale, rows=want,
+                               heads=heads)
+    return {(h, t): val for (_, h, t), val in res.items()}
+
+
+def _varlen_global_positions(Q, K, V, cu_seqlens, s, c, base=10000.0, scale=0.0, rows=None,
+                             heads=None):
+    # own keys only, but query and key positions taken from the packed index
+    cu = [int(x) for x in cu_seqlens]
+    T, Hq, D = Q.shape
+    G = Hq // K.shape[1]
+    sc = 1.0 / np.sqrt(D) if not scale else scale
+    out = {}
+    for b in range(len(cu) - 1):
+        a = cu[b]
+        for t in range(a, cu[b + 1]):
+            if rows is not None and t not in set(rows):
+                continue
+            j = np.arange(a, t + 1)
+            pq = orc.query_position(t, j, s, c)
+            for h in range(Hq) if heads is None else heads:
+                k_rot = orc.rotate(K[a:t + 1, h // G], orc.key_position(j, s), base)
+                z = np.array([k_rot[n] @ orc.rotate(Q[t, h], pq[n], base)
+                              for n in range(len(j))])
+                out[(h, t)] = orc.softmax_row(sc * z, V[a:t + 1, h // G])
+    return out
+
+
+def _varlen_local_keys(*args, **kw):
+    # results keyed from the first sequence's start instead of packed row 0
+    return {(h, t - min(tt for _, tt in _ORIG_VARLEN(*args, **kw))): v
+            for (h, t), v in _ORIG_VARLEN(*args, **kw).items()}
+
+
 MUTANTS = {
     "succ_rule_le": ("query_position", _qpos_succ_le),
     "succ_far_pos_c": ("query_position", _qpos_succ_c),
@@ -175,6 +220,9 @@ MUTANTS = {
     "selfextend_no_shift": ("selfextend_positions", _se_no_shift),
     "selfextend_window_le": ("selfextend_positions", _se_window_le),
     "selfextend_key_not_grouped": ("selfextend_positions", _se_key_not_grouped),
+    "varlen_whole_pack": ("dca_prefill_varlen_rows", _varlen_whole_pack),
+    "varlen_global_positions": ("dca_prefill_varlen_rows", _varlen_global_positions),
+    "varlen_local_keys": ("dca_prefill_varlen_rows", _varlen_local_keys),
 }
 
 

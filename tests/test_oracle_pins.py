@@ -266,6 +266,45 @@ def pin_chunk_equals_prefill_rows():
             np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
 
 
+def pin_varlen_equals_padded_batch():
+    # equal-length sequences packed back to back give the rows of the padded
+    # batch [B, n]; n is not a multiple of s, so counting chunks from the
+    # packed start (or attending an earlier sequence) moves them
+    B, n, s, c = 3, 17, 5, 8
+    Q, K, V = _rand((B, n, 4, 8), 43), _rand((B, n, 2, 8), 44), _rand((B, n, 2, 8), 45)
+    cu = [b * n for b in range(B + 1)]
+    got = orc.dca_prefill_varlen_rows(Q.reshape(B * n, 4, 8), K.reshape(B * n, 2, 8),
+                                      V.reshape(B * n, 2, 8), cu, s, c)
+    assert set(got) == {(h, t) for h in range(4) for t in range(B * n)}
+    full = orc.dca_prefill_rows(Q, K, V, s, c)
+    for (h, t), (o, lse) in got.items():
+        o_ref, lse_ref = full[(t // n, h, t % n)]
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
+def pin_varlen_q_zero_closed_form():
+    # Q = 0: every score is 0, so LSE = ln(r + 1) and O is the mean of the
+    # sequence's own values 0 .. r (local row r); rows before the first
+    # sequence, after the last one and empty sequences produce nothing
+    lens = [7, 1, 12, 0, 9]
+    cu = [2]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    T = cu[-1] + 3
+    K, V = _rand((T, 2, 8), 46), _rand((T, 2, 8), 47)
+    Q = np.zeros((T, 4, 8))
+    got = orc.dca_prefill_varlen_rows(Q, K, V, cu, s=4, c=6)
+    assert set(got) == {(h, t) for h in range(4) for t in range(cu[0], cu[-1])}
+    for b in range(len(lens)):
+        for t in range(cu[b], cu[b + 1]):
+            r = t - cu[b]
+            for h in range(4):
+                o, lse = got[(h, t)]
+                np.testing.assert_allclose(lse, math.log(r + 1), atol=1e-13)
+                np.testing.assert_allclose(o, V[cu[b]:t + 1, h // 2].mean(0), atol=1e-13)
+
+
 def pin_merge_partials():
     z, v = _rand(50, 27) * 3, _rand((50, 8), 28)
     o_full, lse_full = orc.softmax_row(z, v)
@@ -346,7 +385,8 @@ PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_rotation_literals, pin_rope_relativity, pin_plain_rope_matches_sdpa,
         pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
         pin_q_zero_closed_form, pin_constant_v, pin_gqa_mapping,
-        pin_decode_equals_prefill_row, pin_chunk_equals_prefill_rows, pin_merge_partials,
+        pin_decode_equals_prefill_row, pin_chunk_equals_prefill_rows,
+        pin_varlen_equals_padded_batch, pin_varlen_q_zero_closed_form, pin_merge_partials,
         pin_rule_positions, pin_selfextend_worked_tables, pin_selfextend_reduces_to_plain_rope,
         pin_selfextend_distance_bounds]
 
