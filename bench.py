@@ -577,9 +577,7 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
     ms = timed(selfextend)
     out["prefill_selfextend"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                                  "ms": ms, "G": G_se, "W": W_se,
-                                 "path": "RoPE (2 planes) + " + (
-                                     "tcgen05 per-row intervals" if D == 128
-                                     else "general (warp MMA)"),
+                                 "path": "RoPE (2 planes) + tcgen05 per-row intervals",
                                  "launches_per_call": 2}
     del sws, Ose, Lse
 

@@ -16,6 +16,8 @@ cudaError_t launch_rope_rotate(const void* x, void* out, int B, int L, int H, in
                                cudaStream_t stream);
 
 // Writes Krot [B][L][Hkv][D] and Qrot [3][B][L][Hq][D] (intra, succ, inter), fp16.
+// Packed batch: B = 1, L = T rows, cu_seqlens device [n_seq+1]; each row is
+// rotated at its index within its sequence.
 cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* Krot, int B,
                                 int L, int Hq, int Hkv, int D, int s, int c, float base,
                                 cudaStream_t stream, const int* cu_seqlens = nullptr,
@@ -60,19 +62,22 @@ cudaError_t launch_merge3(const float* Op, const float* LSEp, void* O, float* LS
 // tcgen05 ping-pong variant: two query tiles per CTA (D = 128, s % 256 == 0).
 // Chunk form: query rows q_off .. q_off+L-1 (q_off % 256 == 0) against keys
 // 0 .. q_off+L-1 held with k_rows / v_rows rows per sequence (0: q_off + L).
+// Packed form (cu_seqlens device [B+1], q_off 0): Qrot [3][T][Hq][D], Krot and
+// V [T][Hkv][D], O [T][Hq][D], LSE [Hq][T]; B sequences of at most L rows.
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
                                          int q_off = 0, int k_rows = 0, int v_rows = 0,
                                          const int* cu_seqlens = nullptr, int T = 0);
-// tcgen05 prefill attention for any chunk size (D = 128): per-row key
+// tcgen05 prefill attention for any chunk size (D = 64 or 128): per-row key
 // intervals per piece, straddling tiles visited once per piece they hold.
+// Same chunk and packed forms as the ping-pong variant (any q_off).
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off = 0, int k_rows = 0, int v_rows = 0,
                                           const int* cu_seqlens = nullptr, int T = 0);
-// SelfExtend on the per-row-interval tcgen05 kernel (D = 128).
+// SelfExtend on the per-row-interval tcgen05 kernel (D = 64 or 128).
 cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
                                                  const void* V, void* O, float* LSE, int B,
                                                  int L, int Hq, int Hkv, int D, int W,
