@@ -274,8 +274,10 @@ dca_status_t dca_attn_prefill_host(const void* Q, const void* K, const void* V, 
 int dca_prefill_path(int L, int D, int s, int c);
 
 /* Workspace bytes needed by dca_attn_decode: per (sequence, query head,
- * split of 1024 keys) an unnormalised fp32 output row plus running max and
- * sum.  Returns 0 for unsupported arguments. */
+ * split of the cache) an unnormalised fp32 output row plus running max and
+ * sum.  Splits hold 2048 keys when B * ceil(Hq/8) * ceil(Tcap/2048) >= 1184
+ * (at least 8 CTAs per SM on 148 SMs), else 1024.  Returns 0 for unsupported
+ * arguments. */
 size_t dca_attn_decode_workspace(int B, int Hq, int D, int Tcap);
 
 /* DCA decode of one new token per sequence.  q [B][Hq][D] is the UNROTATED

@@ -3,7 +3,7 @@
 // 100k+ Context Guide, "Strategic Recommendations", item 3: pair DCA with
 // FlashDecoding, i.e. split the cache across SMs) followed by an LSE merge.
 //
-// Kernel 1, one CTA per (split of kDecSplit keys, kv head, group of <= 8
+// Kernel 1, one CTA per (split of 1024 or 2048 keys, kv head, group of <= 8
 // query heads, sequence):
 //   * prologue: rotate the group's queries at the three DCA positions of
 //     i = t[b] (intra i mod s, successive min(s + i mod s, c - 1), inter c - 1)
@@ -28,10 +28,21 @@ namespace dec_path {
 
 constexpr int kDecKeys = 64;      // keys per pipeline stage
 constexpr int kDecStages = 3;
-constexpr int kDecSplit = 1024;   // keys per CTA
 constexpr int kDecHeads = 8;      // query heads per CTA (MMA N)
 constexpr int kDecThreads = 160;  // 4 consumer warps + 1 producer warp
 constexpr int kBoxBytes = kDecKeys * 128;  // one [64 keys x 64 dims] bf16 box
+
+// Keys per split CTA.  Longer splits write fewer partials and give each CTA a
+// longer TMA stream (2048: 6.43 TB/s on 16 sequences of 32k-64k keys, 1024:
+// 6.07); shorter ones keep small problems spread over the SMs.  2048 while
+// that still makes at least 8 CTAs per SM of the 148, else 1024; chosen from
+// (B, Hq, Tcap) alone so that the workspace query and the launch agree.
+constexpr int kDecSplitShort = 1024, kDecSplitLong = 2048;
+inline int decode_split_keys(int B, int Hq, int Tcap) {
+  const long long ctas = (long long)B * ((Hq + kDecHeads - 1) / kDecHeads) *
+                         ((Tcap + kDecSplitLong - 1) / kDecSplitLong);
+  return ctas >= 8LL * 148 ? kDecSplitLong : kDecSplitShort;
+}
 
 template <int D>
 struct DecSmem {
@@ -54,8 +65,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const __nv_bfloat16* __restrict__ q, const int* __restrict__ t, float* __restrict__ Opart,
     float* __restrict__ MLpart, int Hq, int Hkv, int Tcap, int s, int c, double log2_base,
-    float scale_log2, int nsplit_max, int n_hg, const int* __restrict__ block_table,
-    int max_blocks, int block_rows, int num_blocks) {
+    float scale_log2, int nsplit_max, int split, int n_hg,
+    const int* __restrict__ block_table, int max_blocks, int block_rows, int num_blocks) {
   using SM = DecSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -76,9 +87,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     return;
   }
   const int n_keys = tb + 1;
-  const int k_begin = sp * kDecSplit;
+  const int k_begin = sp * split;
   if (k_begin >= n_keys) return;  // uniform across the CTA
-  const int k_end = min(k_begin + kDecSplit, n_keys);
+  const int k_end = min(k_begin + split, n_keys);
   const int n_tiles = (k_end - k_begin + kDecKeys - 1) / kDecKeys;
   const int h_base = hk * G + hg * kDecHeads;
   const int n_heads = min(kDecHeads, G - hg * kDecHeads);
@@ -313,7 +324,8 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const float* __restrict
                                                          const int* __restrict__ t,
                                                          __nv_bfloat16* __restrict__ O,
                                                          float* __restrict__ LSE, int Hq,
-                                                         int Tcap, int nsplit_max) {
+                                                         int Tcap, int nsplit_max,
+                                                         int split) {
   __shared__ float stat_s[2];
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int tb = t[b];
@@ -322,7 +334,7 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const float* __restrict
     if (d == 0) LSE[(size_t)b * Hq + h] = __int_as_float(0x7fc00000);
     return;
   }
-  const int n = (tb + 1 + kDecSplit - 1) / kDecSplit;
+  const int n = (tb + split) / split;  // splits holding keys 0 .. tb
   const size_t base = ((size_t)b * Hq + h) * nsplit_max;
   // warp 0: max of the split maxima and the total weighted sum, reading the
   // splits' (max, sum) pairs in parallel
@@ -376,7 +388,8 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
       !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Vc, 4, dims, strides, box,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const int nsplit = (Tcap + kDecSplit - 1) / kDecSplit;
+  const int split = decode_split_keys(B, Hq, Tcap);
+  const int nsplit = (Tcap + split - 1) / split;
   const int G = Hq / Hkv;
   const int n_hg = (G + kDecHeads - 1) / kDecHeads;
   float* Opart = static_cast<float*>(workspace);
@@ -389,12 +402,12 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
   kern<<<grid, kDecThreads, smem, stream>>>(tmK, tmV, static_cast<const __nv_bfloat16*>(q), t,
                                             Opart, MLpart, Hq, Hkv, Tcap, s, c,
                                             log2((double)base),
-                                            scale * 1.4426950408889634f, nsplit, n_hg,
+                                            scale * 1.4426950408889634f, nsplit, split, n_hg,
                                             block_table, max_blocks, block_rows, num_blocks);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_merge_kernel<D><<<dim3(Hq, B), D, 0, stream>>>(
-      Opart, MLpart, t, static_cast<__nv_bfloat16*>(O), LSE, Hq, Tcap, nsplit);
+      Opart, MLpart, t, static_cast<__nv_bfloat16*>(O), LSE, Hq, Tcap, nsplit, split);
   return cudaGetLastError();
 }
 
@@ -403,7 +416,8 @@ cudaError_t launch_decode_t(const void* q, const void* Kc, const void* Vc, const
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int Tcap) {
   using namespace dec_path;
-  const size_t nsplit = ((size_t)Tcap + kDecSplit - 1) / kDecSplit;
+  const int split = decode_split_keys(B, Hq, Tcap);
+  const size_t nsplit = ((size_t)Tcap + split - 1) / split;
   return (size_t)B * Hq * nsplit * (D + 2) * sizeof(float);
 }
 

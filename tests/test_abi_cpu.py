@@ -52,9 +52,12 @@ def test_workspace_queries(lib):
     assert dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D) == up(q) + up(k)
     assert dca.dca_attn_prefill_workspace(1, 10, 3, 2, 64) == 0  # Hq % Hkv
     assert dca.dca_attn_prefill_workspace(1, 10, 2, 2, 96) == 0  # D
-    # decode: one fp32 row + (max, sum) per (b, head, split of 1024 keys)
-    assert dca.dca_attn_decode_workspace(16, 64, 128, 65536) == 16 * 64 * 64 * 130 * 4
+    # decode: one fp32 row + (max, sum) per (b, head, split); splits of 2048
+    # keys while B * ceil(Hq/8) * ceil(Tcap/2048) >= 1184, else of 1024
+    assert dca.dca_attn_decode_workspace(16, 64, 128, 65536) == 16 * 64 * 32 * 130 * 4
     assert dca.dca_attn_decode_workspace(2, 8, 64, 1025) == 2 * 8 * 2 * 66 * 4
+    assert dca.dca_attn_decode_workspace(4, 64, 128, 65536) == 4 * 64 * 64 * 130 * 4
+    assert dca.dca_attn_decode_workspace(5, 64, 128, 65536) == 5 * 64 * 32 * 130 * 4
     # chunked prefill: three fp16 query rotations of the chunk + fp16 keys 0 .. t0+Lq-1
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, 50) == (
         up(3 * 2 * 100 * 8 * 128 * 2) + up(2 * 150 * 2 * 128 * 2))
