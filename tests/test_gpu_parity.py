@@ -43,11 +43,6 @@ def _prefill_gpu(Q, K, V, s, c, path, base=10000.0):
     return O.cpu(), LSE.cpu()
 
 
-def _path_ok(path, D, s):
-    # the tcgen05 path takes every chunk size and both head dimensions
-    return path in (dca.DCA_PATH_GENERAL, dca.DCA_PATH_TCGEN05)
-
-
 # ---------------------------------------------------------------------------
 # index rule
 # ---------------------------------------------------------------------------
@@ -164,8 +159,6 @@ SMALL = [  # (B, L, Hq, Hkv, D, s, c)
 @pytest.mark.parametrize("case", SMALL, ids=[str(c) for c in SMALL])
 def test_prefill_small_full(case, path):
     B, L, Hq, Hkv, D, s, c = case
-    if not _path_ok(path, D, s):
-        pytest.skip("shape outside the tcgen05 path")
     cfg = dict(B=B, L=L, Hq=Hq, Hkv=Hkv, D=D)
     Q, K, V = W.make_prefill_inputs(cfg, seed=L)
     O, LSE = _prefill_gpu(Q, K, V, s, c, path)
@@ -205,8 +198,6 @@ def test_prefill_closed_forms_on_gpu():
 @pytest.mark.parametrize("name", ["llama2_7b_16k", "llama2_70b_32k", "prefill_100k"])
 def test_prefill_workload_sampled(name, path):
     cfg = W.CONFIGS[name]
-    if not _path_ok(path, cfg["D"], cfg["s"]):
-        pytest.skip("shape outside the tcgen05 path")
     Q, K, V = W.make_prefill_inputs(cfg)
     O, LSE = _prefill_gpu(Q, K, V, cfg["s"], cfg["c"], path)
     rows = pu.sample_rows(cfg["L"], cfg["s"], cfg["c"])
@@ -287,6 +278,23 @@ def test_decode_workload():
           f"LSE rel {lse:.3e}")
     pu.assert_close(mx, mean, lse, "decode_b16")
     assert torch.isfinite(O.float()).all()
+
+
+def test_decode_long_splits_with_short_sequences():
+    # 8 sequences x 8 head groups x 19 splits = 1216 CTAs: the launch takes
+    # 2048-key splits; positions on both sides of split and tile edges, the
+    # first key alone and the last cache row
+    cfg = dict(B=8, Hq=64, Hkv=8, D=128, Tcap=19 * 2048, t_lo=0, t_hi=1)
+    _, q, Kc, Vc = W.make_decode_inputs(cfg, seed=9)
+    t = torch.tensor([0, 1, 63, 2047, 2048, 2049, 20000, 19 * 2048 - 1], dtype=torch.int32)
+    s, c = 3072, 4096
+    O, LSE = _decode_gpu(t, q, Kc, Vc, s, c)
+    heads = pu.sample_heads(cfg["Hq"], cfg["Hkv"])
+    mx, mean, lse = _decode_compare(O, LSE, t, q, Kc, Vc, s, c, heads=heads)
+    print(f"decode, 2048-key splits: O max {mx:.3e} mean {mean:.3e} LSE rel {lse:.3e}")
+    pu.assert_close(mx, mean, lse, "decode 2048-key splits")
+    # t = 0: every head returns its kv head's only value
+    assert (O[0].float() - Vc[0, 0].float().repeat_interleave(8, dim=0)).abs().max() <= 2e-2
 
 
 def test_decode_equals_prefill_row_on_gpu():
