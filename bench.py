@@ -440,11 +440,15 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                      map, G = 8, W = 1024 (dca_attn_prefill_selfextend);
       prefill_varlen a packed batch of eight Llama-2 7B prompts of mixed length
                      (dca_attn_prefill_varlen, RoPE included);
+      prefill_varlen_chunk  the next chunks (256 .. 2048 tokens) of eight
+                     sequences with 0 .. 14000 cached tokens, packed
+                     (dca_attn_prefill_varlen_chunk);
       decode_paged   the decode workload over a paged copy of its caches
                      (dca_attn_decode_paged, 256-row blocks in random order);
       kv_append      one decoded token appended per sequence of the decode
                      batch (dca_kv_append), 100 calls back to back."""
     import ctypes
+    import numpy as np
     P = ctypes.c_void_p
     B, L, Hq, D = Q.shape
     Hkv = K.shape[2]
@@ -609,6 +613,45 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
                                      else "per-row intervals"),
         "launches_per_call": 2}
     del Qv, Kv, Vv, vws, Ov, Lv
+
+    # packed chunks over per-sequence caches: Llama-2 7B heads, eight
+    # sequences with seeded 0 .. 14000 cached tokens and new chunks of
+    # 256 .. 2048 tokens (RoPE, cache writes, key conversion and attention)
+    rng = np.random.default_rng(7)
+    t0c = [int(x) for x in rng.integers(0, 14001, 8)]
+    lensc = [int(x) for x in rng.integers(256, 2049, 8)]
+    Tc, Tcap_c = sum(lensc), 16384
+    gen_c = torch.Generator(device=dev)
+    gen_c.manual_seed(7)
+    Qc = torch.randn(Tc, Hqv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+    Kn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+    Vn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+    Kcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+    Vcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+    cu_c = torch.zeros(9, dtype=torch.int32)
+    cu_c[1:] = torch.cumsum(torch.tensor(lensc), 0).to(torch.int32)
+    cu_c, t0_d = cu_c.to(dev), torch.tensor(t0c, dtype=torch.int32, device=dev)
+    max_kv = max(a + n for a, n in zip(t0c, lensc))
+    wsz = dca.dca_attn_prefill_varlen_chunk_workspace(8, Tc, max_kv, Hqv, Hkvv, Dv)
+    cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    Occ = torch.empty_like(Qc)
+    Lcc = torch.empty(Hqv, Tc, dtype=torch.float32, device=dev)
+
+    def varlen_chunk():
+        st = lib.dca_attn_prefill_varlen_chunk(
+            P(Qc.data_ptr()), P(Kn.data_ptr()), P(Vn.data_ptr()), P(Kcc.data_ptr()),
+            P(Vcc.data_ptr()), P(Occ.data_ptr()), P(Lcc.data_ptr()), P(cu_c.data_ptr()),
+            P(t0_d.data_ptr()), 8, max(lensc), Tc, max_kv, Hqv, Hkvv, Dv, Tcap_c, vc["s"],
+            vc["c"], vc["base"], 0.0, P(cws.data_ptr()), wsz, P(stream.cuda_stream))
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+    ms = timed(varlen_chunk)
+    out["prefill_varlen_chunk"] = {
+        "value": W.varlen_chunk_flops(t0c, lensc, Hqv, Dv) / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "ms": ms, "t0": t0c, "lens": lensc,
+        "path": "chunk RoPE + key conversion + tcgen05 per-row intervals",
+        "launches_per_call": 3}
+    del Qc, Kn, Vn, Kcc, Vcc, cws, Occ, Lcc
 
     # decode over a paged cache: the decode workload's caches scattered into
     # 256-row blocks in a seeded random physical order

@@ -211,6 +211,49 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
                                     int Hkv, int D, int t0, int Tcap, int s, int c, float base,
                                     float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/* Workspace bytes for dca_attn_prefill_varlen_chunk: the fp16 query
+ * rotations [3][T][Hq][D] and fp16 keys [B][max_kv][Hkv][D], each rounded up
+ * to 256 bytes.  Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq, int Hkv,
+                                               int D);
+
+/* Chunked prefill of a packed batch against per-sequence caches: the next
+ * chunk of each of B sequences, of different lengths and at different
+ * positions, in one call (dca_attn_prefill_chunk with a cache offset per
+ * sequence, on dca_attn_prefill_varlen's packed layout).  Sequence b already
+ * holds t0[b] tokens in its caches; its new rows are absolute indices
+ * t0[b] .. t0[b]+n_b-1, each row of a one-shot DCA prefill over that
+ * sequence alone (Guide, "Strategic Recommendations", item 1).
+ *   Q [T][Hq][D], K, V [T][Hkv][D]: the new tokens' UNROTATED queries and keys
+ *     and their values, bf16, packed: sequence b owns rows cu_seqlens[b] ..
+ *     cu_seqlens[b+1]-1 (n_b of them).
+ *   cu_seqlens: DEVICE int32 [B+1] as for dca_attn_prefill_varlen;
+ *     t0: DEVICE int32 [B]; max_seqlen (host) >= every n_b; max_kv (host,
+ *     <= Tcap) >= every t0[b] + n_b.
+ *   Kcache, Vcache [B][Tcap][Hkv][D] bf16: rows 0 .. t0[b]-1 of entry b hold
+ *     keys already rotated at j mod s and their values.  This call writes
+ *     the new rotated keys and values to rows t0[b] .. t0[b]+n_b-1 of entry
+ *     b and zeroes value rows t0[b]+n_b .. up to the next multiple of 128
+ *     (at most max_kv-1; positions the sequence does not have yet, read with
+ *     zero weight by its last key tile); no other row changes.
+ *   O [T][Hq][D] bf16, LSE [Hq][T] fp32: results for the packed rows; rows of
+ *     no sequence are left untouched.
+ * Kernels: the fused RoPE kernel in chunk form, the key conversion to fp16
+ * of rows 0 .. t0[b]-1, then the per-row-interval tcgen05 kernel with each
+ * sequence's offset.  Offsets that break the rules above are checked where
+ * the kernels read them: that sequence is skipped (no cache row, O or LSE
+ * written) and the device error word is set (DCA_ERR_INVALID_ARG at the next
+ * dca_sync_status).  The call owns no memory; `workspace`
+ * (dca_attn_prefill_varlen_chunk_workspace bytes) is the caller's.
+ * D in {64, 128}.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const void* V,
+                                           void* Kcache, void* Vcache, void* O, float* LSE,
+                                           const int* cu_seqlens, const int* t0, int B,
+                                           int max_seqlen, int T, int max_kv, int Hq, int Hkv,
+                                           int D, int Tcap, int s, int c, float base,
+                                           float scale, void* workspace, size_t ws_bytes,
+                                           void* stream);
+
 /* Workspace bytes for dca_attn_prefill_selfextend: the neighbour and grouped
  * rotations of Q [2][B][L][Hq][D] and K [2][B][L][Hkv][D], fp16, each rounded
  * up to 256 bytes.  Returns 0 for unsupported arguments. */

@@ -26,6 +26,7 @@ __all__ = [
     "dca_attn_prefill_3pass_workspace", "dca_attn_prefill_3pass",
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
     "dca_attn_prefill_varlen_workspace", "dca_attn_prefill_varlen",
+    "dca_attn_prefill_varlen_chunk_workspace", "dca_attn_prefill_varlen_chunk",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
     "dca_attn_decode_paged", "dca_kv_append_paged",
@@ -53,6 +54,9 @@ _SIGS = {
     "dca_prefill_path": (_I, [_I, _I, _I, _I]),
     "dca_attn_prefill_3pass_workspace": (_Z, [_I, _I, _I, _I, _I]),
     "dca_attn_prefill_varlen_workspace": (_Z, [_I, _I, _I, _I]),
+    "dca_attn_prefill_varlen_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "dca_attn_prefill_varlen_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
+                                           _I, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
     "dca_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                      _F, _P, _Z, _P]),
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -243,6 +247,42 @@ def dca_attn_prefill_varlen(Q, K, V, cu_seqlens, max_seqlen, s, c, base=10000.0,
     _check(lib().dca_attn_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
                                          _ptr(cu_seqlens), B, int(max_seqlen), T, Hq, Hkv, D, s,
                                          c, base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_varlen_chunk_workspace(B: int, T: int, max_kv: int, Hq: int, Hkv: int,
+                                            D: int) -> int:
+    return int(lib().dca_attn_prefill_varlen_chunk_workspace(B, T, max_kv, Hq, Hkv, D))
+
+
+def dca_attn_prefill_varlen_chunk(Q, K, V, Kcache, Vcache, cu_seqlens, t0, max_seqlen, max_kv,
+                                  s, c, base=10000.0, scale=0.0, workspace=None, O=None,
+                                  LSE=None):
+    """Packed chunks over per-sequence caches.  Q [T, Hq, D], K, V [T, Hkv, D]
+    bf16 (sequence b's new tokens at rows cu_seqlens[b] .. cu_seqlens[b+1]-1);
+    Kcache, Vcache [B, Tcap, Hkv, D] bf16 holding t0[b] cached rows each;
+    cu_seqlens int32 [B+1] and t0 int32 [B] on the device.  Returns
+    (O [T, Hq, D] bf16, LSE [Hq, T] fp32) and extends the caches."""
+    _need(Q, "Q", torch.bfloat16, 3)
+    _need(K, "K", torch.bfloat16, 3)
+    _need(V, "V", torch.bfloat16, 3)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    _need(t0, "t0", torch.int32, 1)
+    T, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    B, Tcap = Kcache.shape[:2]
+    nbytes = dca_attn_prefill_varlen_chunk_workspace(B, T, int(max_kv), Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    O = torch.empty_like(Q) if O is None else O
+    LSE = torch.empty((Hq, T), dtype=torch.float32, device=Q.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 3)
+    _need(LSE, "LSE", torch.float32, 2)
+    _check(lib().dca_attn_prefill_varlen_chunk(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(Kcache), _ptr(Vcache), _ptr(O), _ptr(LSE),
+        _ptr(cu_seqlens), _ptr(t0), B, int(max_seqlen), T, int(max_kv), Hq, Hkv, D, Tcap, s, c,
+        base, scale, _ptr(ws), ws.numel(), _stream(Q)))
     return O, LSE
 
 

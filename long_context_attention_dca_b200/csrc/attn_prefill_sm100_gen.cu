@@ -62,7 +62,7 @@ struct Lay2 {
   static constexpr int kSmMisc = Lay<D>::kSmBar + kNumBars * 8;  // TMEM base, abort flag
   static constexpr int kSmPlan = kSmMisc + 16;                    // the CTA's visit plan
   static constexpr int kSmSeq = kSmPlan + 128;                    // its sequence's rows
-  static constexpr int kSmTotal = kSmSeq + 32 + 1024;
+  static constexpr int kSmTotal = kSmSeq + 48 + 1024;
   static_assert(kSmTotal <= 232448, "shared memory budget");
 };
 constexpr uint32_t kTmemCols = 512;
@@ -189,17 +189,20 @@ __device__ __forceinline__ float row_max_range(uint32_t (&v)[4][32], int clo, in
   return row_max(v);
 }
 
-template <int D, class Rule>
+// kSeqOff: the queries' absolute offsets come per sequence from t0s (packed
+// chunks over caches) instead of the q_off argument.
+template <int D, class Rule, bool kSeqOff>
 __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
-    int q_off, int group_units, const int* __restrict__ cu_seqlens, int T) {
+    int q_off, int group_units, const int* __restrict__ cu_seqlens, int T,
+    const int* __restrict__ t0s, int kv_rows) {
   using LD = Lay<D>;
   constexpr int kHalves = LD::kHalves, kTileBytes = LD::kTileBytes;
   constexpr int kSmQ = LD::kSmQ, kSmK = LD::kSmK, kSmV = LD::kSmV, kSmBar = LD::kSmBar;
   constexpr int kSmMisc = Lay2<D>::kSmMisc, kSmPlan = Lay2<D>::kSmPlan, kSmSeq = Lay2<D>::kSmSeq;
-  static_assert(sizeof(Plan) <= 128 && sizeof(SeqSpan) <= 32, "plan / span slots");
+  static_assert(sizeof(Plan) <= 128 && sizeof(SeqSpan) <= 48, "plan / span slots");
   constexpr uint32_t kOCols = (uint32_t)D;  // O accumulator columns per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -220,24 +223,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const int hk = h / (Hq / Hkv);
   const int q0_loc = m * 2 * kTile;          // row of this call
   SeqSpan sq0;
-  if (!seq_span(cu_seqlens, b, B, L, T, sq0)) {  // reported, no work
+  if (!seq_span(cu_seqlens, t0s, b, B, L, T, q_off, kv_rows, sq0)) {  // reported, no work
     if (tid == 0) report_error(kDevBadArg, 312);
     return;
   }
   if (q0_loc >= sq0.n) return;  // the pair lies past a shorter sequence's end
-  const int last_row = q_off + sq0.n - 1;    // absolute
-  int rows_lo[2], rows_hi[2];
-  for (int x = 0; x < 2; ++x) {
-    rows_lo[x] = q_off + q0_loc + x * kTile;
-    rows_hi[x] = min(rows_lo[x] + kTile - 1, last_row);
-  }
   const Plan& pl = *reinterpret_cast<const Plan*>(smem + kSmPlan);
-  // read from shared memory where used (fewer live registers)
-  const SeqSpan& sq = *reinterpret_cast<const SeqSpan*>(smem + kSmSeq);
+  // read from shared memory where used (fewer live registers; volatile so
+  // that each use reloads instead of holding a register)
+  const volatile SeqSpan& sq = *reinterpret_cast<const volatile SeqSpan*>(smem + kSmSeq);
 
   if (tid == 0) {
+    const int last_row = sq0.q_off + sq0.n - 1;  // absolute
+    int rows_lo[2], rows_hi[2];
+    for (int x = 0; x < 2; ++x) {
+      rows_lo[x] = sq0.q_off + q0_loc + x * kTile;
+      rows_hi[x] = min(rows_lo[x] + kTile - 1, last_row);
+    }
     *reinterpret_cast<Plan*>(smem + kSmPlan) = make_plan(rule, rows_lo, rows_hi);
-    *reinterpret_cast<SeqSpan*>(smem + kSmSeq) = sq0;
+    *reinterpret_cast<SeqSpan*>(smem + kSmSeq) = sq0;  // published by the barrier below
     for (int i = 0; i < kNumQSlots; ++i) {
       mbar_init(bar(kQFull + i), 1);
       mbar_init(bar(kQEmpty + i), 1);
@@ -303,11 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
             break;
           mbar_arrive_expect_tx(bar(kKFull + sg), kTileBytes);
           const uint32_t kd = sbase + kSmK + sg * kTileBytes;
-          const int kb = rule.kplane(pl.pc[k]) * sq.nb + sq.bt;  // key plane of the piece
+          const int kb = rule.kplane(pl.pc[k]) * sq.knb + sq.kbt;  // key plane of the piece
 #pragma unroll
           for (int hf = 0; hf < kHalves; ++hf)
             tma_load_4d(kd + hf * kBox, &tmK, bar(kKFull + sg), hf * 64, hk,
-                        sq.row0 + t * kTile, kb);
+                        sq.krow0 + t * kTile, kb);
           k_last[sg] = st;
           if (first && !(ok = load_q(2 * k + 1, pl.pc[k]))) break;
           if (st >= 2 &&
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
 #pragma unroll
           for (int hf = 0; hf < kHalves; ++hf)
             tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk,
-                        sq.row0 + t * kTile, sq.bt);
+                        sq.krow0 + t * kTile, sq.kbt);
           v_last[sg] = st;
         }
       }
@@ -428,7 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const int wq = warp & 3;               // TMEM lane quarter
     const int row = wq * 32 + lane;        // row within the tile
     const int i_row = q0_loc + x * kTile + row;  // row of this call
-    const int i_abs = q_off + i_row;
+    // (the offset taken from the kernel arguments, not from the span in
+    // shared memory: that keeps the softmax warps from spilling)
+    int i_abs;
+    if constexpr (kSeqOff) i_abs = __ldg(t0s + b) + i_row;
+    else i_abs = q_off + i_row;
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_addr = t_lane + 128u * (uint32_t)x;
     const uint32_t o_addr = t_lane + 256u + 128u * (uint32_t)x;
@@ -537,13 +545,15 @@ template <int D, class Rule>
 cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
                          int B, int L, int Hq, int Hkv, Rule rule, int nq, float scale,
                          cudaStream_t stream, int q_off, int k_rows, int v_rows,
-                         const int* cu_seqlens, int T) {
+                         const int* cu_seqlens, int T, const int* t0s, int kv_rows) {
   if (q_off < 0) return cudaErrorInvalidValue;
   if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
+  if (t0s != nullptr && (cu_seqlens == nullptr || kv_rows < 1)) return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
-  const int Bm = cu_seqlens ? 1 : B;       // tensor batch extent
-  const int Lrows = cu_seqlens ? T : L;    // tensor query rows per batch entry
-  const int Lkv = cu_seqlens ? T : q_off + L;
+  const int Bm = cu_seqlens ? 1 : B;       // query tensor batch extent
+  const int Bk = cu_seqlens && !t0s ? 1 : B;  // key / value tensor batch extent
+  const int Lrows = cu_seqlens ? T : L;    // query tensor rows per batch entry
+  const int Lkv = cu_seqlens ? (t0s ? kv_rows : T) : q_off + L;
   if (k_rows == 0) k_rows = Lkv;
   if (v_rows == 0) v_rows = Lkv;
   CUtensorMap tmQ, tmK, tmV;
@@ -558,8 +568,8 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
   }
   {
     const uint64_t kdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv,
-                               (uint64_t)Rule::kKPlanes * Bm};
-    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)Bm};
+                               (uint64_t)Rule::kKPlanes * Bk};
+    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)Bk};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
     const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
@@ -571,30 +581,36 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
       return cudaErrorInvalidValue;
   }
   constexpr int kSmTotal = Lay2<D>::kSmTotal;
-  auto kern = prefill_attn_gen_kernel<D, Rule>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
-  if (e != cudaSuccess) return e;
   const int num_qt = (L + kTile - 1) / kTile;
-  dim3 grid((unsigned)(((num_qt + 1) / 2) * Hq * B));
-  kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O), LSE,
-                                             B, L, Hq, Hkv, rule, scale * 1.4426950408889634f,
-                                             q_off, B * Hkv,  // one group: longest first
-                                             cu_seqlens, T);
-  return cudaGetLastError();
+  const dim3 grid((unsigned)(((num_qt + 1) / 2) * Hq * B));
+  auto run = [&](auto kern) -> cudaError_t {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, kSmTotal, stream>>>(tmQ, tmK, tmV, static_cast<__nv_bfloat16*>(O),
+                                               LSE, B, L, Hq, Hkv, rule,
+                                               scale * 1.4426950408889634f, q_off,
+                                               B * Hkv,  // one group: longest first
+                                               cu_seqlens, T, t0s, Lkv);
+    return cudaGetLastError();
+  };
+  if (t0s == nullptr) return run(prefill_attn_gen_kernel<D, Rule, false>);
+  if constexpr (Rule::kKPlanes == 1) return run(prefill_attn_gen_kernel<D, Rule, true>);
+  return cudaErrorInvalidValue;  // per-sequence offsets: DCA rule only
 }
 
 template <class Rule>
 cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
                        int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
                        cudaStream_t stream, int q_off, int k_rows, int v_rows,
-                       const int* cu_seqlens = nullptr, int T = 0) {
+                       const int* cu_seqlens = nullptr, int T = 0, const int* t0s = nullptr,
+                       int kv_rows = 0) {
   if (D == 64)
     return launch_gen_d<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream, q_off,
-                            k_rows, v_rows, cu_seqlens, T);
+                            k_rows, v_rows, cu_seqlens, T, t0s, kv_rows);
   if (D == 128)
     return launch_gen_d<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream,
-                             q_off, k_rows, v_rows, cu_seqlens, T);
+                             q_off, k_rows, v_rows, cu_seqlens, T, t0s, kv_rows);
   return cudaErrorInvalidValue;
 }
 
@@ -607,11 +623,12 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off, int k_rows, int v_rows,
-                                          const int* cu_seqlens, int T) {
+                                          const int* cu_seqlens, int T, const int* t0s,
+                                          int kv_rows) {
   if (s < 1) return cudaErrorInvalidValue;
   return gen_path::launch_gen(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, D,
                               gen_path::DcaIntervals{s}, 3, scale, stream, q_off, k_rows,
-                              v_rows, cu_seqlens, T);
+                              v_rows, cu_seqlens, T, t0s, kv_rows);
 }
 
 // SelfExtend on the same kernel: Qse, Kse [2][B][L][H][D] fp16 (neighbour,

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   const int q0 = m * 2 * kTile;              // absolute
   const int q0_loc = q0 - pair_off * 2 * kTile;
   SeqSpan sq;
-  if (!seq_span(cu_seqlens, b, B, L, T, sq)) {  // reported, no work
+  if (!seq_span(cu_seqlens, nullptr, b, B, L, T, pair_off * 2 * kTile, 0, sq)) {  // reported
     if (tid == 0) report_error(kDevBadArg, 311);
     return;
   }
@@ -168,16 +168,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
           break;
         mbar_arrive_expect_tx(bar(kKFull + st), kTileBytes);
         const uint32_t kd = sbase + kSmK + st * kTileBytes;
-        tma_load_4d(kd, &tmK, bar(kKFull + st), 0, hk, sq.row0 + i * kTile, sq.bt);
-        tma_load_4d(kd + kBox, &tmK, bar(kKFull + st), 64, hk, sq.row0 + i * kTile, sq.bt);
+        tma_load_4d(kd, &tmK, bar(kKFull + st), 0, hk, sq.krow0 + i * kTile, sq.kbt);
+        tma_load_4d(kd + kBox, &tmK, bar(kKFull + st), 64, hk, sq.krow0 + i * kTile, sq.kbt);
         k_last[st] = i;
         if (boundary && !(ok = load_q(2 * p + 1))) break;
         if (i >= 2 && !(ok = mbar_wait(bar(kVEmpty + st), ((i >> 1) + 1) & 1, abort_flag, 403)))
           break;
         mbar_arrive_expect_tx(bar(kVFull + st), kTileBytes);
         const uint32_t vd = sbase + kSmV + st * kTileBytes;
-        tma_load_4d(vd, &tmV, bar(kVFull + st), 0, hk, sq.row0 + i * kTile, sq.bt);
-        tma_load_4d(vd + kBox, &tmV, bar(kVFull + st), 64, hk, sq.row0 + i * kTile, sq.bt);
+        tma_load_4d(vd, &tmV, bar(kVFull + st), 0, hk, sq.krow0 + i * kTile, sq.kbt);
+        tma_load_4d(vd + kBox, &tmV, bar(kVFull + st), 64, hk, sq.krow0 + i * kTile, sq.kbt);
         v_last[st] = i;
       }
       // drain: every issued copy has landed before shared memory is released

@@ -360,6 +360,61 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 
+size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq, int Hkv,
+                                               int D) {
+  if (B < 0 || T < 0 || max_kv < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128))
+    return 0;
+  return align256((size_t)3 * T * Hq * D * 2) + align256((size_t)B * max_kv * Hkv * D * 2);
+}
+
+dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const void* V,
+                                           void* Kcache, void* Vcache, void* O, float* LSE,
+                                           const int* cu_seqlens, const int* t0, int B,
+                                           int max_seqlen, int T, int max_kv, int Hq, int Hkv,
+                                           int D, int Tcap, int s, int c, float base,
+                                           float scale, void* workspace, size_t ws_bytes,
+                                           void* stream) {
+  const char* fn = "dca_attn_prefill_varlen_chunk";
+  dca_status_t st = check_heads(fn, B, max_seqlen, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (T < 0) return fail(DCA_ERR_INVALID_ARG, "%s: T=%d", fn, T);
+  if (Tcap < 1 || max_kv < 1 || max_kv > Tcap)
+    return fail(DCA_ERR_INVALID_ARG, "%s: need 1 <= max_kv=%d <= Tcap=%d", fn, max_kv, Tcap);
+  if (auto_path(D, s) != DCA_PATH_TCGEN05)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: library built without the tcgen05 path", fn);
+  if ((long long)B * max_seqlen == 0 || T == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(Kcache);
+  DCA_CHECK_PTR(Vcache);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+      t0 == nullptr || (reinterpret_cast<uintptr_t>(t0) & 3u))
+    return fail(DCA_ERR_INVALID_ARG, "%s: cu_seqlens / t0 null or not 4-byte aligned", fn);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = dca_attn_prefill_varlen_chunk_workspace(B, T, max_kv, Hq, Hkv, D);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  // As dca_attn_prefill_chunk, per sequence: the new keys rotated here go to
+  // the bf16 cache and, rounded once, to fp16; cache rows 0 .. t0[b]-1 are
+  // converted to fp16 as stored.
+  void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * T * Hq * D * 2);
+  cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, 1, T, Hq, Hkv, D,
+                                    0, Tcap, max_kv, s, c, base, strm, cu_seqlens, B, t0);
+  if (e == cudaSuccess)
+    e = launch_keys_to_f16(Kcache, kf16, B, max_kv, Tcap, max_kv, Hkv, D, strm, t0, cu_seqlens,
+                           Vcache);
+  if (e == cudaSuccess)
+    e = launch_prefill_attn_sm100_gen(workspace, kf16, Vcache, O, LSE, B, max_seqlen, Hq, Hkv, D,
+                                      s, sc, strm, 0, max_kv, Tcap, cu_seqlens, T, t0, max_kv);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D) {
   if (B < 0 || L < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
   return align256((size_t)2 * B * L * Hq * D * 2) + align256((size_t)2 * B * L * Hkv * D * 2);

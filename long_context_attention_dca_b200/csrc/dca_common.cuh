@@ -103,29 +103,47 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
-// Where sequence b's rows sit in the prefill tensors.  A padded batch holds
-// sequence b at tensor batch coordinate b, rows 0 .. L-1.  A packed batch
-// (cu_seqlens != null) is one tensor of T rows; sequence b owns rows
-// cu_seqlens[b] .. cu_seqlens[b+1]-1, at most L (the longest sequence), and
-// its local row r is query index r of its own prefill.
+// Where sequence b's rows sit in the prefill tensors.
+//   * Padded batch (cu_seqlens null): queries at tensor batch coordinate b,
+//     rows 0 .. L-1, at absolute indices q_off + r (q_off the call's chunk
+//     start); keys and values at batch coordinate b, rows from 0.
+//   * Packed batch (cu_seqlens set, t0 null): every tensor is one batch entry
+//     of T rows; sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (at
+//     most L of them) for its queries and for its keys and values, and its
+//     local row r is query index r of its own prefill.
+//   * Packed chunks over caches (cu_seqlens and t0 set): the queries are
+//     packed as above, but sequence b's local row r is absolute index
+//     t0[b] + r, and its keys and values are rows 0 .. t0[b]+n-1 of batch
+//     entry b of tensors with kv_rows rows per entry.
 struct SeqSpan {
-  int row0;  // tensor row of local row 0
-  int n;     // rows of the sequence
-  int bt;    // tensor batch coordinate
-  int nb;    // tensor batch extent
-  int rows;  // tensor rows per batch entry (the O / LSE row stride)
+  int row0;   // query tensor row of local row 0
+  int n;      // query rows of the sequence
+  int bt;     // query tensor batch coordinate
+  int nb;     // query tensor batch extent
+  int rows;   // query tensor rows per batch entry (the O / LSE row stride)
+  int q_off;  // absolute index of local row 0
+  int krow0;  // key / value tensor row of absolute index 0
+  int kbt;    // key / value tensor batch coordinate
+  int knb;    // key / value tensor batch extent (per key plane)
 };
-// False when the packed offsets of sequence b are not a valid span of at
-// most L rows inside [0, T).
-__device__ __forceinline__ bool seq_span(const int* cu_seqlens, int b, int B, int L, int T,
-                                         SeqSpan& sq) {
+// False when the packed offsets (or cache offsets) of sequence b do not give
+// a valid span: queries of at most L rows inside [0, T), keys inside
+// [0, kv_rows).
+__device__ __forceinline__ bool seq_span(const int* cu_seqlens, const int* t0, int b, int B,
+                                         int L, int T, int q_off, int kv_rows, SeqSpan& sq) {
   if (cu_seqlens == nullptr) {
-    sq = SeqSpan{0, L, b, B, L};
+    sq = SeqSpan{0, L, b, B, L, q_off, 0, b, B};
     return true;
   }
   const int a = __ldg(cu_seqlens + b), e = __ldg(cu_seqlens + b + 1);
-  sq = SeqSpan{a, e - a, 0, 1, T};
-  return a >= 0 && e >= a && e - a <= L && e <= T;
+  const bool ok = a >= 0 && e >= a && e - a <= L && e <= T;
+  if (t0 == nullptr) {
+    sq = SeqSpan{a, e - a, 0, 1, T, 0, a, 0, 1};
+    return ok;
+  }
+  const int off = __ldg(t0 + b);
+  sq = SeqSpan{a, e - a, 0, 1, T, off, 0, b, B};
+  return ok && off >= 0 && (long long)off + (e - a) <= kv_rows;
 }
 
 // Dispatch order of the two-tile prefill kernels' (query-tile pair, head,

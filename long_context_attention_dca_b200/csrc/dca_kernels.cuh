@@ -27,10 +27,15 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
 // fp16; rotated keys go in bf16 to cache rows t0 + r (pitch Tcap; skipped when
 // Kcache is null) and in fp16 to rows t0 + r of Kf16 (kh_rows rows per
 // sequence); values to cache rows t0 + r (skipped when Vcache is null).
+// Packed form (cu_seqlens device [n_seq+1], B = 1, Lq = T, t0 = 0): row r of
+// sequence b is absolute index t0s[b] + r and writes cache rows of entry b;
+// rows outside every sequence, or of a sequence that would leave the caches,
+// write no cache row.
 cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
                               int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
-                              float base, cudaStream_t stream);
+                              float base, cudaStream_t stream, const int* cu_seqlens = nullptr,
+                              int n_seq = 0, const int* t0s = nullptr);
 // Attention of that chunk over keys 0 .. t0+Lq-1 of Kf16 (k_rows rows per
 // sequence) and V (v_rows rows per sequence) (general path).
 cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* V,
@@ -71,21 +76,30 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
                                          const int* cu_seqlens = nullptr, int T = 0);
 // tcgen05 prefill attention for any chunk size (D = 64 or 128): per-row key
 // intervals per piece, straddling tiles visited once per piece they hold.
-// Same chunk and packed forms as the ping-pong variant (any q_off).
+// Same chunk and packed forms as the ping-pong variant (any q_off), and
+// packed chunks over caches: with cu_seqlens and t0s (device [B]) sequence
+// b's packed query rows sit at absolute indices t0s[b] + r and attend rows
+// 0 .. t0s[b]+r of batch entry b of Krot [B][k_rows pitch] and V [B][v_rows
+// pitch], kv_rows rows valid per entry.
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off = 0, int k_rows = 0, int v_rows = 0,
-                                          const int* cu_seqlens = nullptr, int T = 0);
+                                          const int* cu_seqlens = nullptr, int T = 0,
+                                          const int* t0s = nullptr, int kv_rows = 0);
 // SelfExtend on the per-row-interval tcgen05 kernel (D = 64 or 128).
 cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
                                                  const void* V, void* O, float* LSE, int B,
                                                  int L, int Hq, int Hkv, int D, int W,
                                                  float scale, cudaStream_t stream);
 // Rows 0 .. rows-1 of a bf16 key cache [B][Tcap][Hkv][D] -> the same rows of
-// fp16 [B][out_rows][Hkv][D].
+// fp16 [B][out_rows][Hkv][D]; with t0s (device [B]) only rows below t0s[b],
+// and with cu_seqlens and Vcache too the value-cache rows from each
+// sequence's new end to the next multiple of 128 (at most rows) are zeroed.
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
-                               int out_rows, int Hkv, int D, cudaStream_t stream);
+                               int out_rows, int Hkv, int D, cudaStream_t stream,
+                               const int* t0s = nullptr, const int* cu_seqlens = nullptr,
+                               void* Vcache = nullptr);
 
 // Decode-time append of one token per sequence into pre-rotated caches:
 // contiguous [B][Tcap][Hkv][D] (block_table null) or a paged pool

@@ -127,20 +127,26 @@ constexpr int kRopeThreads = 256;
 // against a cache (kChunk true) writes them in bf16 to cache rows q_off + r of
 // pitch Tcap (Kout, unless null) and in fp16 to rows q_off + r of Kh (kh_rows
 // rows per sequence), and copies the chunk's values into the value cache
-// (unless Vc is null).  A packed batch (cu_seqlens != null, B = 1, L = T rows,
-// kChunk false) holds n_seq sequences, sequence b at rows cu_seqlens[b] ..
-// cu_seqlens[b+1]-1; a row's index is counted from its sequence's first row.
+// (unless Vc is null).  A packed batch (cu_seqlens != null, B = 1, L = T rows)
+// holds n_seq sequences, sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1;
+// a row's index is counted from its sequence's first row, plus t0[b] in the
+// chunk form (t0 device [n_seq], the rows sequence b already has in its
+// caches), where the cache rows written are those of batch entry b.  In the
+// chunk form a row outside every sequence, or of a sequence whose rows would
+// leave the caches, writes nothing to the caches.
 template <int D, bool kChunk>
 __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
     __half* __restrict__ Qrot, void* __restrict__ Kout, int B, int L, int Hq, int Hkv, int s,
     int c, double log2_base, int q_off, int Tcap, const __nv_bfloat16* __restrict__ Vsrc,
     __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh, int kh_rows,
-    const int* __restrict__ cu_seqlens, int n_seq) {
+    const int* __restrict__ cu_seqlens, int n_seq, const int* __restrict__ t0) {
   constexpr int kHalf = D / 2;
   constexpr int kGroups = D / 16;
   __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
   __shared__ int im_s[kRopeRows];               // row index mod s
+  __shared__ int seq_s[kRopeRows];              // chunk form: cache entry (-1: none)
+  __shared__ int pos_s[kRopeRows];              // chunk form: absolute index
   const long long total_rows = (long long)B * L;
   const long long row0 = (long long)blockIdx.x * kRopeRows;
   const int nrows = (int)min((long long)kRopeRows, total_rows - row0);
@@ -150,9 +156,14 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     int im;
     if (cu_seqlens == nullptr) {
       im = (int)(((row % L) + q_off) % s);
+      if constexpr (kChunk) {
+        seq_s[threadIdx.x] = (int)(row / L);
+        pos_s[threadIdx.x] = (int)(row % L) + q_off;
+      }
     } else {
-      // last sequence starting at or before the row (rows of no sequence
-      // are rotated as if they continued the last one; nothing reads them)
+      // last sequence starting at or before the row (outside the chunk form,
+      // rows of no sequence are rotated as if they continued the last one;
+      // nothing reads them)
       const int r = (int)row;
       int lo = 0, hi = n_seq - 1;
       while (lo < hi) {
@@ -160,7 +171,18 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
         if (__ldg(cu_seqlens + mid) <= r) lo = mid;
         else hi = mid - 1;
       }
-      im = max(r - __ldg(cu_seqlens + lo), 0) % s;
+      const int a = __ldg(cu_seqlens + lo);
+      long long i = max(r - a, 0);
+      if constexpr (kChunk) {
+        const int e = __ldg(cu_seqlens + lo + 1);
+        const int off = t0 != nullptr ? __ldg(t0 + lo) : 0;
+        const bool ok = r >= a && r < e && off >= 0 &&
+                        (long long)off + (e - a) <= (long long)min(Tcap, kh_rows);
+        if (ok) i += off;
+        seq_s[threadIdx.x] = ok ? lo : -1;
+        pos_s[threadIdx.x] = (int)i;
+      }
+      im = (int)(i % s);
     }
     im_s[threadIdx.x] = im;
   }
@@ -187,8 +209,9 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const int r = it / (kGroups * heads);
     const long long row = row0 + r;
     if constexpr (kChunk) {
-      const long long seq = row / L;
-      const size_t cache_row = (size_t)(seq * Tcap + (row % L) + q_off);
+      const int seq = seq_s[r];
+      const size_t cache_row = (size_t)seq * Tcap + pos_s[r];
+      if (hh < 2 * Hkv && seq < 0) continue;  // no cache rows for this row
       if (hh >= Hkv && hh < 2 * Hkv) {  // value copy
         if (!write_v) continue;
         const size_t src = (size_t)row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
@@ -218,7 +241,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
           *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
         }
         rotate8<true>(lo, hi, cs, olo, ohi);
-        const size_t hdst = ((size_t)(seq * kh_rows + (row % L) + q_off) * Hkv + hh) * D + g * 8;
+        const size_t hdst = (((size_t)seq * kh_rows + pos_s[r]) * Hkv + hh) * D + g * 8;
         *reinterpret_cast<uint4*>(Kh + hdst) = olo;
         *reinterpret_cast<uint4*>(Kh + hdst + kHalf) = ohi;
         continue;
@@ -318,16 +341,37 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
 
 // bf16 -> fp16 copy of cache rows 0 .. rows-1 (pitch Tcap) to rows of pitch
 // out_rows (exact inside the fp16 range), one 16-byte group per thread,
-// grid-stride.
+// grid-stride.  With t0 (device [B]) sequence b copies only its rows
+// 0 .. t0[b]-1 (none when t0[b] is negative), and with cu_seqlens and Vc it
+// also zeroes value-cache rows e .. min(e rounded up to 128, rows)-1 after
+// the sequence's new end e = t0[b] + its chunk length (rows no key reaches
+// yet, read with zero weight by the last key tile; zero keeps 0 * value
+// finite), provided the sequence's span lies inside the cache.
 __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restrict__ Kc,
                                                           uint4* __restrict__ Kh, int rows,
                                                           int Tcap, int out_rows,
                                                           long long groups_per_row,
-                                                          long long total) {
+                                                          long long total,
+                                                          const int* __restrict__ t0,
+                                                          const int* __restrict__ cu_seqlens,
+                                                          uint4* __restrict__ Vc) {
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
        gid += (long long)gridDim.x * blockDim.x) {
     const long long r = gid / groups_per_row, g = gid % groups_per_row;
     const long long seq = r / rows, row = r % rows;
+    if (t0 != nullptr) {
+      const int off = __ldg(t0 + seq);
+      if (row >= off) {
+        if (cu_seqlens != nullptr && Vc != nullptr) {
+          const long long n = (long long)__ldg(cu_seqlens + seq + 1) - __ldg(cu_seqlens + seq);
+          const long long e = (long long)off + n;
+          const long long tail = min((e + 127) / 128 * 128, (long long)rows);
+          if (off >= 0 && n >= 0 && e <= rows && row >= e && row < tail)
+            Vc[(seq * Tcap + row) * groups_per_row + g] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+    }
     uint4 w = __ldg(Kc + (seq * Tcap + row) * groups_per_row + g);
     uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
@@ -402,7 +446,7 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
     kern<<<blocks, kRopeThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Krot, B, L, Hq, Hkv, s, c, log2((double)base), 0, L,
-        nullptr, nullptr, nullptr, 0, cu_seqlens, n_seq);
+        nullptr, nullptr, nullptr, 0, cu_seqlens, n_seq, nullptr);
   };
   if (D == 64) args(prefill_rope_kernel<64, false>);
   else args(prefill_rope_kernel<128, false>);
@@ -412,7 +456,8 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
 cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
                               int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
-                              float base, cudaStream_t stream) {
+                              float base, cudaStream_t stream, const int* cu_seqlens,
+                              int n_seq, const int* t0s) {
   using namespace rope_path;
   const long long rows = (long long)B * Lq;
   if (rows == 0) return cudaSuccess;
@@ -422,7 +467,7 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Kcache, B, Lq, Hq, Hkv, s, c, log2((double)base), t0, Tcap,
         static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(Vcache),
-        static_cast<__half*>(Kf16), kh_rows, nullptr, 0);
+        static_cast<__half*>(Kf16), kh_rows, cu_seqlens, n_seq, t0s);
   };
   if (D == 64) args(prefill_rope_kernel<64, true>);
   else args(prefill_rope_kernel<128, true>);
@@ -449,7 +494,8 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, voi
 
 namespace dca {
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
-                               int out_rows, int Hkv, int D, cudaStream_t stream) {
+                               int out_rows, int Hkv, int D, cudaStream_t stream,
+                               const int* t0s, const int* cu_seqlens, void* Vcache) {
   using namespace rope_path;
   const long long gpr = (long long)Hkv * D / 8;
   const long long total = (long long)B * rows * gpr;
@@ -458,7 +504,8 @@ cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, 
   const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
   keys_to_f16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(Kcache),
                                                  static_cast<uint4*>(Kf16), rows, Tcap,
-                                                 out_rows, gpr, total);
+                                                 out_rows, gpr, total, t0s, cu_seqlens,
+                                                 static_cast<uint4*>(Vcache));
   return cudaGetLastError();
 }
 }  // namespace dca

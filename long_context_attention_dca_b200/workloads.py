@@ -135,6 +135,12 @@ def varlen_flops(lens, Hq: int, D: int) -> float:
     return sum(4.0 * D * Hq * n * (n + 1) / 2 for n in lens)
 
 
+def varlen_chunk_flops(t0, lens, Hq: int, D: int) -> float:
+    """Algorithmic FLOPs of packed chunks over caches: row r of sequence b
+    attends t0[b] + r + 1 keys."""
+    return sum(4.0 * D * Hq * (n * a + n * (n + 1) / 2) for a, n in zip(t0, lens))
+
+
 def decode_bytes(cfg: dict, t) -> float:
     """Algorithmic bytes of one decode step.
 

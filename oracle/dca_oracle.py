@@ -30,7 +30,9 @@ fusion or reordering:
 * Chunked prefill (dca_prefill_chunk): rows t0 .. t0+Lq-1 of the same
   definition with keys 0 .. t0-1 read, already rotated, from a cache.
 * Variable-length batch (dca_prefill_varlen_rows): sequences packed one after
-  another, each its own prefill (chunks from its first token, own keys only).
+  another, each its own prefill (chunks from its first token, own keys only);
+  with a cache per sequence (dca_prefill_varlen_chunk_rows) each packed
+  sequence is the chunked prefill of its own cache at its own offset.
 * SelfExtend (prior art; LLM Maybe LongLM: Self-Extend LLM Context Window
   Without Tuning, abstract): neighbour pairs (i - j < W) at positions (i, j),
   grouped pairs at (floor(i/G) + W - floor(W/G), floor(j/G)), one softmax.
@@ -335,6 +337,36 @@ def dca_prefill_varlen_rows(Q, K, V, cu_seqlens, s: int, c: int, base: float = 1
             continue
         res = dca_prefill_rows(Q[None, a:e], K[None, a:e], V[None, a:e], s, c, base, scale,
                                rows=local, heads=heads)
+        for (_, h, r), val in res.items():
+            out[(h, a + r)] = val
+    return out
+
+
+def dca_prefill_varlen_chunk_rows(Q, K, V, cu_seqlens, t0, k_cache_rot, v_cache, s: int,
+                                  c: int, base: float = 10000.0, scale: float = 0.0,
+                                  rows=None, heads=None):
+    """Packed chunks, one per sequence, each against that sequence's cache.
+
+    Q: [T, Hq, D]; K, V: [T, Hkv, D] (unrotated new tokens, packed as for
+    dca_prefill_varlen_rows).  Sequence b's packed row cu_seqlens[b] + r is
+    token t0[b] + r of sequence b, evaluated as in dca_prefill_chunk with
+    keys 0 .. t0[b]-1 taken, as stored, from k_cache_rot[b] (already rotated
+    at j mod s) and values from v_cache[b].  rows: packed indices (default
+    all).  Returns {(h, t): (O [D], LSE)} keyed by packed row.
+    """
+    cu = [int(x) for x in cu_seqlens]
+    want = None if rows is None else {int(r) for r in rows}
+    out = {}
+    for b in range(len(cu) - 1):
+        a, e, tb = cu[b], cu[b + 1], int(t0[b])
+        if e <= a:
+            continue
+        local = [t - a for t in range(a, e) if want is None or t in want]
+        if not local:
+            continue
+        res = dca_prefill_chunk(Q[None, a:e], K[None, a:e], V[None, a:e],
+                                k_cache_rot[b:b + 1], v_cache[b:b + 1], tb, s, c, base, scale,
+                                rows=local, heads=heads)
         for (_, h, r), val in res.items():
             out[(h, a + r)] = val
     return out

@@ -77,6 +77,11 @@ def test_workspace_queries(lib):
     assert dca.dca_attn_prefill_varlen_workspace(777, 8, 2, 128) == (
         up(3 * 777 * 8 * 128 * 2) + up(777 * 2 * 128 * 2))
     assert dca.dca_attn_prefill_varlen_workspace(777, 8, 3, 128) == 0
+    # packed chunks over caches: query rotations of the T rows + fp16 keys of
+    # max_kv rows per sequence
+    assert dca.dca_attn_prefill_varlen_chunk_workspace(3, 100, 300, 4, 2, 128) == (
+        up(3 * 100 * 4 * 128 * 2) + up(3 * 300 * 2 * 128 * 2))
+    assert dca.dca_attn_prefill_varlen_chunk_workspace(3, 100, -1, 4, 2, 128) == 0
 
 
 def test_prefill_path_selection(lib):
@@ -185,6 +190,18 @@ def test_argument_errors_return_codes(lib):
     # empty batches are no-ops even with null pointers
     assert _code(lib.dca_attn_prefill_varlen(None, None, None, None, None, None, 0, 64, 100, 4,
                                              2, 128, 16, 32, 1e4, 0.0, None, 0, None)) == 0
+    # packed chunks over caches: max_kv beyond the cache, null t0, short workspace
+    cargs7 = (fake,) * 7
+    assert _code(lib.dca_attn_prefill_varlen_chunk(*cargs7, fake, fake, 3, 64, 100, 500, 4, 2,
+                                                   128, 400, 16, 32, 1e4, 0.0, ws, 1 << 30,
+                                                   None)) == 1
+    assert "max_kv" in dca.dca_last_error_string()
+    assert _code(lib.dca_attn_prefill_varlen_chunk(*cargs7, fake, None, 3, 64, 100, 300, 4, 2,
+                                                   128, 400, 16, 32, 1e4, 0.0, ws, 1 << 30,
+                                                   None)) == 1
+    assert _code(lib.dca_attn_prefill_varlen_chunk(*cargs7, fake, fake, 3, 64, 100, 300, 4, 2,
+                                                   128, 400, 16, 32, 1e4, 0.0, ws, 64,
+                                                   None)) == 5
     # wait self-test: deadline out of range
     assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
     assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1

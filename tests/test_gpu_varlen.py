@@ -150,3 +150,157 @@ def test_varlen_bad_offsets_are_reported(bad):
                                np.log(np.arange(1, 101))[None, :].repeat(Hq, 0), atol=1e-5)
     assert (O[100:].float() == O_FILL).all() and (LSE[:, 100:] == LSE_FILL).all()
     dca.dca_sync_status()  # cleared; the context keeps working
+
+
+# ---------------------------------------------------------------------------
+# packed chunks over per-sequence caches (dca_attn_prefill_varlen_chunk)
+# ---------------------------------------------------------------------------
+
+def _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed):
+    """Packed new tokens and caches whose rows 0 .. t0[b]-1 hold random bf16
+    keys (standing for keys already rotated at j mod s: a rotation of i.i.d.
+    N(0, 1) pairs is again i.i.d. N(0, 1)) and values; every later cache row
+    holds NaN, so a row read or written by mistake shows."""
+    gen = torch.Generator().manual_seed(seed)
+    T, B = sum(lens), len(lens)
+    Q = torch.randn(T, Hq, D, generator=gen).to(torch.bfloat16)
+    K = torch.randn(T, Hkv, D, generator=gen).to(torch.bfloat16)
+    V = torch.randn(T, Hkv, D, generator=gen).to(torch.bfloat16)
+    Kc = torch.full((B, Tcap, Hkv, D), float("nan"), dtype=torch.bfloat16)
+    Vc = torch.full((B, Tcap, Hkv, D), float("nan"), dtype=torch.bfloat16)
+    for b in range(B):
+        Kc[b, :t0[b]] = torch.randn(t0[b], Hkv, D, generator=gen).to(torch.bfloat16)
+        Vc[b, :t0[b]] = torch.randn(t0[b], Hkv, D, generator=gen).to(torch.bfloat16)
+    cu = torch.zeros(B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens), 0).to(torch.int32)
+    return Q, K, V, Kc, Vc, cu
+
+
+def _run_chunk(Q, K, V, Kc, Vc, cu, t0, s, c, max_kv):
+    T, Hq, _ = Q.shape
+    O = torch.full(Q.shape, O_FILL, dtype=torch.bfloat16, device="cuda")
+    LSE = torch.full((Hq, T), LSE_FILL, dtype=torch.float32, device="cuda")
+    Kd, Vd = Kc.cuda(), Vc.cuda()
+    max_len = max(1, int((cu[1:] - cu[:-1]).max()))
+    dca.dca_attn_prefill_varlen_chunk(Q.cuda(), K.cuda(), V.cuda(), Kd, Vd, cu.cuda(),
+                                      torch.tensor(t0, dtype=torch.int32, device="cuda"),
+                                      max_len, max_kv, s, c, O=O, LSE=LSE)
+    return O, LSE, Kd, Vd
+
+
+VARLEN_CHUNK_CASES = [
+    # lens, t0, Hq, Hkv, D, s, c, Tcap
+    ([300, 1, 700, 0, 513], [0, 256, 77, 5, 1000], 4, 2, 128, 256, 400, 1600),
+    ([129, 400, 64], [511, 3, 0], 2, 1, 64, 192, 256, 700),
+    ([2000, 37], [300, 4000], 8, 1, 128, 512, 640, 4100),
+    ([90, 260], [1, 129], 2, 2, 128, 100, 150, 420),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_CHUNK_CASES, ids=str)
+def test_varlen_chunk_matches_oracle(case):
+    lens, t0, Hq, Hkv, D, s, c, Tcap = case
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed=61)
+    max_kv = max(a + n for a, n in zip(t0, lens))
+    O, LSE, Kd, Vd = _run_chunk(Q, K, V, Kc, Vc, cu, t0, s, c, max_kv)
+    dca.dca_sync_status()
+    O, LSE, Kg, Vg = O.cpu(), LSE.cpu(), Kd.cpu(), Vd.cpu()
+    assert torch.isfinite(O.float()).all() and torch.isfinite(LSE).all()
+    ref = orc.dca_prefill_varlen_chunk_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V),
+                                            cu.tolist(), t0, pu.F64View(Kc), pu.F64View(Vc),
+                                            s, c)
+    assert len(ref) == Hq * sum(lens)
+    _compare(O, LSE, ref, f"varlen chunk {case}")
+    for b, (a, n) in enumerate(zip(t0, lens)):
+        r0 = int(cu[b])
+        # cached rows unchanged, new rows written, the tail zeroed, the rest as it was
+        assert torch.equal(Kg[b, :a], Kc[b, :a]) and torch.equal(Vg[b, :a], Vc[b, :a])
+        assert torch.equal(Vg[b, a:a + n], V[r0:r0 + n])
+        ref_k = orc.rotate(K[r0:r0 + n].double().numpy().transpose(1, 0, 2),
+                           orc.key_position(a + np.arange(n), s), 10000.0).transpose(1, 0, 2)
+        err = np.abs(Kg[b, a:a + n].double().numpy() - ref_k)
+        assert (err <= np.abs(ref_k) * 2.0 ** -8 + 1e-5).all(), (case, b)
+        tail = min((a + n + 127) // 128 * 128, max_kv)
+        assert (Vg[b, a + n:tail].float() == 0).all()
+        assert torch.isnan(Vg[b, max(tail, a + n):].float()).all()
+        assert torch.isnan(Kg[b, a + n:].float()).all()
+
+
+def test_varlen_chunk_continues_a_packed_prefill():
+    # two calls (first chunks at t0 = 0, then the rest) give what one packed
+    # prefill of the whole sequences gives, up to the bf16 rounding of the
+    # cached keys (the second call reads them as stored)
+    Hq, Hkv, D, s, c = 4, 2, 128, 256, 384
+    first, rest = [300, 513, 64], [400, 1, 700]
+    full = [a + b for a, b in zip(first, rest)]
+    cfg = dict(Hq=Hq, Hkv=Hkv, D=D)
+    Q, K, V, cu_full, _ = W.make_varlen_inputs(cfg, seed=62, lens=full)
+    Tcap = max(full) + 100
+    pick = lambda X, lo, hi: torch.cat([X[int(cu_full[b]) + lo[b]:int(cu_full[b]) + hi[b]]
+                                        for b in range(3)])
+    zeros = [0, 0, 0]
+    Kd = torch.zeros(3, Tcap, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    Vd = torch.zeros_like(Kd)
+    outs = []
+    for lo, hi in ((zeros, first), (first, full)):
+        n = [h - l for l, h in zip(lo, hi)]
+        cu = torch.zeros(4, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(n), 0).to(torch.int32)
+        O, LSE = dca.dca_attn_prefill_varlen_chunk(
+            pick(Q, lo, hi).cuda(), pick(K, lo, hi).cuda(), pick(V, lo, hi).cuda(), Kd, Vd,
+            cu.cuda(), torch.tensor(lo, dtype=torch.int32, device="cuda"), max(n), Tcap, s, c)
+        outs.append((O.cpu(), LSE.cpu(), cu))
+    dca.dca_sync_status()
+    Of, Lf = dca.dca_attn_prefill_varlen(Q.cuda(), K.cuda(), V.cuda(), cu_full.cuda(), max(full),
+                                         s, c)
+    Of, Lf = Of.cpu(), Lf.cpu()
+    for b in range(3):
+        a = int(cu_full[b])
+        for (O, LSE, cu), lo in zip(outs, (zeros, first)):
+            r0, n = int(cu[b]), int(cu[b + 1] - cu[b])
+            d_o = (O[r0:r0 + n].float() - Of[a + lo[b]:a + lo[b] + n].float()).abs().max()
+            d_l = (LSE[:, r0:r0 + n] - Lf[:, a + lo[b]:a + lo[b] + n]).abs().max()
+            assert d_o <= 2e-2 and d_l <= 3e-3, (b, lo, float(d_o), float(d_l))
+
+
+def test_varlen_chunk_workload_sampled():
+    # Llama-2 7B heads: eight sequences with 0 .. 14000 cached tokens and new
+    # chunks of 256 .. 2048 tokens, packed
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, D, s, c = 8, 32, 32, 128, 3072, 4096
+    t0 = [int(x) for x in rng.integers(0, 14001, B)]
+    lens = [int(x) for x in rng.integers(256, 2049, B)]
+    Tcap = 16384
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed=63)
+    max_kv = max(a + n for a, n in zip(t0, lens))
+    O, LSE, _, _ = _run_chunk(Q, K, V, Kc, Vc, cu, t0, s, c, max_kv)
+    dca.dca_sync_status()
+    O, LSE = O.cpu(), LSE.cpu()
+    heads = pu.sample_heads(Hq, Hkv)
+    for b in (0, 3, 7):
+        a = int(cu[b])
+        rows = [a + r for r in pu.sample_rows(lens[b], s, c, n_random=16, seed=b)]
+        ref = orc.dca_prefill_varlen_chunk_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V),
+                                                cu.tolist(), t0, pu.F64View(Kc),
+                                                pu.F64View(Vc), s, c, rows=rows, heads=heads)
+        _compare(O, LSE, ref, f"varlen chunk 7B sequence {b} (t0={t0[b]}, n={lens[b]})")
+
+
+@pytest.mark.parametrize("bad", ["past_max_kv", "negative_t0"])
+def test_varlen_chunk_bad_offsets_are_reported(bad):
+    Hq, Hkv, D, s, c, Tcap = 2, 1, 128, 256, 384, 600
+    lens, t0 = [100, 200], {"past_max_kv": [0, 450], "negative_t0": [0, -3]}[bad]
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, [max(a, 0) for a in t0], Hq, Hkv, D, Tcap, seed=64)
+    O, LSE, Kd, Vd = _run_chunk(Q, K, V, Kc, Vc, cu, t0, s, c, max_kv=600 if bad == "negative_t0"
+                                else 500)
+    with pytest.raises(dca.DcaError) as ei:
+        dca.dca_sync_status()
+    assert ei.value.status == 1
+    O, LSE, Kg, Vg = O.cpu(), LSE.cpu(), Kd.cpu(), Vd.cpu()
+    # sequence 0 computed and cached; sequence 1 neither computed nor cached
+    assert torch.isfinite(O[:100].float()).all()
+    assert (O[100:].float() == O_FILL).all() and (LSE[:, 100:] == LSE_FILL).all()
+    assert torch.equal(Vg[0, :100], V[:100])
+    assert torch.equal(Kg[1].view(torch.int16), Kc[1].view(torch.int16))
+    assert torch.equal(Vg[1].view(torch.int16), Vc[1].view(torch.int16))
+    dca.dca_sync_status()

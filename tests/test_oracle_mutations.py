@@ -8,7 +8,8 @@ causal off-by-one, a wrong GQA mapping, a shifted chunk origin, a broken
 partial merge, a decode that reads one key too few, a chunked prefill
 that ignores or misaligns its cache, or a packed variable-length batch that
 leaks across sequences, counts positions from the packed start or reports
-local rows.  The pins of
+local rows, and packed chunks that ignore their cache offsets or read
+another sequence's cache.  The pins of
 ``test_oracle_pins`` must reject each one.
 """
 
@@ -199,6 +200,22 @@ def _varlen_local_keys(*args, **kw):
             for (h, t), v in _ORIG_VARLEN(*args, **kw).items()}
 
 
+_ORIG_VARLEN_CHUNK = orc.dca_prefill_varlen_chunk_rows
+
+
+def _varlen_chunk_no_offset(Q, K, V, cu_seqlens, t0, k_cache_rot, v_cache, *args, **kw):
+    # every sequence's chunk taken as its first tokens (cache offsets ignored)
+    return _ORIG_VARLEN_CHUNK(Q, K, V, cu_seqlens, [0] * len(t0), k_cache_rot, v_cache, *args,
+                              **kw)
+
+
+def _varlen_chunk_first_cache(Q, K, V, cu_seqlens, t0, k_cache_rot, v_cache, *args, **kw):
+    # every sequence reads batch entry 0 of the caches
+    B = len(t0)
+    return _ORIG_VARLEN_CHUNK(Q, K, V, cu_seqlens, t0, np.repeat(k_cache_rot[:1], B, axis=0),
+                              np.repeat(v_cache[:1], B, axis=0), *args, **kw)
+
+
 MUTANTS = {
     "succ_rule_le": ("query_position", _qpos_succ_le),
     "succ_far_pos_c": ("query_position", _qpos_succ_c),
@@ -223,6 +240,8 @@ MUTANTS = {
     "varlen_whole_pack": ("dca_prefill_varlen_rows", _varlen_whole_pack),
     "varlen_global_positions": ("dca_prefill_varlen_rows", _varlen_global_positions),
     "varlen_local_keys": ("dca_prefill_varlen_rows", _varlen_local_keys),
+    "varlen_chunk_no_offset": ("dca_prefill_varlen_chunk_rows", _varlen_chunk_no_offset),
+    "varlen_chunk_first_cache": ("dca_prefill_varlen_chunk_rows", _varlen_chunk_first_cache),
 }
 
 

@@ -305,6 +305,50 @@ def pin_varlen_q_zero_closed_form():
                 np.testing.assert_allclose(o, V[cu[b]:t + 1, h // 2].mean(0), atol=1e-13)
 
 
+def pin_varlen_chunk_equals_whole_sequences():
+    # next chunks of three sequences at offsets 7, 0 and 12, packed: each
+    # packed row equals row t0[b] + r of sequence b's whole-sequence prefill,
+    # with the cached keys rotated by the independent complex-number RoPE
+    s, c = 5, 8
+    t0, n = [7, 0, 12], [6, 4, 9]
+    B, Lmax = 3, max(a + m for a, m in zip(t0, n))
+    Q, K, V = _rand((B, Lmax, 2, 8), 48), _rand((B, Lmax, 1, 8), 49), _rand((B, Lmax, 1, 8), 50)
+    k_rot = _complex_rotate(K, (np.arange(Lmax) % s)[None, :, None], 10000.0)
+    cu = [0]
+    for m in n:
+        cu.append(cu[-1] + m)
+    pack = lambda X: np.concatenate([X[b, t0[b]:t0[b] + n[b]] for b in range(B)])
+    got = orc.dca_prefill_varlen_chunk_rows(pack(Q), pack(K), pack(V), cu, t0, k_rot, V, s, c)
+    assert set(got) == {(h, t) for h in range(2) for t in range(cu[-1])}
+    for b in range(B):
+        full = orc.dca_prefill_rows(Q[b:b + 1, :t0[b] + n[b]], K[b:b + 1, :t0[b] + n[b]],
+                                    V[b:b + 1, :t0[b] + n[b]], s, c)
+        for r in range(n[b]):
+            for h in range(2):
+                o, lse = got[(h, cu[b] + r)]
+                np.testing.assert_allclose(o, full[(0, h, t0[b] + r)][0], atol=1e-12)
+                np.testing.assert_allclose(lse, full[(0, h, t0[b] + r)][1], atol=1e-12)
+
+
+def pin_varlen_chunk_q_zero_closed_form():
+    # Q = 0: LSE = ln(t0[b] + r + 1), O = mean of the cached values and the new
+    # values up to the row
+    t0, n = [3, 0, 10], [5, 2, 4]
+    cu = [0, 5, 7, 11]
+    Kc, Vc = _rand((3, 16, 2, 8), 51), _rand((3, 16, 2, 8), 52)
+    K, V = _rand((11, 2, 8), 53), _rand((11, 2, 8), 54)
+    Q = np.zeros((11, 4, 8))
+    got = orc.dca_prefill_varlen_chunk_rows(Q, K, V, cu, t0, Kc, Vc, s=4, c=6)
+    for b in range(3):
+        for r in range(n[b]):
+            t = cu[b] + r
+            for h in range(4):
+                o, lse = got[(h, t)]
+                vals = np.concatenate([Vc[b, :t0[b], h // 2], V[cu[b]:t + 1, h // 2]])
+                np.testing.assert_allclose(lse, math.log(t0[b] + r + 1), atol=1e-13)
+                np.testing.assert_allclose(o, vals.mean(0), atol=1e-13)
+
+
 def pin_merge_partials():
     z, v = _rand(50, 27) * 3, _rand((50, 8), 28)
     o_full, lse_full = orc.softmax_row(z, v)
@@ -386,7 +430,9 @@ PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
         pin_q_zero_closed_form, pin_constant_v, pin_gqa_mapping,
         pin_decode_equals_prefill_row, pin_chunk_equals_prefill_rows,
-        pin_varlen_equals_padded_batch, pin_varlen_q_zero_closed_form, pin_merge_partials,
+        pin_varlen_equals_padded_batch, pin_varlen_q_zero_closed_form,
+        pin_varlen_chunk_equals_whole_sequences, pin_varlen_chunk_q_zero_closed_form,
+        pin_merge_partials,
         pin_rule_positions, pin_selfextend_worked_tables, pin_selfextend_reduces_to_plain_rope,
         pin_selfextend_distance_bounds]
 
