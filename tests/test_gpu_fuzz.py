@@ -100,3 +100,45 @@ def test_random_shape_varlen_equals_per_sequence(k):
         dca.dca_sync_status()
         assert torch.equal(O[a:a + n], Ob[0].cpu()), (cs, lens, b)
         assert torch.equal(LSE[:, a:a + n], Lb[0].cpu()), (cs, lens, b)
+
+
+@pytest.mark.parametrize("k", range(N_CASES // 2))
+def test_random_shape_varlen_chunk_matches_oracle(k):
+    # the same shapes as packed chunks over caches: random cached lengths and
+    # chunk lengths (some empty), random cache contents standing for rotated
+    # keys; every row against the oracle
+    cs = _case(k)
+    rng = np.random.default_rng(4000 + k)
+    B = int(rng.integers(1, 5))
+    t0 = [int(rng.integers(0, 600)) for _ in range(B)]
+    lens = [int(rng.integers(0, 300)) for _ in range(B)]
+    lens[-1] = max(lens[-1], 1)
+    Hq, Hkv, D, s, c = cs["Hq"], cs["Hkv"], cs["D"], cs["s"], cs["c"]
+    gen = torch.Generator().manual_seed(5000 + k)
+    T = sum(lens)
+    Tcap = max(a + n for a, n in zip(t0, lens)) + int(rng.integers(0, 200))
+    Q = torch.randn(T, Hq, D, generator=gen).to(torch.bfloat16)
+    K = torch.randn(T, Hkv, D, generator=gen).to(torch.bfloat16)
+    V = torch.randn(T, Hkv, D, generator=gen).to(torch.bfloat16)
+    Kc = torch.randn(B, Tcap, Hkv, D, generator=gen).to(torch.bfloat16)
+    Vc = torch.randn(B, Tcap, Hkv, D, generator=gen).to(torch.bfloat16)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    max_kv = max(a + n for a, n in zip(t0, lens))
+    O, LSE = dca.dca_attn_prefill_varlen_chunk(
+        Q.cuda(), K.cuda(), V.cuda(), Kc.cuda(), Vc.cuda(), cu.cuda(),
+        torch.tensor(t0, dtype=torch.int32, device="cuda"), max(lens), max_kv, s, c)
+    dca.dca_sync_status()
+    O, LSE = O.cpu(), LSE.cpu()
+    ref = orc.dca_prefill_varlen_chunk_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V),
+                                            cu.tolist(), t0, pu.F64View(Kc), pu.F64View(Vc),
+                                            s, c)
+    keys = sorted(ref)
+    o_ref = np.stack([ref[key][0] for key in keys])
+    l_ref = np.array([ref[key][1] for key in keys])
+    o_got = np.stack([O[t, h].double().numpy() for h, t in keys])
+    l_got = np.array([float(LSE[h, t]) for h, t in keys])
+    err = np.abs(o_got - o_ref)
+    lse = float(np.max(np.abs(l_got - l_ref) / np.maximum(np.abs(l_ref), 1.0)))
+    print(f"{cs} t0={t0} lens={lens}: O max {err.max():.3e} mean {err.mean():.3e} "
+          f"LSE rel {lse:.3e}")
+    pu.assert_close(float(err.max()), float(err.mean()), lse, f"{cs} t0={t0} lens={lens}")
