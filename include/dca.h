@@ -254,6 +254,30 @@ dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const v
                                            float scale, void* workspace, size_t ws_bytes,
                                            void* stream);
 
+/* dca_attn_prefill_varlen_chunk over paged caches: Kpool, Vpool
+ * [num_blocks][block_rows][Hkv][D] bf16; position p of sequence b lives in
+ * row p % block_rows of block block_table[b][p / block_rows] (block_table
+ * DEVICE int32 [B][max_blocks]; Tcap = max_blocks * block_rows bounds max_kv).
+ * block_rows must be a multiple of 128 so that a 128-key tile never crosses a
+ * block; blocks may sit anywhere in the pool, in any order.  Same inputs,
+ * outputs, cache rows written and workspace
+ * (dca_attn_prefill_varlen_chunk_workspace) as the contiguous call, whose
+ * results it reproduces bit for bit; the value rows zeroed after each
+ * sequence's new end run to the 128-row tile edge (inside the same block)
+ * even past max_kv, since the pool is read by whole tiles.  The attention reads values straight
+ * from the pool (each tile's block looked up once by the copying thread); a
+ * table entry outside [0, num_blocks) is reported as DCA_ERR_INVALID_ARG at
+ * the next dca_sync_status, nothing is written through it, and the affected
+ * sequence's outputs are undefined.
+ * Errors: INVALID_ARG, UNSUPPORTED (block_rows not a multiple of 128, D),
+ * WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_varlen_chunk_paged(
+    const void* Q, const void* K, const void* V, void* Kpool, void* Vpool,
+    const int* block_table, int max_blocks, int block_rows, int num_blocks, void* O, float* LSE,
+    const int* cu_seqlens, const int* t0, int B, int max_seqlen, int T, int max_kv, int Hq,
+    int Hkv, int D, int s, int c, float base, float scale, void* workspace, size_t ws_bytes,
+    void* stream);
+
 /* Workspace bytes for dca_attn_prefill_selfextend: the neighbour and grouped
  * rotations of Q [2][B][L][Hq][D] and K [2][B][L][Hkv][D], fp16, each rounded
  * up to 256 bytes.  Returns 0 for unsupported arguments. */

@@ -27,6 +27,7 @@ __all__ = [
     "dca_attn_prefill_chunk_workspace", "dca_attn_prefill_chunk",
     "dca_attn_prefill_varlen_workspace", "dca_attn_prefill_varlen",
     "dca_attn_prefill_varlen_chunk_workspace", "dca_attn_prefill_varlen_chunk",
+    "dca_attn_prefill_varlen_chunk_paged",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
     "dca_attn_decode_paged", "dca_kv_append_paged",
@@ -57,6 +58,9 @@ _SIGS = {
     "dca_attn_prefill_varlen_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "dca_attn_prefill_varlen_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
                                            _I, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
+    "dca_attn_prefill_varlen_chunk_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P,
+                                                 _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F,
+                                                 _P, _Z, _P]),
     "dca_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                      _F, _P, _Z, _P]),
     "dca_attn_prefill_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
@@ -283,6 +287,38 @@ def dca_attn_prefill_varlen_chunk(Q, K, V, Kcache, Vcache, cu_seqlens, t0, max_s
         _ptr(Q), _ptr(K), _ptr(V), _ptr(Kcache), _ptr(Vcache), _ptr(O), _ptr(LSE),
         _ptr(cu_seqlens), _ptr(t0), B, int(max_seqlen), T, int(max_kv), Hq, Hkv, D, Tcap, s, c,
         base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
+
+
+def dca_attn_prefill_varlen_chunk_paged(Q, K, V, Kpool, Vpool, block_table, cu_seqlens, t0,
+                                        max_seqlen, max_kv, s, c, base=10000.0, scale=0.0,
+                                        workspace=None, O=None, LSE=None):
+    """dca_attn_prefill_varlen_chunk over paged pools Kpool, Vpool
+    [num_blocks, block_rows, Hkv, D] bf16 and block_table int32 [B, max_blocks]
+    on the device (block_rows a multiple of 128)."""
+    _need(Q, "Q", torch.bfloat16, 3)
+    _need(K, "K", torch.bfloat16, 3)
+    _need(V, "V", torch.bfloat16, 3)
+    _need(Kpool, "Kpool", torch.bfloat16, 4)
+    _need(Vpool, "Vpool", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    _need(t0, "t0", torch.int32, 1)
+    T, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    num_blocks, block_rows = Kpool.shape[:2]
+    B, max_blocks = block_table.shape
+    nbytes = dca_attn_prefill_varlen_chunk_workspace(B, T, int(max_kv), Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    O = torch.empty_like(Q) if O is None else O
+    LSE = torch.empty((Hq, T), dtype=torch.float32, device=Q.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 3)
+    _need(LSE, "LSE", torch.float32, 2)
+    _check(lib().dca_attn_prefill_varlen_chunk_paged(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(Kpool), _ptr(Vpool), _ptr(block_table), max_blocks,
+        block_rows, num_blocks, _ptr(O), _ptr(LSE), _ptr(cu_seqlens), _ptr(t0), B,
+        int(max_seqlen), T, int(max_kv), Hq, Hkv, D, s, c, base, scale, _ptr(ws), ws.numel(),
+        _stream(Q)))
     return O, LSE
 
 

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
     int q_off, int group_units, const int* __restrict__ cu_seqlens, int T,
-    const int* __restrict__ t0s, int kv_rows) {
+    const int* __restrict__ t0s, int kv_rows, CacheMap vmap) {
   using LD = Lay<D>;
   constexpr int kHalves = LD::kHalves, kTileBytes = LD::kTileBytes;
   constexpr int kSmQ = LD::kSmQ, kSmK = LD::kSmK, kSmV = LD::kSmV, kSmBar = LD::kSmBar;
@@ -319,10 +319,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
             break;
           mbar_arrive_expect_tx(bar(kVFull + sg), kTileBytes);
           const uint32_t vd = sbase + kSmV + sg * kTileBytes;
+          int vrow = sq.krow0 + t * kTile, vbt = sq.kbt;
+          if constexpr (kSeqOff) {
+            if (vmap.table != nullptr) {  // paged values: the tile lies in one block
+              const long long pr = cache_row(vmap, vbt, vrow);
+              if (pr < 0) {  // reported; the coordinate past the pool reads zeros
+                report_error(kDevBadArg, 313);
+                vrow = 0;
+                vbt = vmap.num_blocks;
+              } else {
+                vrow = (int)(pr % vmap.block_rows);
+                vbt = (int)(pr / vmap.block_rows);
+              }
+            }
+          }
 #pragma unroll
           for (int hf = 0; hf < kHalves; ++hf)
-            tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk,
-                        sq.krow0 + t * kTile, sq.kbt);
+            tma_load_4d(vd + hf * kBox, &tmV, bar(kVFull + sg), hf * 64, hk, vrow, vbt);
           v_last[sg] = st;
         }
       }
@@ -545,10 +558,14 @@ template <int D, class Rule>
 cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void* O, float* LSE,
                          int B, int L, int Hq, int Hkv, Rule rule, int nq, float scale,
                          cudaStream_t stream, int q_off, int k_rows, int v_rows,
-                         const int* cu_seqlens, int T, const int* t0s, int kv_rows) {
+                         const int* cu_seqlens, int T, const int* t0s, int kv_rows,
+                         CacheMap vmap) {
   if (q_off < 0) return cudaErrorInvalidValue;
   if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
   if (t0s != nullptr && (cu_seqlens == nullptr || kv_rows < 1)) return cudaErrorInvalidValue;
+  const bool paged = vmap.table != nullptr;
+  if (paged && (t0s == nullptr || vmap.block_rows % kTile != 0 || vmap.num_blocks < 1))
+    return cudaErrorInvalidValue;
   if (L == 0 || B == 0) return cudaSuccess;
   const int Bm = cu_seqlens ? 1 : B;       // query tensor batch extent
   const int Bk = cu_seqlens && !t0s ? 1 : B;  // key / value tensor batch extent
@@ -569,7 +586,10 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
   {
     const uint64_t kdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv,
                                (uint64_t)Rule::kKPlanes * Bk};
-    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)Lkv, (uint64_t)Bk};
+    // paged values: the map spans the pool, rows within a block
+    const uint64_t vdims[4] = {(uint64_t)D, (uint64_t)Hkv,
+                               paged ? (uint64_t)vmap.block_rows : (uint64_t)Lkv,
+                               paged ? (uint64_t)vmap.num_blocks : (uint64_t)Bk};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
     const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
@@ -591,7 +611,7 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
                                                LSE, B, L, Hq, Hkv, rule,
                                                scale * 1.4426950408889634f, q_off,
                                                B * Hkv,  // one group: longest first
-                                               cu_seqlens, T, t0s, Lkv);
+                                               cu_seqlens, T, t0s, Lkv, vmap);
     return cudaGetLastError();
   };
   if (t0s == nullptr) return run(prefill_attn_gen_kernel<D, Rule, false>);
@@ -604,13 +624,13 @@ cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* 
                        int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
                        cudaStream_t stream, int q_off, int k_rows, int v_rows,
                        const int* cu_seqlens = nullptr, int T = 0, const int* t0s = nullptr,
-                       int kv_rows = 0) {
+                       int kv_rows = 0, CacheMap vmap = CacheMap{nullptr, 0, 0, 0, 0}) {
   if (D == 64)
     return launch_gen_d<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream, q_off,
-                            k_rows, v_rows, cu_seqlens, T, t0s, kv_rows);
+                            k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap);
   if (D == 128)
     return launch_gen_d<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream,
-                             q_off, k_rows, v_rows, cu_seqlens, T, t0s, kv_rows);
+                             q_off, k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap);
   return cudaErrorInvalidValue;
 }
 
@@ -624,11 +644,13 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off, int k_rows, int v_rows,
                                           const int* cu_seqlens, int T, const int* t0s,
-                                          int kv_rows) {
+                                          int kv_rows, const int* block_table, int max_blocks,
+                                          int block_rows, int num_blocks) {
   if (s < 1) return cudaErrorInvalidValue;
   return gen_path::launch_gen(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, D,
                               gen_path::DcaIntervals{s}, 3, scale, stream, q_off, k_rows,
-                              v_rows, cu_seqlens, T, t0s, kv_rows);
+                              v_rows, cu_seqlens, T, t0s, kv_rows,
+                              CacheMap{block_table, max_blocks, block_rows, num_blocks, 0});
 }
 
 // SelfExtend on the same kernel: Qse, Kse [2][B][L][H][D] fp16 (neighbour,

@@ -367,14 +367,18 @@ size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq,
   return align256((size_t)3 * T * Hq * D * 2) + align256((size_t)B * max_kv * Hkv * D * 2);
 }
 
-dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const void* V,
-                                           void* Kcache, void* Vcache, void* O, float* LSE,
-                                           const int* cu_seqlens, const int* t0, int B,
-                                           int max_seqlen, int T, int max_kv, int Hq, int Hkv,
-                                           int D, int Tcap, int s, int c, float base,
-                                           float scale, void* workspace, size_t ws_bytes,
-                                           void* stream) {
-  const char* fn = "dca_attn_prefill_varlen_chunk";
+}  // extern "C"
+
+namespace {
+
+// Shared body of the contiguous and paged packed-chunk entry points.
+dca_status_t varlen_chunk_impl(const char* fn, const void* Q, const void* K, const void* V,
+                               void* Kcache, void* Vcache, void* O, float* LSE,
+                               const int* cu_seqlens, const int* t0, int B, int max_seqlen,
+                               int T, int max_kv, int Hq, int Hkv, int D, int Tcap, int s, int c,
+                               float base, float scale, void* workspace, size_t ws_bytes,
+                               void* stream, const int* block_table, int max_blocks,
+                               int block_rows, int num_blocks) {
   dca_status_t st = check_heads(fn, B, max_seqlen, Hq, Hkv, D);
   if (st == DCA_OK) st = check_chunking(fn, s, c, base);
   if (st != DCA_OK) return st;
@@ -405,14 +409,54 @@ dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const v
   // converted to fp16 as stored.
   void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * T * Hq * D * 2);
   cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, 1, T, Hq, Hkv, D,
-                                    0, Tcap, max_kv, s, c, base, strm, cu_seqlens, B, t0);
+                                    0, Tcap, max_kv, s, c, base, strm, cu_seqlens, B, t0,
+                                    block_table, max_blocks, block_rows, num_blocks);
   if (e == cudaSuccess)
     e = launch_keys_to_f16(Kcache, kf16, B, max_kv, Tcap, max_kv, Hkv, D, strm, t0, cu_seqlens,
-                           Vcache);
+                           Vcache, block_table, max_blocks, block_rows, num_blocks);
   if (e == cudaSuccess)
     e = launch_prefill_attn_sm100_gen(workspace, kf16, Vcache, O, LSE, B, max_seqlen, Hq, Hkv, D,
-                                      s, sc, strm, 0, max_kv, Tcap, cu_seqlens, T, t0, max_kv);
+                                      s, sc, strm, 0, max_kv, Tcap, cu_seqlens, T, t0, max_kv,
+                                      block_table, max_blocks, block_rows, num_blocks);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
+}  // namespace
+
+extern "C" {
+
+dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const void* V,
+                                           void* Kcache, void* Vcache, void* O, float* LSE,
+                                           const int* cu_seqlens, const int* t0, int B,
+                                           int max_seqlen, int T, int max_kv, int Hq, int Hkv,
+                                           int D, int Tcap, int s, int c, float base,
+                                           float scale, void* workspace, size_t ws_bytes,
+                                           void* stream) {
+  return varlen_chunk_impl("dca_attn_prefill_varlen_chunk", Q, K, V, Kcache, Vcache, O, LSE,
+                           cu_seqlens, t0, B, max_seqlen, T, max_kv, Hq, Hkv, D, Tcap, s, c,
+                           base, scale, workspace, ws_bytes, stream, nullptr, 0, 0, 0);
+}
+
+dca_status_t dca_attn_prefill_varlen_chunk_paged(
+    const void* Q, const void* K, const void* V, void* Kpool, void* Vpool,
+    const int* block_table, int max_blocks, int block_rows, int num_blocks, void* O, float* LSE,
+    const int* cu_seqlens, const int* t0, int B, int max_seqlen, int T, int max_kv, int Hq,
+    int Hkv, int D, int s, int c, float base, float scale, void* workspace, size_t ws_bytes,
+    void* stream) {
+  const char* fn = "dca_attn_prefill_varlen_chunk_paged";
+  if (max_blocks < 1 || num_blocks < 1 || block_rows < 1)
+    return fail(DCA_ERR_INVALID_ARG, "%s: need max_blocks, num_blocks, block_rows >= 1", fn);
+  if (block_rows % 128)
+    return fail(DCA_ERR_UNSUPPORTED, "%s: block_rows=%d (need a multiple of 128)", fn,
+                block_rows);
+  if ((long long)max_blocks * block_rows > 2147483647LL)
+    return fail(DCA_ERR_INVALID_ARG, "%s: max_blocks * block_rows overflows int32", fn);
+  if (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return fail(DCA_ERR_INVALID_ARG, "%s: block_table null or not 4-byte aligned", fn);
+  return varlen_chunk_impl(fn, Q, K, V, Kpool, Vpool, O, LSE, cu_seqlens, t0, B, max_seqlen, T,
+                           max_kv, Hq, Hkv, D, max_blocks * block_rows, s, c, base, scale,
+                           workspace, ws_bytes, stream, block_table, max_blocks, block_rows,
+                           num_blocks);
 }
 
 size_t dca_selfextend_workspace(int B, int L, int Hq, int Hkv, int D) {

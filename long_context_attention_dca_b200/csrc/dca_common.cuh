@@ -146,6 +146,23 @@ __device__ __forceinline__ bool seq_span(const int* cu_seqlens, const int* t0, i
   return ok && off >= 0 && (long long)off + (e - a) <= kv_rows;
 }
 
+// A key / value cache addressed by (sequence, position): contiguous
+// [B][Tcap][H][D] when `table` is null, else paged pools
+// [num_blocks][block_rows][H][D] with the block of position p of sequence b
+// at table[b * max_blocks + p / block_rows].
+struct CacheMap {
+  const int* table;
+  int max_blocks, block_rows, num_blocks, Tcap;
+};
+// Row index into the cache (times H*D elements), or -1 for a table entry
+// outside the pool.
+__device__ __forceinline__ long long cache_row(const CacheMap& m, int b, int pos) {
+  if (m.table == nullptr) return (long long)b * m.Tcap + pos;
+  const int blk = __ldg(m.table + (size_t)b * m.max_blocks + pos / m.block_rows);
+  if (blk < 0 || blk >= m.num_blocks) return -1;
+  return (long long)blk * m.block_rows + pos % m.block_rows;
+}
+
 // Dispatch order of the two-tile prefill kernels' (query-tile pair, head,
 // sequence) work items, from a 1-D block index: the (sequence, kv head) units
 // are taken in groups of `k`, one group after another; within a group the

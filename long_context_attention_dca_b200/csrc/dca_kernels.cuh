@@ -28,14 +28,17 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
 // Kcache is null) and in fp16 to rows t0 + r of Kf16 (kh_rows rows per
 // sequence); values to cache rows t0 + r (skipped when Vcache is null).
 // Packed form (cu_seqlens device [n_seq+1], B = 1, Lq = T, t0 = 0): row r of
-// sequence b is absolute index t0s[b] + r and writes cache rows of entry b;
+// sequence b is absolute index t0s[b] + r and writes sequence b's cache rows;
 // rows outside every sequence, or of a sequence that would leave the caches,
-// write no cache row.
+// write no cache row.  With block_table the caches are paged pools
+// [num_blocks][block_rows][Hkv][D] (Tcap = max_blocks * block_rows).
 cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void* Qrot,
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
                               int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
                               float base, cudaStream_t stream, const int* cu_seqlens = nullptr,
-                              int n_seq = 0, const int* t0s = nullptr);
+                              int n_seq = 0, const int* t0s = nullptr,
+                              const int* block_table = nullptr, int max_blocks = 0,
+                              int block_rows = 0, int num_blocks = 0);
 // Attention of that chunk over keys 0 .. t0+Lq-1 of Kf16 (k_rows rows per
 // sequence) and V (v_rows rows per sequence) (general path).
 cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, const void* V,
@@ -80,13 +83,16 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
 // packed chunks over caches: with cu_seqlens and t0s (device [B]) sequence
 // b's packed query rows sit at absolute indices t0s[b] + r and attend rows
 // 0 .. t0s[b]+r of batch entry b of Krot [B][k_rows pitch] and V [B][v_rows
-// pitch], kv_rows rows valid per entry.
+// pitch], kv_rows rows valid per entry; with block_table the values come
+// from a paged pool [num_blocks][block_rows][Hkv][D] (block_rows % 128 == 0).
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
                                           int q_off = 0, int k_rows = 0, int v_rows = 0,
                                           const int* cu_seqlens = nullptr, int T = 0,
-                                          const int* t0s = nullptr, int kv_rows = 0);
+                                          const int* t0s = nullptr, int kv_rows = 0,
+                                          const int* block_table = nullptr, int max_blocks = 0,
+                                          int block_rows = 0, int num_blocks = 0);
 // SelfExtend on the per-row-interval tcgen05 kernel (D = 64 or 128).
 cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
                                                  const void* V, void* O, float* LSE, int B,
@@ -96,10 +102,12 @@ cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Ks
 // fp16 [B][out_rows][Hkv][D]; with t0s (device [B]) only rows below t0s[b],
 // and with cu_seqlens and Vcache too the value-cache rows from each
 // sequence's new end to the next multiple of 128 (at most rows) are zeroed.
+// With block_table the caches are paged pools as for launch_chunk_rope.
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
                                int out_rows, int Hkv, int D, cudaStream_t stream,
                                const int* t0s = nullptr, const int* cu_seqlens = nullptr,
-                               void* Vcache = nullptr);
+                               void* Vcache = nullptr, const int* block_table = nullptr,
+                               int max_blocks = 0, int block_rows = 0, int num_blocks = 0);
 
 // Decode-time append of one token per sequence into pre-rotated caches:
 // contiguous [B][Tcap][Hkv][D] (block_table null) or a paged pool

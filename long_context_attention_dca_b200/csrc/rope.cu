@@ -131,22 +131,25 @@ constexpr int kRopeThreads = 256;
 // holds n_seq sequences, sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1;
 // a row's index is counted from its sequence's first row, plus t0[b] in the
 // chunk form (t0 device [n_seq], the rows sequence b already has in its
-// caches), where the cache rows written are those of batch entry b.  In the
-// chunk form a row outside every sequence, or of a sequence whose rows would
-// leave the caches, writes nothing to the caches.
+// caches), where the cache rows written are those of sequence b (contiguous,
+// or through a block table: `cmap`).  In the chunk form a row outside every
+// sequence, or of a sequence whose rows would leave the caches, writes
+// nothing to the caches, nor does a row whose table entry is outside the pool
+// (reported).
 template <int D, bool kChunk>
 __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
     __half* __restrict__ Qrot, void* __restrict__ Kout, int B, int L, int Hq, int Hkv, int s,
     int c, double log2_base, int q_off, int Tcap, const __nv_bfloat16* __restrict__ Vsrc,
     __nv_bfloat16* __restrict__ Vc, __half* __restrict__ Kh, int kh_rows,
-    const int* __restrict__ cu_seqlens, int n_seq, const int* __restrict__ t0) {
+    const int* __restrict__ cu_seqlens, int n_seq, const int* __restrict__ t0, CacheMap cmap) {
   constexpr int kHalf = D / 2;
   constexpr int kGroups = D / 16;
   __shared__ float2 cs_s[kRopeRows][3][kHalf];  // (cos, sin) per row, position kind, pair
   __shared__ int im_s[kRopeRows];               // row index mod s
-  __shared__ int seq_s[kRopeRows];              // chunk form: cache entry (-1: none)
+  __shared__ int seq_s[kRopeRows];              // chunk form: sequence (-1: no cache rows)
   __shared__ int pos_s[kRopeRows];              // chunk form: absolute index
+  __shared__ long long crow_s[kRopeRows];       // chunk form: cache row (-1: none)
   const long long total_rows = (long long)B * L;
   const long long row0 = (long long)blockIdx.x * kRopeRows;
   const int nrows = (int)min((long long)kRopeRows, total_rows - row0);
@@ -185,6 +188,14 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
       im = (int)(i % s);
     }
     im_s[threadIdx.x] = im;
+    if constexpr (kChunk) {
+      long long cr = -1;
+      if (seq_s[threadIdx.x] >= 0) {
+        cr = cache_row(cmap, seq_s[threadIdx.x], pos_s[threadIdx.x]);
+        if (cr < 0) report_error(kDevBadArg, 104);
+      }
+      crow_s[threadIdx.x] = cr;
+    }
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < nrows * 3 * kHalf; idx += kRopeThreads) {
@@ -210,8 +221,9 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     const long long row = row0 + r;
     if constexpr (kChunk) {
       const int seq = seq_s[r];
-      const size_t cache_row = (size_t)seq * Tcap + pos_s[r];
-      if (hh < 2 * Hkv && seq < 0) continue;  // no cache rows for this row
+      const long long crow = crow_s[r];
+      const size_t cache_row = (size_t)crow;
+      if (hh < 2 * Hkv && crow < 0) continue;  // no cache rows for this row
       if (hh >= Hkv && hh < 2 * Hkv) {  // value copy
         if (!write_v) continue;
         const size_t src = (size_t)row * Hkv * D + (size_t)(hh - Hkv) * D + g * 8;
@@ -346,7 +358,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
 // also zeroes value-cache rows e .. min(e rounded up to 128, rows)-1 after
 // the sequence's new end e = t0[b] + its chunk length (rows no key reaches
 // yet, read with zero weight by the last key tile; zero keeps 0 * value
-// finite), provided the sequence's span lies inside the cache.
+// finite), provided the sequence's span ends by kv_rows.
 __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restrict__ Kc,
                                                           uint4* __restrict__ Kh, int rows,
                                                           int Tcap, int out_rows,
@@ -354,7 +366,8 @@ __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restric
                                                           long long total,
                                                           const int* __restrict__ t0,
                                                           const int* __restrict__ cu_seqlens,
-                                                          uint4* __restrict__ Vc) {
+                                                          uint4* __restrict__ Vc, CacheMap cmap,
+                                                          int kv_rows) {
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
        gid += (long long)gridDim.x * blockDim.x) {
     const long long r = gid / groups_per_row, g = gid % groups_per_row;
@@ -366,13 +379,21 @@ __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restric
           const long long n = (long long)__ldg(cu_seqlens + seq + 1) - __ldg(cu_seqlens + seq);
           const long long e = (long long)off + n;
           const long long tail = min((e + 127) / 128 * 128, (long long)rows);
-          if (off >= 0 && n >= 0 && e <= rows && row >= e && row < tail)
-            Vc[(seq * Tcap + row) * groups_per_row + g] = make_uint4(0u, 0u, 0u, 0u);
+          if (off >= 0 && n >= 0 && e <= kv_rows && row >= e && row < tail) {
+            const long long vr = cache_row(cmap, (int)seq, (int)row);
+            if (vr >= 0) Vc[vr * groups_per_row + g] = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
         continue;
       }
     }
-    uint4 w = __ldg(Kc + (seq * Tcap + row) * groups_per_row + g);
+    if (row >= out_rows) continue;  // (rows may run past out_rows to zero a tail)
+    const long long kr = cache_row(cmap, (int)seq, (int)row);
+    if (kr < 0) {  // table entry outside the pool: reported, the key left unset
+      if (g == 0) report_error(kDevBadArg, 105);
+      continue;
+    }
+    uint4 w = __ldg(Kc + kr * groups_per_row + g);
     uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
     for (int k = 0; k < 4; ++k) u[k] = pack_f16(bf16_lo(u[k]), bf16_hi(u[k]));
@@ -446,7 +467,7 @@ cudaError_t launch_prefill_rope(const void* Q, const void* K, void* Qrot, void* 
     kern<<<blocks, kRopeThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Krot, B, L, Hq, Hkv, s, c, log2((double)base), 0, L,
-        nullptr, nullptr, nullptr, 0, cu_seqlens, n_seq, nullptr);
+        nullptr, nullptr, nullptr, 0, cu_seqlens, n_seq, nullptr, CacheMap{nullptr, 0, 0, 0, L});
   };
   if (D == 64) args(prefill_rope_kernel<64, false>);
   else args(prefill_rope_kernel<128, false>);
@@ -457,7 +478,8 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
                               void* Kcache, void* Vcache, void* Kf16, int B, int Lq, int Hq,
                               int Hkv, int D, int t0, int Tcap, int kh_rows, int s, int c,
                               float base, cudaStream_t stream, const int* cu_seqlens,
-                              int n_seq, const int* t0s) {
+                              int n_seq, const int* t0s, const int* block_table, int max_blocks,
+                              int block_rows, int num_blocks) {
   using namespace rope_path;
   const long long rows = (long long)B * Lq;
   if (rows == 0) return cudaSuccess;
@@ -467,7 +489,8 @@ cudaError_t launch_chunk_rope(const void* Q, const void* K, const void* V, void*
         static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
         static_cast<__half*>(Qrot), Kcache, B, Lq, Hq, Hkv, s, c, log2((double)base), t0, Tcap,
         static_cast<const __nv_bfloat16*>(V), static_cast<__nv_bfloat16*>(Vcache),
-        static_cast<__half*>(Kf16), kh_rows, cu_seqlens, n_seq, t0s);
+        static_cast<__half*>(Kf16), kh_rows, cu_seqlens, n_seq, t0s,
+        CacheMap{block_table, max_blocks, block_rows, num_blocks, Tcap});
   };
   if (D == 64) args(prefill_rope_kernel<64, true>);
   else args(prefill_rope_kernel<128, true>);
@@ -495,9 +518,17 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* Kc, voi
 namespace dca {
 cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, int Tcap,
                                int out_rows, int Hkv, int D, cudaStream_t stream,
-                               const int* t0s, const int* cu_seqlens, void* Vcache) {
+                               const int* t0s, const int* cu_seqlens, void* Vcache,
+                               const int* block_table, int max_blocks, int block_rows,
+                               int num_blocks) {
   using namespace rope_path;
   const long long gpr = (long long)Hkv * D / 8;
+  // Paged values are read by whole 128-row tiles inside a block, past the
+  // last valid row too, so the value tail is zeroed up to the tile edge; a
+  // contiguous cache is read only up to `rows` (the tensor map's extent).
+  const int kv_rows = rows;
+  if (block_table != nullptr && Vcache != nullptr)
+    rows = (int)std::min<long long>(((long long)rows + 127) / 128 * 128, Tcap);
   const long long total = (long long)B * rows * gpr;
   if (total == 0) return cudaSuccess;
   const long long want = (total + 255) / 256;
@@ -505,7 +536,10 @@ cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, 
   keys_to_f16_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(Kcache),
                                                  static_cast<uint4*>(Kf16), rows, Tcap,
                                                  out_rows, gpr, total, t0s, cu_seqlens,
-                                                 static_cast<uint4*>(Vcache));
+                                                 static_cast<uint4*>(Vcache),
+                                                 CacheMap{block_table, max_blocks, block_rows,
+                                                          num_blocks, Tcap},
+                                                 kv_rows);
   return cudaGetLastError();
 }
 }  // namespace dca

@@ -202,6 +202,17 @@ def test_argument_errors_return_codes(lib):
     assert _code(lib.dca_attn_prefill_varlen_chunk(*cargs7, fake, fake, 3, 64, 100, 300, 4, 2,
                                                    128, 400, 16, 32, 1e4, 0.0, ws, 64,
                                                    None)) == 5
+    # paged: block_rows not a multiple of 128, null table, max_kv past the pool's reach
+    pv = (fake,) * 5
+    assert _code(lib.dca_attn_prefill_varlen_chunk_paged(*pv, fake, 4, 64, 16, fake, fake, fake,
+                                                         fake, 3, 64, 100, 200, 4, 2, 128, 16,
+                                                         32, 1e4, 0.0, ws, 1 << 30, None)) == 2
+    assert _code(lib.dca_attn_prefill_varlen_chunk_paged(*pv, None, 4, 128, 16, fake, fake, fake,
+                                                         fake, 3, 64, 100, 200, 4, 2, 128, 16,
+                                                         32, 1e4, 0.0, ws, 1 << 30, None)) == 1
+    assert _code(lib.dca_attn_prefill_varlen_chunk_paged(*pv, fake, 1, 128, 16, fake, fake, fake,
+                                                         fake, 3, 64, 100, 200, 4, 2, 128, 16,
+                                                         32, 1e4, 0.0, ws, 1 << 30, None)) == 1
     # wait self-test: deadline out of range
     assert _code(lib.dca_debug_wait_timeout(0, None)) == 1
     assert _code(lib.dca_debug_wait_timeout(5000000, None)) == 1

@@ -304,3 +304,68 @@ def test_varlen_chunk_bad_offsets_are_reported(bad):
     assert torch.equal(Kg[1].view(torch.int16), Kc[1].view(torch.int16))
     assert torch.equal(Vg[1].view(torch.int16), Vc[1].view(torch.int16))
     dca.dca_sync_status()
+
+
+def _to_pool(cache, block_rows, perm, num_blocks):
+    """Scatter a contiguous cache [B][Tcap][H][D] into a pool of num_blocks
+    blocks; block j of sequence b goes to pool block perm[b * max_blocks + j]."""
+    B, Tcap, H, D = cache.shape
+    nb = Tcap // block_rows
+    pool = torch.full((num_blocks, block_rows, H, D), float("nan"), dtype=cache.dtype)
+    pool[perm] = cache.reshape(B * nb, block_rows, H, D)
+    return pool
+
+
+def _from_pool(pool, perm, B):
+    nb = len(perm) // B
+    blocks = pool[perm]
+    return blocks.reshape(B, nb * pool.shape[1], *pool.shape[2:])
+
+
+@pytest.mark.parametrize("block_rows", [128, 256])
+@pytest.mark.parametrize("case", VARLEN_CHUNK_CASES[:3], ids=str)
+def test_varlen_chunk_paged_equals_contiguous(case, block_rows):
+    lens, t0, Hq, Hkv, D, s, c, _ = case
+    max_kv = max(a + n for a, n in zip(t0, lens))
+    Tcap = (max_kv + block_rows - 1) // block_rows * block_rows + block_rows
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed=65)
+    O1, L1, Kd, Vd = _run_chunk(Q, K, V, Kc, Vc, cu, t0, s, c, max_kv)
+    dca.dca_sync_status()
+    B, nb = len(lens), Tcap // block_rows
+    num_blocks = B * nb + 3
+    perm = torch.randperm(num_blocks, generator=torch.Generator().manual_seed(66))[:B * nb]
+    Kp, Vp = _to_pool(Kc, block_rows, perm, num_blocks), _to_pool(Vc, block_rows, perm,
+                                                                   num_blocks)
+    Kpd, Vpd = Kp.cuda(), Vp.cuda()
+    table = perm.view(B, nb).to(torch.int32).cuda()
+    O2, L2 = dca.dca_attn_prefill_varlen_chunk_paged(
+        Q.cuda(), K.cuda(), V.cuda(), Kpd, Vpd, table, cu.cuda(),
+        torch.tensor(t0, dtype=torch.int32, device="cuda"), max(lens), max_kv, s, c)
+    dca.dca_sync_status()
+    # same bits out, same cache rows written and zeroed (the pool's unused
+    # blocks untouched)
+    assert torch.equal(O1.cpu(), O2.cpu()) and torch.equal(L1.cpu(), L2.cpu())
+    Kp2, Vp2 = Kpd.cpu(), Vpd.cpu()
+    assert torch.equal(_from_pool(Kp2, perm, B).view(torch.int16), Kd.cpu().view(torch.int16))
+    assert torch.equal(_from_pool(Vp2, perm, B).view(torch.int16), Vd.cpu().view(torch.int16))
+    unused = sorted(set(range(num_blocks)) - set(perm.tolist()))
+    assert torch.isnan(Kp2[unused].float()).all() and torch.isnan(Vp2[unused].float()).all()
+
+
+def test_varlen_chunk_paged_table_out_of_range_is_reported():
+    lens, t0, Hq, Hkv, D, s, c = [100, 200], [300, 0], 2, 1, 128, 256, 384
+    block_rows, Tcap = 128, 512
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed=67)
+    B, nb = 2, Tcap // block_rows
+    perm = torch.arange(B * nb)
+    Kpd, Vpd = _to_pool(Kc, block_rows, perm, B * nb).cuda(), \
+        _to_pool(Vc, block_rows, perm, B * nb).cuda()
+    table = perm.view(B, nb).to(torch.int32)
+    table[0, 1] = B * nb  # sequence 0's cached rows 128 .. 255: a block past the pool
+    dca.dca_attn_prefill_varlen_chunk_paged(
+        Q.cuda(), K.cuda(), V.cuda(), Kpd, Vpd, table.cuda(), cu.cuda(),
+        torch.tensor(t0, dtype=torch.int32, device="cuda"), max(lens), 400, s, c)
+    with pytest.raises(dca.DcaError) as ei:
+        dca.dca_sync_status()
+    assert ei.value.status == 1
+    dca.dca_sync_status()  # cleared; the context keeps working
