@@ -592,8 +592,9 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
                                paged ? (uint64_t)vmap.num_blocks : (uint64_t)Bk};
     const uint64_t ks[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
                             (uint64_t)k_rows * Hkv * D * 2};
-    const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
-                            (uint64_t)v_rows * Hkv * D * 2};
+    // paged values: consecutive blocks are block_rows rows apart in the pool
+    const uint64_t vpitch = paged ? (uint64_t)vmap.block_rows : (uint64_t)v_rows;
+    const uint64_t vs[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2, vpitch * Hkv * D * 2};
     if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Krot, 4, kdims, ks, box,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, 4, vdims, vs, box,
