@@ -342,12 +342,16 @@ def test_varlen_chunk_paged_equals_contiguous(case, block_rows):
         Q.cuda(), K.cuda(), V.cuda(), Kpd, Vpd, table, cu.cuda(),
         torch.tensor(t0, dtype=torch.int32, device="cuda"), max(lens), max_kv, s, c)
     dca.dca_sync_status()
-    # same bits out, same cache rows written and zeroed (the pool's unused
-    # blocks untouched)
+    # same bits out, same cache rows written; the value tail zeroed to the
+    # 128-row tile edge (the contiguous call stops at max_kv, which its value
+    # map does not read past); the pool's unused blocks untouched
     assert torch.equal(O1.cpu(), O2.cpu()) and torch.equal(L1.cpu(), L2.cpu())
     Kp2, Vp2 = Kpd.cpu(), Vpd.cpu()
     assert torch.equal(_from_pool(Kp2, perm, B).view(torch.int16), Kd.cpu().view(torch.int16))
-    assert torch.equal(_from_pool(Vp2, perm, B).view(torch.int16), Vd.cpu().view(torch.int16))
+    want_v = Vd.cpu().clone()
+    for b, (a, n) in enumerate(zip(t0, lens)):
+        want_v[b, a + n:min((a + n + 127) // 128 * 128, Tcap)] = 0
+    assert torch.equal(_from_pool(Vp2, perm, B).view(torch.int16), want_v.view(torch.int16))
     unused = sorted(set(range(num_blocks)) - set(perm.tolist()))
     assert torch.isnan(Kp2[unused].float()).all() and torch.isnan(Vp2[unused].float()).all()
 
