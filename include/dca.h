@@ -212,8 +212,9 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
                                     float scale, void* workspace, size_t ws_bytes, void* stream);
 
 /* Workspace bytes for dca_attn_prefill_varlen_chunk: the fp16 query
- * rotations [3][T][Hq][D] and fp16 keys [B][max_kv][Hkv][D], each rounded up
- * to 256 bytes.  Returns 0 for unsupported arguments. */
+ * rotations [3][T][Hq][D], fp16 keys [B][max_kv][Hkv][D] and the attention's
+ * work order (B * ceil(T / 256) ints), each rounded up to 256 bytes.
+ * Returns 0 for unsupported arguments. */
 size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq, int Hkv,
                                                int D);
 
@@ -239,8 +240,9 @@ size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq,
  *   O [T][Hq][D] bf16, LSE [Hq][T] fp32: results for the packed rows; rows of
  *     no sequence are left untouched.
  * Kernels: the fused RoPE kernel in chunk form, the key conversion to fp16
- * of rows 0 .. t0[b]-1, then the per-row-interval tcgen05 kernel with each
- * sequence's offset.  Offsets that break the rules above are checked where
+ * of rows 0 .. t0[b]-1, a one-block counting sort of the (sequence, 256-row
+ * query pair) items by decreasing key count, then the per-row-interval
+ * tcgen05 kernel with each sequence's offset, dispatched in that order.  Offsets that break the rules above are checked where
  * the kernels read them: that sequence is skipped (no cache row, O or LSE
  * written) and the device error word is set (DCA_ERR_INVALID_ARG at the next
  * dca_sync_status).  The call owns no memory; `workspace`

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, Rule rule, float scale_log2,
     int q_off, int group_units, const int* __restrict__ cu_seqlens, int T,
-    const int* __restrict__ t0s, int kv_rows, CacheMap vmap) {
+    const int* __restrict__ t0s, int kv_rows, CacheMap vmap, const int* __restrict__ order) {
   using LD = Lay<D>;
   constexpr int kHalves = LD::kHalves, kTileBytes = LD::kTileBytes;
   constexpr int kSmQ = LD::kSmQ, kSmK = LD::kSmK, kSmV = LD::kSmV, kSmBar = LD::kSmBar;
@@ -216,10 +216,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
   const int num_qt = (L + kTile - 1) / kTile;
   const int num_pairs = (num_qt + 1) / 2;
   // longest pairs first over all (sequence, kv head) units (one group: with
-  // L2-sized groups the longer, uneven visits of this kernel left a tail)
-  const PairOrder po = pair_order((int)blockIdx.x, num_pairs, Hq, Hkv, B, group_units);
-  const int m = num_pairs - 1 - po.m_rank;
-  const int h = po.h, b = po.b;
+  // L2-sized groups the longer, uneven visits of this kernel left a tail);
+  // with per-sequence offsets the work of a pair depends on its sequence's
+  // offset too, and a precomputed order (sequence, pair) by decreasing key
+  // count is read instead, all q heads of an item in a row
+  int m, h, b;
+  if (kSeqOff && order != nullptr) {
+    const int item = __ldg(order + blockIdx.x / Hq);
+    if (item < 0) return;  // uniform across the CTA: fewer items than slots
+    b = item / num_pairs;
+    m = item - b * num_pairs;
+    h = (int)(blockIdx.x % Hq);
+  } else {
+    const PairOrder po = pair_order((int)blockIdx.x, num_pairs, Hq, Hkv, B, group_units);
+    m = num_pairs - 1 - po.m_rank;
+    h = po.h;
+    b = po.b;
+  }
   const int hk = h / (Hq / Hkv);
   const int q0_loc = m * 2 * kTile;          // row of this call
   SeqSpan sq0;
@@ -550,6 +563,52 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_gen_kernel(
 
 namespace gen_path {
 
+// Work order of packed chunks over caches: every (sequence b, query-tile pair
+// m) item, m < ceil(n_b / 256) (one item with m = 0 for an empty or invalid
+// sequence, so that its span is still checked), sorted by decreasing key
+// count t0[b] + 256 m + 256 in 256-key buckets (a counting sort, one CTA);
+// slots past the items hold -1.  Item = b * num_pairs + m.
+constexpr int kOrderBuckets = 2048;
+__global__ void __launch_bounds__(1024) pair_work_order_kernel(const int* __restrict__ cu_seqlens,
+                                                               const int* __restrict__ t0, int B,
+                                                               int num_pairs,
+                                                               int* __restrict__ order) {
+  __shared__ int cnt[kOrderBuckets];
+  const long long slots = (long long)B * num_pairs;
+  for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  auto pairs_of = [&](int b) {
+    const long long n = (long long)__ldg(cu_seqlens + b + 1) - __ldg(cu_seqlens + b);
+    const long long p = n > 0 ? (n + 255) / 256 : 1;
+    return (int)(p < num_pairs ? p : num_pairs);
+  };
+  auto bucket_of = [&](int b, int m) {
+    const long long keys = (long long)max(__ldg(t0 + b), 0) + 256ll * m + 256;
+    const long long k = keys / 256;
+    return kOrderBuckets - 1 - (int)(k < kOrderBuckets - 1 ? k : kOrderBuckets - 1);
+  };
+  for (long long it = threadIdx.x; it < slots; it += blockDim.x) {
+    const int b = (int)(it / num_pairs), m = (int)(it % num_pairs);
+    if (m < pairs_of(b)) atomicAdd(&cnt[bucket_of(b, m)], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // exclusive prefix sum (2048 buckets)
+    int run = 0;
+    for (int i = 0; i < kOrderBuckets; ++i) {
+      const int c = cnt[i];
+      cnt[i] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (long long it = threadIdx.x; it < slots; it += blockDim.x) order[it] = -1;
+  __syncthreads();
+  for (long long it = threadIdx.x; it < slots; it += blockDim.x) {
+    const int b = (int)(it / num_pairs), m = (int)(it % num_pairs);
+    if (m < pairs_of(b)) order[atomicAdd(&cnt[bucket_of(b, m)], 1)] = (int)it;
+  }
+}
+
 // Tensor maps and launch: Qrot [nq planes][B][L][Hq][D] and Krot [kKPlanes]
 // [B][k_rows][Hkv][D] fp16, V [B][v_rows][Hkv][D] bf16.  With cu_seqlens
 // (device [B+1], q_off == 0) each tensor is one packed batch of T rows
@@ -559,7 +618,7 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
                          int B, int L, int Hq, int Hkv, Rule rule, int nq, float scale,
                          cudaStream_t stream, int q_off, int k_rows, int v_rows,
                          const int* cu_seqlens, int T, const int* t0s, int kv_rows,
-                         CacheMap vmap) {
+                         CacheMap vmap, int* order) {
   if (q_off < 0) return cudaErrorInvalidValue;
   if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
   if (t0s != nullptr && (cu_seqlens == nullptr || kv_rows < 1)) return cudaErrorInvalidValue;
@@ -612,10 +671,16 @@ cudaError_t launch_gen_d(const void* Qrot, const void* Krot, const void* V, void
                                                LSE, B, L, Hq, Hkv, rule,
                                                scale * 1.4426950408889634f, q_off,
                                                B * Hkv,  // one group: longest first
-                                               cu_seqlens, T, t0s, Lkv, vmap);
+                                               cu_seqlens, T, t0s, Lkv, vmap, order);
     return cudaGetLastError();
   };
   if (t0s == nullptr) return run(prefill_attn_gen_kernel<D, Rule, false>);
+  if (order != nullptr) {  // (sequence, pair) items by decreasing key count
+    const int num_pairs = ((L + kTile - 1) / kTile + 1) / 2;
+    pair_work_order_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, t0s, B, num_pairs, order);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if constexpr (Rule::kKPlanes == 1) return run(prefill_attn_gen_kernel<D, Rule, true>);
   return cudaErrorInvalidValue;  // per-sequence offsets: DCA rule only
 }
@@ -625,13 +690,14 @@ cudaError_t launch_gen(const void* Qrot, const void* Krot, const void* V, void* 
                        int B, int L, int Hq, int Hkv, int D, Rule rule, int nq, float scale,
                        cudaStream_t stream, int q_off, int k_rows, int v_rows,
                        const int* cu_seqlens = nullptr, int T = 0, const int* t0s = nullptr,
-                       int kv_rows = 0, CacheMap vmap = CacheMap{nullptr, 0, 0, 0, 0}) {
+                       int kv_rows = 0, CacheMap vmap = CacheMap{nullptr, 0, 0, 0, 0},
+                       int* order = nullptr) {
   if (D == 64)
     return launch_gen_d<64>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream, q_off,
-                            k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap);
+                            k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap, order);
   if (D == 128)
     return launch_gen_d<128>(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, rule, nq, scale, stream,
-                             q_off, k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap);
+                             q_off, k_rows, v_rows, cu_seqlens, T, t0s, kv_rows, vmap, order);
   return cudaErrorInvalidValue;
 }
 
@@ -646,12 +712,13 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
                                           int q_off, int k_rows, int v_rows,
                                           const int* cu_seqlens, int T, const int* t0s,
                                           int kv_rows, const int* block_table, int max_blocks,
-                                          int block_rows, int num_blocks) {
+                                          int block_rows, int num_blocks, int* order) {
   if (s < 1) return cudaErrorInvalidValue;
   return gen_path::launch_gen(Qrot, Krot, V, O, LSE, B, L, Hq, Hkv, D,
                               gen_path::DcaIntervals{s}, 3, scale, stream, q_off, k_rows,
                               v_rows, cu_seqlens, T, t0s, kv_rows,
-                              CacheMap{block_table, max_blocks, block_rows, num_blocks, 0});
+                              CacheMap{block_table, max_blocks, block_rows, num_blocks, 0},
+                              order);
 }
 
 // SelfExtend on the same kernel: Qse, Kse [2][B][L][H][D] fp16 (neighbour,

@@ -67,6 +67,9 @@ dca_status_t check_heads(const char* fn, int B, int L, int Hq, int Hkv, int D) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Query-tile pairs (256 rows) of a sequence of n rows, at least 1.
+size_t varlen_pair_slots(int n) { return n > 0 ? ((size_t)n + 255) / 256 : 1; }
+
 struct PrefillWs {
   void* qrot;
   void* krot;
@@ -362,9 +365,12 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
 
 size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq, int Hkv,
                                                int D) {
+  // (the work order of the attention: one int per (sequence, 256-row query
+  // pair) slot, T bounding every sequence's length)
   if (B < 0 || T < 0 || max_kv < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128))
     return 0;
-  return align256((size_t)3 * T * Hq * D * 2) + align256((size_t)B * max_kv * Hkv * D * 2);
+  return align256((size_t)3 * T * Hq * D * 2) + align256((size_t)B * max_kv * Hkv * D * 2) +
+         align256((size_t)B * varlen_pair_slots(T) * 4);
 }
 
 }  // extern "C"
@@ -383,6 +389,7 @@ dca_status_t varlen_chunk_impl(const char* fn, const void* Q, const void* K, con
   if (st == DCA_OK) st = check_chunking(fn, s, c, base);
   if (st != DCA_OK) return st;
   if (T < 0) return fail(DCA_ERR_INVALID_ARG, "%s: T=%d", fn, T);
+  if (max_seqlen > T) max_seqlen = T;  // no sequence is longer than the pack
   if (Tcap < 1 || max_kv < 1 || max_kv > Tcap)
     return fail(DCA_ERR_INVALID_ARG, "%s: need 1 <= max_kv=%d <= Tcap=%d", fn, max_kv, Tcap);
   if (auto_path(D, s) != DCA_PATH_TCGEN05)
@@ -408,6 +415,8 @@ dca_status_t varlen_chunk_impl(const char* fn, const void* Q, const void* K, con
   // the bf16 cache and, rounded once, to fp16; cache rows 0 .. t0[b]-1 are
   // converted to fp16 as stored.
   void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * T * Hq * D * 2);
+  int* order = reinterpret_cast<int*>(static_cast<char*>(kf16) +
+                                      align256((size_t)B * max_kv * Hkv * D * 2));
   cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, 1, T, Hq, Hkv, D,
                                     0, Tcap, max_kv, s, c, base, strm, cu_seqlens, B, t0,
                                     block_table, max_blocks, block_rows, num_blocks);
@@ -417,7 +426,7 @@ dca_status_t varlen_chunk_impl(const char* fn, const void* Q, const void* K, con
   if (e == cudaSuccess)
     e = launch_prefill_attn_sm100_gen(workspace, kf16, Vcache, O, LSE, B, max_seqlen, Hq, Hkv, D,
                                       s, sc, strm, 0, max_kv, Tcap, cu_seqlens, T, t0, max_kv,
-                                      block_table, max_blocks, block_rows, num_blocks);
+                                      block_table, max_blocks, block_rows, num_blocks, order);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 

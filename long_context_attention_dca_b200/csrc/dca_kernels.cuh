@@ -85,6 +85,8 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
 // 0 .. t0s[b]+r of batch entry b of Krot [B][k_rows pitch] and V [B][v_rows
 // pitch], kv_rows rows valid per entry; with block_table the values come
 // from a paged pool [num_blocks][block_rows][Hkv][D] (block_rows % 128 == 0).
+// `order` (device, B * ceil(ceil(L/128)/2) ints of scratch) lets the packed
+// chunk form dispatch its (sequence, pair) items by decreasing key count.
 cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, const void* V,
                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                           int D, int s, float scale, cudaStream_t stream,
@@ -92,7 +94,8 @@ cudaError_t launch_prefill_attn_sm100_gen(const void* Qrot, const void* Krot, co
                                           const int* cu_seqlens = nullptr, int T = 0,
                                           const int* t0s = nullptr, int kv_rows = 0,
                                           const int* block_table = nullptr, int max_blocks = 0,
-                                          int block_rows = 0, int num_blocks = 0);
+                                          int block_rows = 0, int num_blocks = 0,
+                                          int* order = nullptr);
 // SelfExtend on the per-row-interval tcgen05 kernel (D = 64 or 128).
 cudaError_t launch_prefill_attn_sm100_selfextend(const void* Qse, const void* Kse,
                                                  const void* V, void* O, float* LSE, int B,

@@ -80,7 +80,9 @@ def test_workspace_queries(lib):
     # packed chunks over caches: query rotations of the T rows + fp16 keys of
     # max_kv rows per sequence
     assert dca.dca_attn_prefill_varlen_chunk_workspace(3, 100, 300, 4, 2, 128) == (
-        up(3 * 100 * 4 * 128 * 2) + up(3 * 300 * 2 * 128 * 2))
+        up(3 * 100 * 4 * 128 * 2) + up(3 * 300 * 2 * 128 * 2) + up(3 * 1 * 4))
+    assert dca.dca_attn_prefill_varlen_chunk_workspace(3, 1000, 300, 4, 2, 128) == (
+        up(3 * 1000 * 4 * 128 * 2) + up(3 * 300 * 2 * 128 * 2) + up(3 * 4 * 4))
     assert dca.dca_attn_prefill_varlen_chunk_workspace(3, 100, -1, 4, 2, 128) == 0
 
 
