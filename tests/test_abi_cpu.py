@@ -34,6 +34,42 @@ def test_header_declares_the_binding_surface():
     assert _header_functions() == sorted(dca.EXPORTED_SYMBOLS)
 
 
+def _header_prototypes():
+    """{name: [parameter type strings]} for every function in the header."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(dca_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip()]
+        if params == ["void"]:
+            params = []
+        out[m.group(1)] = params
+    return out
+
+
+def _ctype_of(param):
+    """The ctypes class the binding must use for a C parameter."""
+    t = re.sub(r"\b[A-Za-z_][A-Za-z0-9_]*$", "", param).strip() if " " in param else param
+    if "*" in t:
+        return ctypes.c_void_p
+    t = t.replace("const", "").strip()
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "dca_pos_rule_t": ctypes.c_int}[t]
+
+
+def test_binding_signatures_match_the_header():
+    # every argument the ctypes binding passes has the C type of the
+    # header's parameter at that position (a count or type slip would pass
+    # garbage through the ABI)
+    protos = _header_prototypes()
+    assert sorted(protos) == sorted(dca.EXPORTED_SYMBOLS)
+    for name, params in protos.items():
+        _, argtypes = dca._SIGS[name]
+        assert len(argtypes) == len(params), (name, len(argtypes), len(params))
+        for i, (want, got) in enumerate(zip(params, argtypes)):
+            assert _ctype_of(want) is got, (name, i, want, got)
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in _header_functions():
         assert hasattr(lib, name), name
