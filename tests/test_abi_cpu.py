@@ -264,3 +264,20 @@ def test_binding_fails_loudly_without_cuda_tensors(lib):
     x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(dca.DcaError):
         dca.dca_rope_rotate(x, dca.DCA_POS_KEY, 4, 6)
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary header must stay usable from C: compile a translation unit
+    # that includes it with a strict C99 compiler (no CUDA or C++ types)
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "dca.h"\n'
+                   "size_t f(void) { return dca_attn_prefill_workspace(1, 1, 1, 1, 64); }\n")
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                          os.path.dirname(HEADER), "-c", str(src), "-o",
+                          str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
