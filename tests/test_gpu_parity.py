@@ -297,6 +297,21 @@ def test_decode_long_splits_with_short_sequences():
     assert (O[0].float() - Vc[0, 0].float().repeat_interleave(8, dim=0)).abs().max() <= 2e-2
 
 
+def test_decode_independent_of_split_size():
+    # the same four sequences decoded alone (4 x 8 x 19 = 608 CTAs: 1024-key
+    # splits) and inside a batch of eight (1216 CTAs: 2048-key splits) agree
+    # to fp32 reordering: the LSE merge of partial softmaxes is exact
+    cfg = dict(B=8, Hq=64, Hkv=8, D=128, Tcap=19 * 2048, t_lo=30000, t_hi=19 * 2048)
+    t, q, Kc, Vc = W.make_decode_inputs(cfg, seed=10)
+    s, c = 3072, 4096
+    O8, L8 = _decode_gpu(t, q, Kc, Vc, s, c)
+    O4, L4 = _decode_gpu(t[:4].contiguous(), q[:4].contiguous(), Kc[:4].contiguous(),
+                         Vc[:4].contiguous(), s, c)
+    assert (L8[:4] - L4).abs().max() <= 5e-5
+    # bf16 outputs: at most one rounding step apart
+    assert (O8[:4].float() - O4.float()).abs().max() <= 8e-3
+
+
 def test_decode_equals_prefill_row_on_gpu():
     # Same K/V: the decode of token t (cache rotated by the library's RoPE at
     # j mod s) must equal row t of prefill, and both must match the oracle.
