@@ -24,7 +24,8 @@
  *   - Pointers are DEVICE pointers unless stated; the caller owns all memory
  *     and the library allocates none.  Scratch comes from the caller's
  *     workspace (size from the *_workspace query; 256-byte alignment is
- *     recommended, 16-byte alignment is required of every pointer).
+ *     recommended, 16-byte alignment is required of every tensor pointer;
+ *     int32 index arrays such as t, cu_seqlens, t0 and block tables need 4).
  *   - Tensors are contiguous.  bf16 unless stated; LSE is fp32.
  *       Q, O      [B][L][Hq][D]        K, V          [B][L][Hkv][D]
  *       LSE       [B][Hq][L]           q (decode)    [B][Hq][D]
@@ -35,8 +36,11 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous: they enqueue kernels and return.  A kernel-side failure
  *     (a pipeline wait that ran past its deadline, a decode position outside
- *     the cache) is recorded in a per-device error word and reported by
- *     dca_sync_status().  Nothing is thrown across the ABI and no kernel traps.
+ *     the cache, packed or cache offsets that do not form a valid span, a
+ *     block-table entry outside its pool) is recorded in a per-device error
+ *     word and reported by dca_sync_status(); the kernels skip the offending
+ *     work instead of following the bad value.  Nothing is thrown across the
+ *     ABI and no kernel traps.
  *   - On a non-DCA_OK return nothing was enqueued; dca_last_error_string()
  *     (per host thread) says why.
  */
