@@ -45,7 +45,10 @@ Pins that hold this module to something other than itself live in
 reduction to plain RoPE attention, Q = 0 and constant-V closed forms, RoPE
 relativity, decode = prefill row, chunk = whole-sequence rows, packed batch =
 padded batch and its Q = 0 closed form, hand-worked
-SelfExtend distance tables and its reductions to plain RoPE attention) and
+SelfExtend distance tables and its reductions to plain RoPE attention, whole
+DCA and SelfExtend rows rebuilt from the hand-worked distance tables, the
+tensor rotation under every rule and offset against positions listed row by
+row) and
 ``tests/test_oracle_mutations.py``
 (plausible mistakes planted here must each fail a pin).
 """

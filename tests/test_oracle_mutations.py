@@ -8,8 +8,11 @@ causal off-by-one, a wrong GQA mapping, a shifted chunk origin, a broken
 partial merge, a decode that reads one key too few, a chunked prefill
 that ignores or misaligns its cache, or a packed variable-length batch that
 leaks across sequences, counts positions from the packed start or reports
-local rows, and packed chunks that ignore their cache offsets or read
-another sequence's cache.  The pins of
+local rows, packed chunks that ignore their cache offsets or read
+another sequence's cache, a tensor rotation that drops its position offset
+or lays positions along the head axis, a SelfExtend row that rotates a
+grouped query at its own index, and a DCA row that rotates its query once
+for all keys.  The pins of
 ``test_oracle_pins`` must reject each one.
 """
 
@@ -216,6 +219,42 @@ def _varlen_chunk_first_cache(Q, K, V, cu_seqlens, t0, k_cache_rot, v_cache, *ar
                               np.repeat(v_cache[:1], B, axis=0), *args, **kw)
 
 
+_ORIG_RULE_POS = orc.rule_positions
+_ORIG_SE_ROW = orc.selfextend_row
+_ORIG_DCA_ROW = orc.dca_row
+
+
+def _rope_rotate_no_offset(x, rule, s, c, base, pos_offset=0):
+    # pos_offset dropped: every call rotates as if the rows started at index 0
+    x = np.asarray(x, np.float64)
+    pos = _ORIG_RULE_POS(x.shape[1], rule, s, c, 0)
+    return orc.rotate(x, pos[None, :, None], base)
+
+
+def _rope_rotate_head_axis(x, rule, s, c, base, pos_offset=0):
+    # positions laid along the head axis instead of the row axis
+    x = np.asarray(x, np.float64)
+    pos = _ORIG_RULE_POS(x.shape[2], rule, s, c, pos_offset)
+    return orc.rotate(x, pos[None, None, :], base)
+
+
+def _se_row_query_at_i(q, k, v, i, G, W, base, scale):
+    # grouped pairs rotate the query at its own index i instead of the
+    # shifted grouped position
+    j = np.arange(i + 1, dtype=np.int64)
+    _, kpos = orc.selfextend_positions(i, j, G, W)
+    z = orc.rotate(k, kpos, base) @ orc.rotate(q, i, base)
+    return orc.softmax_row(scale * z, v)
+
+
+def _dca_row_one_rotation(q, k_rot, v, i, s, c, base, scale):
+    # the query rotated once, at the position its first key asks for, and
+    # used for every key
+    pq = orc.query_position(i, np.arange(i + 1), s, c)
+    z = k_rot @ orc.rotate(q, pq[0], base)
+    return orc.softmax_row(scale * z, v)
+
+
 MUTANTS = {
     "succ_rule_le": ("query_position", _qpos_succ_le),
     "succ_far_pos_c": ("query_position", _qpos_succ_c),
@@ -242,6 +281,10 @@ MUTANTS = {
     "varlen_local_keys": ("dca_prefill_varlen_rows", _varlen_local_keys),
     "varlen_chunk_no_offset": ("dca_prefill_varlen_chunk_rows", _varlen_chunk_no_offset),
     "varlen_chunk_first_cache": ("dca_prefill_varlen_chunk_rows", _varlen_chunk_first_cache),
+    "rope_rotate_no_offset": ("rope_rotate", _rope_rotate_no_offset),
+    "rope_rotate_head_axis": ("rope_rotate", _rope_rotate_head_axis),
+    "selfextend_query_at_i": ("selfextend_row", _se_row_query_at_i),
+    "dca_row_one_rotation": ("dca_row", _dca_row_one_rotation),
 }
 
 

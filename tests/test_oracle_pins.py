@@ -21,7 +21,11 @@ them against the oracle as committed.  Sources of each fact:
   rows (the rule depends only on absolute indices);
 * SelfExtend (LLM Maybe LongLM, abstract): hand-worked neighbour / grouped
   distance tables under ``tests/golden/``, its reduction to plain RoPE
-  attention for G = 1 or W >= L (torch SDPA), and distance bounds.
+  attention for G = 1 or W >= L (torch SDPA), and distance bounds;
+* whole attention rows (DCA and SelfExtend) rebuilt from the hand-worked
+  distance tables alone, through RoPE relativity;
+* the rotation of a whole tensor under each position rule and offset,
+  against positions listed row by row and a few literal values.
 """
 
 import math
@@ -425,6 +429,88 @@ def pin_selfextend_distance_bounds():
             assert (np.diff(d[::-1]) >= 0).all()
 
 
+def pin_rope_rotate():
+    # rope_rotate on [B, L, H, D] with L != H: row r of every batch entry and
+    # head is turned to the rule's position of absolute index pos_offset + r.
+    # The positions are listed per row here from the rule as the pages state
+    # it; the rotation is the complex-number RoPE.
+    s, c = 5, 8
+    x = _rand((2, 11, 3, 8), 60)
+    for off in (0, 17, s - 1, 3 * s + 2):
+        for rule in (orc.POS_KEY, orc.POS_Q_INTRA, orc.POS_Q_SUCC, orc.POS_Q_INTER,
+                     orc.POS_ABSOLUTE):
+            want_pos = []
+            for r in range(x.shape[1]):
+                i = off + r
+                if rule == orc.POS_ABSOLUTE:
+                    want_pos.append(i)
+                elif rule in (orc.POS_KEY, orc.POS_Q_INTRA):
+                    want_pos.append(i % s)
+                elif rule == orc.POS_Q_SUCC:
+                    want_pos.append(s + i % s if i % s < c - s else c - 1)
+                else:
+                    want_pos.append(c - 1)
+            want = _complex_rotate(x, np.array(want_pos)[None, :, None], 100.0)
+            got = orc.rope_rotate(x, rule, s, c, 100.0, pos_offset=off)
+            assert got.shape == x.shape
+            np.testing.assert_allclose(got, want, atol=1e-12, err_msg=f"rule {rule} off {off}")
+    # literal values, D = 2 (one pair, theta_0 = 1): x = (1, 0) turned by the
+    # angle p gives (cos p, sin p).  s = 3, c = 5 (w = 2): index 4 has
+    # 4 mod 3 = 1 < w, so the successive position is 3 + 1 = 4; index 5 has
+    # 5 mod 3 = 2 >= w, so it is c - 1 = 4 as well; index 3 has intra 0.
+    e = np.zeros((1, 3, 1, 2))
+    e[..., 0] = 1.0
+    got = orc.rope_rotate(e, orc.POS_Q_SUCC, 3, 5, 10000.0, pos_offset=3)
+    np.testing.assert_allclose(got[0, :, 0], [[math.cos(3), math.sin(3)],
+                                              [math.cos(4), math.sin(4)],
+                                              [math.cos(4), math.sin(4)]], atol=1e-15)
+    got = orc.rope_rotate(e, orc.POS_Q_INTRA, 3, 5, 10000.0, pos_offset=3)
+    np.testing.assert_allclose(got[0, :, 0], [[1, 0], [math.cos(1), math.sin(1)],
+                                              [math.cos(2), math.sin(2)]], atol=1e-15)
+
+
+def _softmax_from_distances(q, k, v, dist, base, sc):
+    """Row outputs from an explicit distance per key: by RoPE relativity the
+    score of the pair is <R(d) q, k>, so only the distance is needed."""
+    z = np.array([_complex_rotate(q, d, base) @ k[n] for n, d in enumerate(dist)]) * sc
+    m = z.max()
+    e = np.exp(z - m)
+    return (e @ v) / e.sum(), m + math.log(e.sum())
+
+
+def pin_dca_rows_from_worked_tables():
+    # every row of a DCA prefill rebuilt from the hand-worked distance tables
+    # alone: score = scale * <R(d_ij) q_i, k_j>, one naive softmax per row
+    for name, s, c in TABLES:
+        _, want_d = parse_table(name)
+        L = want_d.shape[0]
+        Q, K, V = _rand((1, L, 2, 8), 61), _rand((1, L, 1, 8), 62), _rand((1, L, 1, 8), 63)
+        O, LSE = orc.dca_prefill(Q, K, V, s, c, base=100.0)
+        for h in range(2):
+            for i in range(L):
+                o, lse = _softmax_from_distances(Q[0, i, h], K[0, :i + 1, 0], V[0, :i + 1, 0],
+                                                 want_d[i, :i + 1], 100.0, 1 / math.sqrt(8))
+                np.testing.assert_allclose(O[0, i, h], o, atol=1e-12, err_msg=name)
+                np.testing.assert_allclose(LSE[0, h, i], lse, atol=1e-12, err_msg=name)
+
+
+def pin_selfextend_rows_from_worked_tables():
+    # every SelfExtend row rebuilt from the hand-worked neighbour / grouped
+    # distance tables alone, as for the DCA rows above
+    for name, G, W in SE_TABLES:
+        _, want_d = parse_table(name, {"N": 0, "G": 1})
+        L = want_d.shape[0]
+        Q, K, V = _rand((1, L, 2, 8), 64), _rand((1, L, 1, 8), 65), _rand((1, L, 1, 8), 66)
+        got = orc.selfextend_prefill_rows(Q, K, V, G, W, base=100.0)
+        assert len(got) == 2 * L
+        for (b, h, i), (o, lse) in got.items():
+            o_ref, lse_ref = _softmax_from_distances(Q[0, i, h], K[0, :i + 1, 0],
+                                                     V[0, :i + 1, 0], want_d[i, :i + 1],
+                                                     100.0, 1 / math.sqrt(8))
+            np.testing.assert_allclose(o, o_ref, atol=1e-12, err_msg=name)
+            np.testing.assert_allclose(lse, lse_ref, atol=1e-12, err_msg=name)
+
+
 PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_rotation_literals, pin_rope_relativity, pin_plain_rope_matches_sdpa,
         pin_single_chunk_is_plain_rope, pin_long_sequence_differs_from_plain,
@@ -433,8 +519,9 @@ PINS = [pin_worked_tables, pin_distance_bounds, pin_piece_counts,
         pin_varlen_equals_padded_batch, pin_varlen_q_zero_closed_form,
         pin_varlen_chunk_equals_whole_sequences, pin_varlen_chunk_q_zero_closed_form,
         pin_merge_partials,
-        pin_rule_positions, pin_selfextend_worked_tables, pin_selfextend_reduces_to_plain_rope,
-        pin_selfextend_distance_bounds]
+        pin_rule_positions, pin_rope_rotate, pin_dca_rows_from_worked_tables,
+        pin_selfextend_worked_tables, pin_selfextend_reduces_to_plain_rope,
+        pin_selfextend_distance_bounds, pin_selfextend_rows_from_worked_tables]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
