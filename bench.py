@@ -1,16 +1,21 @@
 """Benchmark of the DCA hot path on B200.
 
 One step = one pass of the whole path on synthetic data:
-  prefill  (Llama-2-7B attention shape, L=16384, 32/32 heads, D=128,
-            c=4096, s=3072): fused RoPE, then DCA attention;
+  prefill  (the 100k-token workload: L=100000, 64 query / 8 kv heads, D=128,
+            c=4096, s=3072, ragged last chunk): fused RoPE, then DCA attention;
   decode   (16 sequences, 64/8 heads, D=128, t ~ U[32768, 65536), cache
             pre-rotated at j mod s): split-KV kernel, then LSE merge.
 `value` is prefill TFLOP/s (algorithmic causal FLOPs 4*D*Hq*B*L(L+1)/2 over
 the device time of RoPE + attention); decode KV GB/s is reported beside it.
+The other prefill workloads (Llama-2 70B-shaped GQA at 32k tokens with K
+doubled on 1% of positions, Llama-2 7B-shaped at 16k, and the tiny one) are
+timed after the step, each on its own inputs, and reported under `configs`.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
-(the path has no exchange step), times are max-reduced over ranks.
+Multi-GPU: one process per GPU; every rank runs its own replica (the path has
+no exchange step), times are max-reduced over ranks.  Under torchrun
+WORLD_SIZE must equal --gpus; without torchrun, --gpus N > 1 starts N local
+ranks itself through torch.distributed.run.
 """
 
 from __future__ import annotations
@@ -30,7 +35,11 @@ sys.path.insert(0, ROOT)
 
 from long_context_attention_dca_b200 import workloads as W  # noqa: E402
 
-PREFILL = "llama2_7b_16k"
+PREFILL = "prefill_100k"
+# prefill workloads timed after the step, each reported on its own
+SUB_CONFIGS = ("llama2_70b_32k", "llama2_7b_16k", "tiny")
+# workload of the calls beyond the step (chunked, packed, three passes, ...)
+NEXT_ROWS_WORKLOAD = "llama2_7b_16k"
 DECODE = "decode_b16"
 METRIC = "DCA prefill TFLOP/s (bf16, % of TC peak); decode KV GB/s (% of HBM peak)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -315,9 +324,21 @@ def run_ours(args, rank, world, dev):
     e2e = None if (args.no_e2e or args.only != "all") else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
                                            t_dec, Kc, Vc)
 
+    configs = None
+    if args.configs and args.only == "all":
+        configs = {name: run_config(dca, lib, name, dev, stream, world, tpk)
+                   for name in SUB_CONFIGS if name != args.workload}
+
     next_rows = None
     if args.next_rows and args.only == "all":
-        next_rows = run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc)
+        nc = W.CONFIGS[NEXT_ROWS_WORKLOAD]
+        if args.workload == NEXT_ROWS_WORKLOAD:
+            nQ, nK, nV = Q, K, V
+        else:
+            nQ, nK, nV = W.make_prefill_inputs(nc, device=dev)
+        next_rows = run_next_rows(dca, lib, nc, dc, dev, stream, nQ, nK, nV, t_dec, Kc, Vc)
+        next_rows["workload"] = NEXT_ROWS_WORKLOAD
+        del nQ, nK, nV
 
     line = None
     if rank == 0:
@@ -340,8 +361,9 @@ def run_ours(args, rank, world, dev):
                        "prefill_path": {1: "general (warp MMA)",
                                         2: "tcgen05/TMEM/TMA"}.get(path, str(path)),
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (prefill Q,K,V >= 402 MB; decode KV "
-                             "3.2 GB); no flush"},
+                       "l2": f"inputs larger than L2 (prefill Q,K,V "
+                             f"{(Q.numel() + K.numel() + V.numel()) * 2 / 1e6:.0f} MB; decode "
+                             f"KV {dec_bytes / 1e9:.1f} GB); no flush"},
             "prefill": {"tflops_rope_plus_attn": value / world, "attn_tflops": attn_tflops,
                         "attn_ms": attn_sum / args.steps, "rope_ms": rope_sum / args.steps,
                         "attn_ms_median": statistics.median(attn_ms),
@@ -352,17 +374,20 @@ def run_ours(args, rank, world, dev):
                        "bytes_per_step": dec_bytes, "frac_of_hbm_peak": dec_gbs / world / hbm},
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpk,
                          "unit": "TFLOP/s", "frac": attn_tflops / tpk,
-                         "traffic": traffic.get("prefill_attn"),
+                         "traffic": traffic.get(f"prefill_attn/{args.workload}"),
                          "kernel": "prefill attention", "peak_source": f"{peak_kind} burst"},
             "rooflines": {
                 "decode_split_kv+merge": {"bound": "hbm", "achieved": dec_gbs / world,
                                           "peak": hbm, "unit": "GB/s",
                                           "frac": dec_gbs / world / hbm,
-                                          "traffic": traffic.get("decode")} if do_dec else None,
+                                          "traffic": traffic.get(f"decode/{DECODE}")}
+                if do_dec else None,
                 "prefill_rope": {"bound": "hbm", "achieved": rope_gbs, "peak": hbm,
                                  "unit": "GB/s", "frac": rope_gbs / hbm,
-                                 "traffic": traffic.get("prefill_rope")} if do_pre else None},
+                                 "traffic": traffic.get(f"prefill_rope/{args.workload}")}
+                if do_pre else None},
             "e2e": e2e,
+            "configs": configs,
             "next_rows": next_rows,
             "gpu_launches": (2 * do_pre + 2 * do_dec) * args.steps,
             "clocks": clocks,
@@ -370,6 +395,67 @@ def run_ours(args, rank, world, dev):
             "cpu_baseline": cpu,
         }
     return line
+
+
+def run_config(dca, lib, name, dev, stream, world, tpk):
+    """One prefill workload on its own seeded inputs: fused RoPE then DCA
+    attention through the C ABI, three untimed calls, then `reps` calls timed
+    with CUDA events on the launching stream (RoPE and attention separately).
+    Reports device time, TFLOP/s of RoPE + attention and of the attention
+    kernel alone, and the attention kernel's fraction of the bf16 peak."""
+    import ctypes
+    P = ctypes.c_void_p
+    cfg = W.CONFIGS[name]
+    Q, K, V = W.make_prefill_inputs(cfg, device=dev)
+    B, L, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    s, c, base = cfg["s"], cfg["c"], cfg["base"]
+    wsb = dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    sp = P(stream.cuda_stream)
+
+    def chk(st):
+        if st != 0:
+            raise dca.DcaError(st, dca.dca_last_error_string())
+
+    def rope():
+        chk(lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s, c, base,
+                                 P(ws.data_ptr()), wsb, sp))
+
+    def attn():
+        chk(lib.dca_prefill_attention(P(V.data_ptr()), P(O.data_ptr()), P(LSE.data_ptr()), B, L,
+                                      Hq, Hkv, D, s, c, 0.0, 0, P(ws.data_ptr()), wsb, sp))
+
+    flops = W.prefill_flops(cfg)
+    reps = int(min(50, max(5, 0.2 / max(flops / 1e15, 1e-6))))
+    for _ in range(3):
+        rope(); attn()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    _barrier(world)
+    for e in ev:
+        e[0].record(stream)
+        rope()
+        e[1].record(stream)
+        attn()
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    dca.dca_sync_status(dev)
+    rope_ms = _max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / reps, world, dev)
+    attn_ms = _max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / reps, world, dev)
+    path = dca.dca_prefill_path(L, D, s, c)
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    out = {"tflops_rope_plus_attn": flops / ((rope_ms + attn_ms) * 1e-3) / 1e12,
+           "attn_tflops": attn_tf, "frac_of_peak": attn_tf / tpk,
+           "attn_ms": attn_ms, "rope_ms": rope_ms, "reps": reps, "flops": flops,
+           **_cfg_summary(cfg), "k_boost_frac": cfg.get("k_boost_frac", 0.0),
+           "attn_kernel": {1: "general (warp MMA)", 2: "tcgen05 " + (
+               "two-tile" if D == 128 and s % 256 == 0 else "per-row intervals")}.get(path),
+           "launches_per_call": 2}
+    del Q, K, V, ws, O, LSE
+    return out
 
 
 def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
@@ -387,7 +473,9 @@ def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
     hOd = torch.empty(q_dec.shape, dtype=torch.bfloat16).pin_memory()
     hLd = torch.empty(q_dec.shape[:2], dtype=torch.float32).pin_memory()
     s, c = pc["s"], pc["c"]
-    chunk = args.e2e_chunk
+    # long prompts in 8192-row chunks (2048 CTAs per chunk launch, several
+    # waves of the 148 SMs), shorter ones in 2048-row chunks
+    chunk = args.e2e_chunk or (8192 if pc["L"] > 32768 else 2048)
     ws = torch.empty(dca.dca_attn_prefill_host_workspace(*Q.shape[:3], K.shape[2], Q.shape[3],
                                                          chunk), dtype=torch.uint8, device=dev)
     dws = torch.empty(dca.dca_attn_decode_workspace(*q_dec.shape[:2], q_dec.shape[2],
@@ -762,24 +850,43 @@ def main():
     ap.add_argument("--override-s", type=int, default=0,
                     help="profiling runs: chunk size s of the prefill workload (e.g. 3000, "
                          "whose tiles straddle chunk boundaries)")
-    ap.add_argument("--e2e-chunk", type=int, default=2048,
-                    help="rows per chunk of the host-buffer prefill in the e2e leg")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="rows per chunk of the host-buffer prefill in the e2e leg "
+                         "(0: 8192 above 32k tokens, else 2048)")
+    ap.add_argument("--configs", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the other prefill workloads (70B-, 7B-shaped, tiny)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default=PREFILL, choices=sorted(
         k for k, v in W.CONFIGS.items() if v["kind"] == "prefill" and v["D"] == 128),
-                    help="prefill workload of the step (default: the 7B-shaped one)")
+                    help="prefill workload of the step (default: the 100k-token one)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="launcher and rank plumbing only: gloo process group, barrier and "
+                         "max over ranks, no GPU work (checks --gpus on a CPU host)")
+    ap.add_argument("--launch-timeout", type=float, default=3600.0,
+                    help="seconds before a self-launched multi-rank run is stopped")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    plan, detail = launch_plan(args.gpus, os.environ)
+    if plan == "error":
+        print(f"bench.py: {detail}", file=sys.stderr, flush=True)
+        sys.exit(2)
+    if plan == "spawn":
+        sys.exit(spawn_ranks(args.gpus, args.launch_timeout))
+
+    world = detail
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, rank, world)
+        return
+
+    if args.dry_run:
+        run_dry(args, rank, world)
         return
 
     if world > 1:
@@ -791,6 +898,77 @@ def main():
         line = run_ours(args, rank, world, dev)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+def launch_plan(gpus: int, env) -> tuple:
+    """How this process takes part in a run of `gpus` ranks.
+
+    ("run", world) when it is one of the ranks (no WORLD_SIZE: a single rank;
+    under torchrun WORLD_SIZE must equal --gpus), ("spawn", None) when --gpus
+    asks for more than one rank and no launcher started this process, and
+    ("error", why) on a mismatch, which must not silently run fewer ranks.
+    """
+    if gpus < 1:
+        return "error", f"--gpus must be >= 1, got {gpus}"
+    ws = env.get("WORLD_SIZE")
+    if ws is None:
+        return ("spawn", None) if gpus > 1 else ("run", 1)
+    if int(ws) != gpus:
+        return "error", (f"WORLD_SIZE={ws} (launcher) but --gpus {gpus}: start "
+                         f"{gpus} ranks or pass --gpus {ws}")
+    return "run", int(ws)
+
+
+def spawn_ranks(gpus: int, timeout_s: float) -> int:
+    """Start `gpus` local ranks of this script through torch.distributed.run
+    (rendezvous on 127.0.0.1) and return the launcher's exit code; the whole
+    process group is stopped if it runs past `timeout_s`."""
+    import signal
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port",
+           str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=timeout_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+            proc.wait()
+        print(f"bench.py: {gpus}-rank run stopped after {timeout_s:.0f} s", file=sys.stderr)
+        return 124
+
+
+def run_dry(args, rank, world):
+    """The rank plumbing of a run without GPU work: a gloo process group, the
+    barrier around the timed region and the max over ranks of a per-rank
+    time; rank 0 prints one JSON line naming the ranks that took part."""
+    import datetime
+    if world > 1:
+        torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        cpu = torch.device("cpu")
+        _barrier(world)
+        slowest = _max_over_ranks(float(rank + 1), world, cpu)
+        ranks = [rank]
+        if world > 1:
+            got = [None] * world
+            torch.distributed.all_gather_object(got, rank)
+            ranks = got
+        _barrier(world)
+        if rank == 0:
+            print(json.dumps({"dry_run": True, "n_gpus": world, "ranks": ranks,
+                              "max_over_ranks": slowest, "steps": args.steps,
+                              "warmup": args.warmup}), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
