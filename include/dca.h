@@ -43,6 +43,16 @@
  *     ABI and no kernel traps.
  *   - On a non-DCA_OK return nothing was enqueued; dca_last_error_string()
  *     (per host thread) says why.
+ *   - fp16 range of the prefill paths: every prefill call (one-shot, chunked,
+ *     packed, host-buffer, three-pass, SelfExtend) rounds the rotated queries
+ *     and keys to fp16, the operands of S = Q K^T, for their 11 significant
+ *     bits.  Rotated |values| above 65504 are out of range (as are non-finite
+ *     inputs): the RoPE and key-conversion kernels check every fp16 value
+ *     they write and report a non-finite one through the error word
+ *     (dca_sync_status returns INVALID_ARG); that call's O and LSE are then
+ *     not meaningful.  A rotation keeps each (x_k, x_{k+D/2}) pair's norm, so
+ *     inputs whose pairs have norm <= 65504 are always in range.  Decode and
+ *     dca_rope_rotate keep bf16 operands and have no such limit.
  */
 #ifndef DCA_B200_H
 #define DCA_B200_H
@@ -93,12 +103,15 @@ dca_status_t dca_rope_rotate(const void* x, void* out, int B, int L, int H, int 
 
 /* Workspace bytes needed by dca_attn_prefill / dca_prefill_rope /
  * dca_prefill_attention: the rotated keys Krot [B][L][Hkv][D] and the three
- * query rotations Qrot [3][B][L][Hq][D] (intra, successive, inter), bf16.
+ * query rotations Qrot [3][B][L][Hq][D] (intra, successive, inter), all fp16
+ * (the operands of S = Q K^T; see the fp16 range rule in the conventions).
  * Returns 0 for unsupported arguments. */
 size_t dca_attn_prefill_workspace(int B, int L, int Hq, int Hkv, int D);
 
 /* Step 1 of prefill alone: fused RoPE.  Reads unrotated Q and K once and
- * writes Krot (keys at j mod s) and the three Qrot planes into the workspace.
+ * writes Krot (keys at j mod s) and the three Qrot planes (fp16) into the
+ * workspace.  A rotated value that is not finite in fp16 is reported by
+ * dca_sync_status (INVALID_ARG).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_prefill_rope(const void* Q, const void* K, int B, int L, int Hq, int Hkv,
                               int D, int s, int c, float base, void* workspace,
@@ -425,7 +438,7 @@ dca_status_t dca_kv_append_paged(const void* k_new, const void* v_new, void* Kpo
  *     Nothing in it needs to start at zero.
  *   - Sizes whose scratch (dca_attn_decode_workspace) exceeds 48 MiB return
  *     DCA_ERR_WORKSPACE; the 16-sequence, 64-head, Tcap 65536 decode workload
- *     needs 32.5 MiB.
+ *     needs 16.25 MiB (2048-key splits).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 dca_status_t dca_attn_decode_noalloc(const void* q, const void* Kcache, const void* Vcache,
                                      const int* t, void* O, float* LSE, int B, int Hq, int Hkv,

@@ -344,7 +344,8 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
     return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
-  // Keys 0 .. t0-1 come from the cache (bf16, exact in fp16); the chunk's own
+  // Keys 0 .. t0-1 come from the cache (bf16, exact in fp16 up to 65504;
+  // a larger key is reported by the conversion); the chunk's own
   // keys are rotated here and rounded once, to fp16, like a one-shot prefill.
   void* kf16 = static_cast<char*>(workspace) + align256((size_t)3 * B * Lq * Hq * D * 2);
   cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, kf16, B, Lq, Hq, Hkv, D,
@@ -662,6 +663,10 @@ dca_status_t dca_sync_status(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, fn);
   if (code == kDevTimeout)
     return fail(DCA_ERR_TIMEOUT, "%s: a kernel wait passed its deadline (site %d)", fn, site);
+  if (site >= 106 && site <= 108)
+    return fail(DCA_ERR_INVALID_ARG,
+                "%s: a rotated query or key is not finite in fp16 (|x| > 65504 or a "
+                "non-finite input; site %d)", fn, site);
   return fail(DCA_ERR_INVALID_ARG, "%s: device-side argument check failed (site %d)", fn, site);
 }
 

@@ -8,7 +8,10 @@
 // Angles are formed and range-reduced in fp64, cos/sin evaluated in fp32 on
 // the reduced argument, the rotation done in fp32 and the result
 // rounded to nearest even: bf16 for dca_rope_rotate (a cache in the caller's
-// type), fp16 for the prefill workspace (operands of S = Q K^T only).
+// type), fp16 for the prefill workspace (operands of S = Q K^T only).  An
+// fp16 result that is not finite (a rotated |x| beyond the fp16 range, or a
+// non-finite input) is reported through the device error word as a bad
+// argument; the call's outputs are then not meaningful.
 //
 // Both kernels are HBM-bound.  dca_rope_rotate's kernel: each thread owns one
 // token row and one group of 8 rotation pairs (16 bytes of the first half and
@@ -47,6 +50,22 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// True when either fp16 half of w is infinite or NaN (exponent field all
+// ones): the rotated value left the fp16 range (|x| >= 65520 rounds to
+// infinity) or an input was not finite.
+__device__ __forceinline__ bool f16x2_nonfinite(uint32_t w) {
+  return ((w & 0x7C00u) == 0x7C00u) | ((w & 0x7C000000u) == 0x7C000000u);
+}
+__device__ __forceinline__ bool f16x8_nonfinite(const uint4& v) {
+  return f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) |
+         f16x2_nonfinite(v.w);
+}
+
+// Device error sites of the fp16 range check (reported as a bad argument).
+constexpr int kSiteRopeF16Range = 106;
+constexpr int kSiteKeysF16Range = 107;
+constexpr int kSiteSelfExtendF16Range = 108;
 
 // out_lo = lo*cos - hi*sin, out_hi = hi*cos + lo*sin for 8 pairs; the result
 // is rounded to bf16 (kHalf = false) or fp16 (kHalf = true).
@@ -150,6 +169,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   __shared__ int seq_s[kRopeRows];              // chunk form: sequence (-1: no cache rows)
   __shared__ int pos_s[kRopeRows];              // chunk form: absolute index
   __shared__ long long crow_s[kRopeRows];       // chunk form: cache row (-1: none)
+  __shared__ bool live_s[kRopeRows];            // row belongs to a sequence
   const long long total_rows = (long long)B * L;
   const long long row0 = (long long)blockIdx.x * kRopeRows;
   const int nrows = (int)min((long long)kRopeRows, total_rows - row0);
@@ -159,6 +179,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     int im;
     if (cu_seqlens == nullptr) {
       im = (int)(((row % L) + q_off) % s);
+      live_s[threadIdx.x] = true;
       if constexpr (kChunk) {
         seq_s[threadIdx.x] = (int)(row / L);
         pos_s[threadIdx.x] = (int)(row % L) + q_off;
@@ -175,6 +196,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
         else hi = mid - 1;
       }
       const int a = __ldg(cu_seqlens + lo);
+      live_s[threadIdx.x] = r >= a && r < __ldg(cu_seqlens + lo + 1);
       long long i = max(r - a, 0);
       if constexpr (kChunk) {
         const int e = __ldg(cu_seqlens + lo + 1);
@@ -213,6 +235,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   const int heads = Hq + (kChunk ? 2 : 1) * Hkv;  // [keys | (values) | queries]
   const bool write_kc = Kout != nullptr, write_v = Vc != nullptr;
   const int items = nrows * heads * kGroups;
+  bool bad = false;  // an fp16 output of a row of some sequence is not finite
 #pragma unroll 2
   for (int it = threadIdx.x; it < items; it += kRopeThreads) {
     const int g = it % kGroups;
@@ -253,6 +276,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
           *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
         }
         rotate8<true>(lo, hi, cs, olo, ohi);
+        bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
         const size_t hdst = (((size_t)seq * kh_rows + pos_s[r]) * Hkv + hh) * D + g * 8;
         *reinterpret_cast<uint4*>(Kh + hdst) = olo;
         *reinterpret_cast<uint4*>(Kh + hdst + kHalf) = ohi;
@@ -275,6 +299,9 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     }
     uint4 olo, ohi;
     rotate8<true>(lo, hi, cs, olo, ohi);
+    // each plane is checked: a rotation keeps a pair's norm, not its
+    // largest component, so one angle can overflow where another does not
+    bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
     if (is_k) {
       __half* Krot = static_cast<__half*>(Kout);
       *reinterpret_cast<uint4*>(Krot + off) = olo;
@@ -290,6 +317,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
       cs.s[e] = v.y;
     }
     rotate8<true>(lo, hi, cs, olo, ohi);  // inter plane (c - 1)
+    bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = olo;
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + kHalf) = ohi;
     if (query_pos_for_piece(kSucc, im_s[r], s, c) != c - 1) {
@@ -300,10 +328,12 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
         cs.s[e] = v.y;
       }
       rotate8<true>(lo, hi, cs, olo, ohi);
+      bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
     }
     *reinterpret_cast<uint4*>(Qrot + plane + off) = olo;  // successive plane
     *reinterpret_cast<uint4*>(Qrot + plane + off + kHalf) = ohi;
   }
+  if (bad) report_error(kDevBadArg, kSiteRopeF16Range);
 }
 
 // Decode-time append: rotate the new key of sequence b at t[b] mod s and
@@ -397,6 +427,7 @@ __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restric
     uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
     for (int k = 0; k < 4; ++k) u[k] = pack_f16(bf16_lo(u[k]), bf16_hi(u[k]));
+    if (f16x8_nonfinite(w)) report_error(kDevBadArg, kSiteKeysF16Range);
     Kh[(seq * out_rows + row) * groups_per_row + g] = w;
   }
 }
@@ -431,12 +462,15 @@ __global__ void __launch_bounds__(256) selfextend_rope_kernel(
   uint4 olo, ohi;
   cos_sin_group(i, g * 8, D, log2_base, cs);
   rotate8<true>(lo, hi, cs, olo, ohi);
+  bool bad = f16x8_nonfinite(olo) | f16x8_nonfinite(ohi);
   *reinterpret_cast<uint4*>(dst + off) = olo;
   *reinterpret_cast<uint4*>(dst + off + D / 2) = ohi;
   cos_sin_group(grouped, g * 8, D, log2_base, cs);
   rotate8<true>(lo, hi, cs, olo, ohi);
+  bad |= f16x8_nonfinite(olo) | f16x8_nonfinite(ohi);
   *reinterpret_cast<uint4*>(dst + plane + off) = olo;
   *reinterpret_cast<uint4*>(dst + plane + off + D / 2) = ohi;
+  if (bad) report_error(kDevBadArg, kSiteSelfExtendF16Range);
 }
 
 }  // namespace rope_path

@@ -353,3 +353,63 @@ def test_empty_and_degenerate_sizes():
     O, LSE = dca.dca_attn_prefill(Q, Q[:, :, :1], Q[:, :, :1], 3072, 4096)
     assert O.numel() == 0 and LSE.numel() == 0
     dca.dca_sync_status()
+
+
+# ---------------------------------------------------------------------------
+# fp16 range of the rotated score operands
+# ---------------------------------------------------------------------------
+def _expect_fp16_range_error():
+    with pytest.raises(dca.DcaError) as ei:
+        dca.dca_sync_status()
+    assert ei.value.status == 1 and "fp16" in str(ei.value)
+    dca.dca_sync_status()  # the error word was cleared
+
+
+@pytest.mark.parametrize("where", ["q", "k"])
+def test_prefill_reports_rotated_value_beyond_fp16(where):
+    # one input element of 1e5 rotates (at the intra position 123 mod 192 and
+    # at the others) into a value fp16 cannot hold: reported as a bad
+    # argument, and the context keeps working for the next call
+    cfg = W.scaled(W.CONFIGS["tiny"], L=300, Hq=2, Hkv=1)
+    s, c = cfg["s"], cfg["c"]
+    Q, K, V = W.make_prefill_inputs(cfg, seed=9)
+    X = Q if where == "q" else K
+    X[0, 123, 0, 5] = 1e5
+    dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), s, c)
+    _expect_fp16_range_error()
+    X[0, 123, 0, 5] = 0.5
+    O, LSE = dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), s, c)
+    dca.dca_sync_status()
+    rows = [0, 123, 191, 192, 299]
+    ref = orc.dca_prefill_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V), s, c, rows=rows)
+    pu.assert_close(*pu.compare_rows(O.cpu(), LSE.cpu(), ref), what=f"after {where} overflow")
+
+
+def test_prefill_accepts_pairs_inside_fp16_range():
+    # a pair of norm below 65504 stays finite under every rotation: no report
+    cfg = W.scaled(W.CONFIGS["tiny"], L=300, Hq=2, Hkv=1)
+    Q, K, V = W.make_prefill_inputs(cfg, seed=10)
+    Q[0, 200, 1, 3] = 60000.0
+    K[0, 17, 0, 40] = -60000.0
+    dca.dca_attn_prefill(Q.cuda(), K.cuda(), V.cuda(), cfg["s"], cfg["c"])
+    dca.dca_sync_status()
+
+
+def test_selfextend_reports_rotated_value_beyond_fp16():
+    cfg = W.scaled(W.CONFIGS["tiny"], L=200, Hq=2, Hkv=1)
+    Q, K, V = W.make_prefill_inputs(cfg, seed=11)
+    K[0, 150, 0, 0] = -1e5
+    dca.dca_attn_prefill_selfextend(Q.cuda(), K.cuda(), V.cuda(), 4, 32)
+    _expect_fp16_range_error()
+
+
+def test_chunk_reports_cached_key_beyond_fp16():
+    # a cached bf16 key of 1e5 cannot be converted to the fp16 score operand
+    B, Lq, Hq, Hkv, D, t0, s, c = 1, 64, 2, 1, 64, 256, 192, 256
+    g = torch.Generator().manual_seed(12)
+    mk = lambda *sh: torch.randn(*sh, generator=g).to(torch.bfloat16)
+    Q, K, V = mk(B, Lq, Hq, D), mk(B, Lq, Hkv, D), mk(B, Lq, Hkv, D)
+    Kc, Vc = mk(B, 512, Hkv, D), mk(B, 512, Hkv, D)
+    Kc[0, 100, 0, 7] = 1e5
+    dca.dca_attn_prefill_chunk(Q.cuda(), K.cuda(), V.cuda(), Kc.cuda(), Vc.cuda(), t0, s, c)
+    _expect_fp16_range_error()
