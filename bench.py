@@ -317,8 +317,14 @@ def run_ours(args, rank, world, dev):
 
     peaks, peak_kind = load_peaks()
     traffic = load_traffic()
-    tpk = peaks["bf16_tflops"]
+    tpk = peaks["bf16_tflops"]  # burst: kernels timed alone for a fraction of a second
     hbm = peaks["hbm_gbs"]
+    # The step's attention kernel runs for seconds back to back inside the
+    # timed region (the GPU settles at its power cap), so its roofline takes
+    # the sustained bf16 figure; a short region takes the burst figure.
+    long_region = total_ms > 1000.0
+    tpk_step = peaks.get("bf16_tflops_sustained", tpk) if long_region else tpk
+    step_peak_kind = f"{peak_kind} {'sustained' if long_region else 'burst'}"
 
     # ---- e2e through the public API with host buffers ----
     e2e = None if (args.no_e2e or args.only != "all") else run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec,
@@ -330,13 +336,15 @@ def run_ours(args, rank, world, dev):
                    for name in SUB_CONFIGS if name != args.workload}
 
     next_rows = None
-    if args.next_rows and args.only == "all":
+    select = set(args.next_rows_select.split(",")) if args.next_rows_select else None
+    if args.next_rows and (args.only == "all" or select):
         nc = W.CONFIGS[NEXT_ROWS_WORKLOAD]
         if args.workload == NEXT_ROWS_WORKLOAD:
             nQ, nK, nV = Q, K, V
         else:
             nQ, nK, nV = W.make_prefill_inputs(nc, device=dev)
-        next_rows = run_next_rows(dca, lib, nc, dc, dev, stream, nQ, nK, nV, t_dec, Kc, Vc)
+        next_rows = run_next_rows(dca, lib, nc, dc, dev, stream, nQ, nK, nV, t_dec, Kc, Vc,
+                                  select=select)
         next_rows["workload"] = NEXT_ROWS_WORKLOAD
         del nQ, nK, nV
 
@@ -368,14 +376,16 @@ def run_ours(args, rank, world, dev):
                         "attn_ms": attn_sum / args.steps, "rope_ms": rope_sum / args.steps,
                         "attn_ms_median": statistics.median(attn_ms),
                         "rope_ms_median": statistics.median(rope_ms),
-                        "rope_gbs": rope_gbs, "frac_of_peak": attn_tflops / tpk},
+                        "rope_gbs": rope_gbs, "frac_of_peak": attn_tflops / tpk_step,
+                        "frac_of_burst_peak": attn_tflops / tpk},
             "decode": {"value": dec_gbs, "unit": "GB/s", "ms": dec_sum / args.steps,
                        "ms_median": statistics.median(dec_ms),
                        "bytes_per_step": dec_bytes, "frac_of_hbm_peak": dec_gbs / world / hbm},
-            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpk,
-                         "unit": "TFLOP/s", "frac": attn_tflops / tpk,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": tpk_step,
+                         "unit": "TFLOP/s", "frac": attn_tflops / tpk_step,
                          "traffic": traffic.get(f"prefill_attn/{args.workload}"),
-                         "kernel": "prefill attention", "peak_source": f"{peak_kind} burst"},
+                         "kernel": "prefill attention", "peak_source": step_peak_kind,
+                         "timed_region_ms": total_ms},
             "rooflines": {
                 "decode_split_kv+merge": {"bound": "hbm", "achieved": dec_gbs / world,
                                           "peak": hbm, "unit": "GB/s",
@@ -513,7 +523,7 @@ def run_e2e(dca, pc, dc, dev, args, world, Q, K, V, q_dec, t_dec, Kc, Vc):
                    "dca_attn_decode (decode KV cache device-resident)"}
 
 
-def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3):
+def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3, select=None):
     """Device time of the calls beyond the step, each on the launching stream
     with CUDA events, after one untimed call:
       prefill_chunk  the prefill workload as four equal chunks against a cache
@@ -544,6 +554,9 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
     flops = W.prefill_flops(pc)
     out = {}
 
+    def want(name):
+        return select is None or name in select
+
     def timed(fn, n=reps):
         fn()
         torch.cuda.synchronize(dev)
@@ -558,249 +571,257 @@ def run_next_rows(dca, lib, pc, dc, dev, stream, Q, K, V, t_dec, Kc, Vc, reps=3)
         return a.elapsed_time(b) / n
 
     # chunked prefill
-    n_chunks = 4
-    bounds = [L * k // n_chunks for k in range(n_chunks + 1)]
-    Kcache = torch.empty(B, L, Hkv, D, dtype=torch.bfloat16, device=dev)
-    Vcache = torch.empty_like(Kcache)
-    Qs = [Q[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
-    Ks = [K[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
-    Vs = [V[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
-    wsz = max(dca.dca_attn_prefill_chunk_workspace(B, e - a, Hq, Hkv, D, a)
-              for a, e in zip(bounds[:-1], bounds[1:]))
-    cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    Oc = torch.empty_like(Q)
-    Lc = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
-    Ob = [torch.empty_like(q) for q in Qs]
-    Lb = [torch.empty(B, Hq, q.shape[1], dtype=torch.float32, device=dev) for q in Qs]
+    if want("prefill_chunk"):
+        n_chunks = 4
+        bounds = [L * k // n_chunks for k in range(n_chunks + 1)]
+        Kcache = torch.empty(B, L, Hkv, D, dtype=torch.bfloat16, device=dev)
+        Vcache = torch.empty_like(Kcache)
+        Qs = [Q[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+        Ks = [K[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+        Vs = [V[:, a:e].contiguous() for a, e in zip(bounds[:-1], bounds[1:])]
+        wsz = max(dca.dca_attn_prefill_chunk_workspace(B, e - a, Hq, Hkv, D, a)
+                  for a, e in zip(bounds[:-1], bounds[1:]))
+        cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        Oc = torch.empty_like(Q)
+        Lc = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+        Ob = [torch.empty_like(q) for q in Qs]
+        Lb = [torch.empty(B, Hq, q.shape[1], dtype=torch.float32, device=dev) for q in Qs]
 
-    def chunks():
-        for k, (a, e) in enumerate(zip(bounds[:-1], bounds[1:])):
-            st = lib.dca_attn_prefill_chunk(
-                P(Qs[k].data_ptr()), P(Ks[k].data_ptr()), P(Vs[k].data_ptr()),
-                P(Kcache.data_ptr()), P(Vcache.data_ptr()), P(Ob[k].data_ptr()),
-                P(Lb[k].data_ptr()), B, e - a, Hq, Hkv, D, a, L, s, c, base, 0.0,
-                P(cws.data_ptr()), wsz, P(stream.cuda_stream))
-            if st != 0:
-                raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(chunks)
-    tc = all(a % 256 == 0 for a in bounds[:-1]) and s % 256 == 0 and D == 128
-    out["prefill_chunk"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                            "ms": ms, "chunks": n_chunks,
-                            "path": "tcgen05/TMEM/TMA" if tc else "general (warp MMA)",
-                            "launches_per_call": 3 if tc else 2}
-    del Kcache, Vcache, cws, Oc, Lc, Ob, Lb, Qs, Ks, Vs
+        def chunks():
+            for k, (a, e) in enumerate(zip(bounds[:-1], bounds[1:])):
+                st = lib.dca_attn_prefill_chunk(
+                    P(Qs[k].data_ptr()), P(Ks[k].data_ptr()), P(Vs[k].data_ptr()),
+                    P(Kcache.data_ptr()), P(Vcache.data_ptr()), P(Ob[k].data_ptr()),
+                    P(Lb[k].data_ptr()), B, e - a, Hq, Hkv, D, a, L, s, c, base, 0.0,
+                    P(cws.data_ptr()), wsz, P(stream.cuda_stream))
+                if st != 0:
+                    raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(chunks)
+        tc = all(a % 256 == 0 for a in bounds[:-1]) and s % 256 == 0 and D == 128
+        out["prefill_chunk"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                "ms": ms, "chunks": n_chunks,
+                                "path": "tcgen05/TMEM/TMA" if tc else "general (warp MMA)",
+                                "launches_per_call": 3 if tc else 2}
+        del Kcache, Vcache, cws, Oc, Lc, Ob, Lb, Qs, Ks, Vs
 
     # the general (warp-MMA) kernel on the same workload: the path of every
     # chunking the tcgen05 kernels do not cover (straddling tiles, per-element
     # piece selection)
-    gws = dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
-    gbuf = torch.empty(gws, dtype=torch.uint8, device=dev)
-    Og = torch.empty_like(Q)
-    Lg = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
-    st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s, c, base,
-                              P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
-    if st != 0:
-        raise dca.DcaError(st, dca.dca_last_error_string())
-
-    def general():
-        st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
-                                       Hq, Hkv, D, s, c, 0.0, dca.DCA_PATH_GENERAL,
-                                       P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+    if want("prefill_general_path") or want("prefill_unaligned_s"):
+        gws = dca.dca_attn_prefill_workspace(B, L, Hq, Hkv, D)
+        gbuf = torch.empty(gws, dtype=torch.uint8, device=dev)
+        Og = torch.empty_like(Q)
+        Lg = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+        st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s, c, base,
+                                  P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
         if st != 0:
             raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(general)
-    out["prefill_general_path"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                                   "ms": ms, "path": "general (warp MMA), attention only",
-                                   "launches_per_call": 1}
 
-    # a chunk size that is not a multiple of the 128-row tiles (s = 3000):
-    # tiles straddle chunk boundaries, the per-row-interval tcgen05 kernel
-    s_u = 3000
-    st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s_u, c, base,
-                              P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
-    if st != 0:
-        raise dca.DcaError(st, dca.dca_last_error_string())
+        def general():
+            st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
+                                           Hq, Hkv, D, s, c, 0.0, dca.DCA_PATH_GENERAL,
+                                           P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(general)
+        out["prefill_general_path"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                       "ms": ms, "path": "general (warp MMA), attention only",
+                                       "launches_per_call": 1}
 
-    def unaligned():
-        st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
-                                       Hq, Hkv, D, s_u, c, 0.0, dca.DCA_PATH_AUTO,
-                                       P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+        # a chunk size that is not a multiple of the 128-row tiles (s = 3000):
+        # tiles straddle chunk boundaries, the per-row-interval tcgen05 kernel
+        s_u = 3000
+        st = lib.dca_prefill_rope(P(Q.data_ptr()), P(K.data_ptr()), B, L, Hq, Hkv, D, s_u, c, base,
+                                  P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
         if st != 0:
             raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(unaligned)
-    out["prefill_unaligned_s"] = {
-        "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms, "s": s_u, "c": c,
-        "path": {1: "general (warp MMA)", 2: "tcgen05 per-row intervals"}.get(
-            dca.dca_prefill_path(L, D, s_u, c)), "launches_per_call": 1}
-    del gbuf, Og, Lg
+
+        def unaligned():
+            st = lib.dca_prefill_attention(P(V.data_ptr()), P(Og.data_ptr()), P(Lg.data_ptr()), B, L,
+                                           Hq, Hkv, D, s_u, c, 0.0, dca.DCA_PATH_AUTO,
+                                           P(gbuf.data_ptr()), gws, P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(unaligned)
+        out["prefill_unaligned_s"] = {
+            "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms, "s": s_u, "c": c,
+            "path": {1: "general (warp MMA)", 2: "tcgen05 per-row intervals"}.get(
+                dca.dca_prefill_path(L, D, s_u, c)), "launches_per_call": 1}
+        del gbuf, Og, Lg
 
     # three passes + LSE merge
-    wsz = dca.dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D)
-    pws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    O3 = torch.empty_like(Q)
-    L3 = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    if want("prefill_3pass"):
+        wsz = dca.dca_attn_prefill_3pass_workspace(B, L, Hq, Hkv, D)
+        pws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        O3 = torch.empty_like(Q)
+        L3 = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
 
-    def three():
-        st = lib.dca_attn_prefill_3pass(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
-                                        P(O3.data_ptr()), P(L3.data_ptr()), B, L, Hq, Hkv, D, s,
-                                        c, base, 0.0, P(pws.data_ptr()), wsz,
-                                        P(stream.cuda_stream))
-        if st != 0:
-            raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(three)
-    out["prefill_3pass"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
-                            "path": "general (warp MMA) x3 + merge", "launches_per_call": 5}
-    del pws, O3, L3
+        def three():
+            st = lib.dca_attn_prefill_3pass(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
+                                            P(O3.data_ptr()), P(L3.data_ptr()), B, L, Hq, Hkv, D, s,
+                                            c, base, 0.0, P(pws.data_ptr()), wsz,
+                                            P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(three)
+        out["prefill_3pass"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
+                                "path": "general (warp MMA) x3 + merge", "launches_per_call": 5}
+        del pws, O3, L3
 
     # SelfExtend position map on the general kernel (group 8, window 1024)
-    G_se, W_se = 8, 1024
-    wsz = dca.dca_selfextend_workspace(B, L, Hq, Hkv, D)
-    sws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    Ose = torch.empty_like(Q)
-    Lse = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
+    if want("prefill_selfextend"):
+        G_se, W_se = 8, 1024
+        wsz = dca.dca_selfextend_workspace(B, L, Hq, Hkv, D)
+        sws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        Ose = torch.empty_like(Q)
+        Lse = torch.empty(B, Hq, L, dtype=torch.float32, device=dev)
 
-    def selfextend():
-        st = lib.dca_attn_prefill_selfextend(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
-                                             P(Ose.data_ptr()), P(Lse.data_ptr()), B, L, Hq, Hkv,
-                                             D, G_se, W_se, base, 0.0, P(sws.data_ptr()), wsz,
-                                             P(stream.cuda_stream))
-        if st != 0:
-            raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(selfextend)
-    out["prefill_selfextend"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                                 "ms": ms, "G": G_se, "W": W_se,
-                                 "path": "RoPE (2 planes) + tcgen05 per-row intervals",
-                                 "launches_per_call": 2}
-    del sws, Ose, Lse
+        def selfextend():
+            st = lib.dca_attn_prefill_selfextend(P(Q.data_ptr()), P(K.data_ptr()), P(V.data_ptr()),
+                                                 P(Ose.data_ptr()), P(Lse.data_ptr()), B, L, Hq, Hkv,
+                                                 D, G_se, W_se, base, 0.0, P(sws.data_ptr()), wsz,
+                                                 P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(selfextend)
+        out["prefill_selfextend"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                     "ms": ms, "G": G_se, "W": W_se,
+                                     "path": "RoPE (2 planes) + tcgen05 per-row intervals",
+                                     "launches_per_call": 2}
+        del sws, Ose, Lse
 
     # packed variable-length batch: Llama-2 7B heads, eight prompts of seeded
     # lengths in [512, 16384] back to back (RoPE + attention in one call)
     vc = W.CONFIGS["varlen_7b_mix"]
-    Qv, Kv, Vv, cu, lens = W.make_varlen_inputs(vc, device=dev)
-    cu_d = cu.to(dev)
-    Tv, Hqv, Dv = Qv.shape
-    Hkvv = Kv.shape[1]
-    wsz = dca.dca_attn_prefill_varlen_workspace(Tv, Hqv, Hkvv, Dv)
-    vws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    Ov = torch.empty_like(Qv)
-    Lv = torch.empty(Hqv, Tv, dtype=torch.float32, device=dev)
+    Hqv, Hkvv, Dv = vc["Hq"], vc["Hkv"], vc["D"]
+    if want("prefill_varlen"):
+        Qv, Kv, Vv, cu, lens = W.make_varlen_inputs(vc, device=dev)
+        cu_d = cu.to(dev)
+        Tv = Qv.shape[0]
+        wsz = dca.dca_attn_prefill_varlen_workspace(Tv, Hqv, Hkvv, Dv)
+        vws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        Ov = torch.empty_like(Qv)
+        Lv = torch.empty(Hqv, Tv, dtype=torch.float32, device=dev)
 
-    def varlen():
-        st = lib.dca_attn_prefill_varlen(P(Qv.data_ptr()), P(Kv.data_ptr()), P(Vv.data_ptr()),
-                                         P(Ov.data_ptr()), P(Lv.data_ptr()), P(cu_d.data_ptr()),
-                                         len(lens), max(lens), Tv, Hqv, Hkvv, Dv, vc["s"],
-                                         vc["c"], vc["base"], 0.0, P(vws.data_ptr()), wsz,
-                                         P(stream.cuda_stream))
-        if st != 0:
-            raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(varlen)
-    out["prefill_varlen"] = {
-        "value": W.varlen_flops(lens, Hqv, Dv) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-        "ms": ms, "workload": "varlen_7b_mix", "lens": lens, "T": Tv,
-        "path": "RoPE + tcgen05 " + ("two-tile" if Dv == 128 and vc["s"] % 256 == 0
-                                     else "per-row intervals"),
-        "launches_per_call": 2}
-    del Qv, Kv, Vv, vws, Ov, Lv
+        def varlen():
+            st = lib.dca_attn_prefill_varlen(P(Qv.data_ptr()), P(Kv.data_ptr()), P(Vv.data_ptr()),
+                                             P(Ov.data_ptr()), P(Lv.data_ptr()), P(cu_d.data_ptr()),
+                                             len(lens), max(lens), Tv, Hqv, Hkvv, Dv, vc["s"],
+                                             vc["c"], vc["base"], 0.0, P(vws.data_ptr()), wsz,
+                                             P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(varlen)
+        out["prefill_varlen"] = {
+            "value": W.varlen_flops(lens, Hqv, Dv) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms": ms, "workload": "varlen_7b_mix", "lens": lens, "T": Tv,
+            "path": "RoPE + tcgen05 " + ("two-tile" if Dv == 128 and vc["s"] % 256 == 0
+                                         else "per-row intervals"),
+            "launches_per_call": 2}
+        del Qv, Kv, Vv, vws, Ov, Lv
 
     # packed chunks over per-sequence caches: Llama-2 7B heads, eight
     # sequences with seeded 0 .. 14000 cached tokens and new chunks of
     # 256 .. 2048 tokens (RoPE, cache writes, key conversion and attention)
-    rng = np.random.default_rng(7)
-    t0c = [int(x) for x in rng.integers(0, 14001, 8)]
-    lensc = [int(x) for x in rng.integers(256, 2049, 8)]
-    Tc, Tcap_c = sum(lensc), 16384
-    gen_c = torch.Generator(device=dev)
-    gen_c.manual_seed(7)
-    Qc = torch.randn(Tc, Hqv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
-    Kn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
-    Vn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
-    Kcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
-    Vcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
-    cu_c = torch.zeros(9, dtype=torch.int32)
-    cu_c[1:] = torch.cumsum(torch.tensor(lensc), 0).to(torch.int32)
-    cu_c, t0_d = cu_c.to(dev), torch.tensor(t0c, dtype=torch.int32, device=dev)
-    max_kv = max(a + n for a, n in zip(t0c, lensc))
-    wsz = dca.dca_attn_prefill_varlen_chunk_workspace(8, Tc, max_kv, Hqv, Hkvv, Dv)
-    cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    Occ = torch.empty_like(Qc)
-    Lcc = torch.empty(Hqv, Tc, dtype=torch.float32, device=dev)
+    if want("prefill_varlen_chunk"):
+        rng = np.random.default_rng(7)
+        t0c = [int(x) for x in rng.integers(0, 14001, 8)]
+        lensc = [int(x) for x in rng.integers(256, 2049, 8)]
+        Tc, Tcap_c = sum(lensc), 16384
+        gen_c = torch.Generator(device=dev)
+        gen_c.manual_seed(7)
+        Qc = torch.randn(Tc, Hqv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+        Kn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+        Vn = torch.randn(Tc, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+        Kcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+        Vcc = torch.randn(8, Tcap_c, Hkvv, Dv, generator=gen_c, device=dev).to(torch.bfloat16)
+        cu_c = torch.zeros(9, dtype=torch.int32)
+        cu_c[1:] = torch.cumsum(torch.tensor(lensc), 0).to(torch.int32)
+        cu_c, t0_d = cu_c.to(dev), torch.tensor(t0c, dtype=torch.int32, device=dev)
+        max_kv = max(a + n for a, n in zip(t0c, lensc))
+        wsz = dca.dca_attn_prefill_varlen_chunk_workspace(8, Tc, max_kv, Hqv, Hkvv, Dv)
+        cws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        Occ = torch.empty_like(Qc)
+        Lcc = torch.empty(Hqv, Tc, dtype=torch.float32, device=dev)
 
-    def varlen_chunk():
-        st = lib.dca_attn_prefill_varlen_chunk(
-            P(Qc.data_ptr()), P(Kn.data_ptr()), P(Vn.data_ptr()), P(Kcc.data_ptr()),
-            P(Vcc.data_ptr()), P(Occ.data_ptr()), P(Lcc.data_ptr()), P(cu_c.data_ptr()),
-            P(t0_d.data_ptr()), 8, max(lensc), Tc, max_kv, Hqv, Hkvv, Dv, Tcap_c, vc["s"],
-            vc["c"], vc["base"], 0.0, P(cws.data_ptr()), wsz, P(stream.cuda_stream))
-        if st != 0:
-            raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(varlen_chunk)
-    out["prefill_varlen_chunk"] = {
-        "value": W.varlen_chunk_flops(t0c, lensc, Hqv, Dv) / (ms * 1e-3) / 1e12,
-        "unit": "TFLOP/s", "ms": ms, "t0": t0c, "lens": lensc,
-        "path": "chunk RoPE + key conversion + tcgen05 per-row intervals",
-        "launches_per_call": 3}
-    del Qc, Kn, Vn, Kcc, Vcc, cws, Occ, Lcc
+        def varlen_chunk():
+            st = lib.dca_attn_prefill_varlen_chunk(
+                P(Qc.data_ptr()), P(Kn.data_ptr()), P(Vn.data_ptr()), P(Kcc.data_ptr()),
+                P(Vcc.data_ptr()), P(Occ.data_ptr()), P(Lcc.data_ptr()), P(cu_c.data_ptr()),
+                P(t0_d.data_ptr()), 8, max(lensc), Tc, max_kv, Hqv, Hkvv, Dv, Tcap_c, vc["s"],
+                vc["c"], vc["base"], 0.0, P(cws.data_ptr()), wsz, P(stream.cuda_stream))
+            if st != 0:
+                raise dca.DcaError(st, dca.dca_last_error_string())
+        ms = timed(varlen_chunk)
+        out["prefill_varlen_chunk"] = {
+            "value": W.varlen_chunk_flops(t0c, lensc, Hqv, Dv) / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "ms": ms, "t0": t0c, "lens": lensc,
+            "path": "chunk RoPE + key conversion + tcgen05 per-row intervals",
+            "launches_per_call": 3}
+        del Qc, Kn, Vn, Kcc, Vcc, cws, Occ, Lcc
 
     # decode over a paged cache: the decode workload's caches scattered into
     # 256-row blocks in a seeded random physical order
-    Bd, Tcap, Hkvd, Dd = Kc.shape
-    rows = 256
-    nb = Tcap // rows
-    gperm = torch.Generator().manual_seed(0)
-    perm = torch.randperm(Bd * nb, generator=gperm).to(dev)
-    Kp = torch.empty(Bd * nb, rows, Hkvd, Dd, dtype=Kc.dtype, device=dev)
-    Vp = torch.empty_like(Kp)
-    Kp[perm] = Kc.view(Bd * nb, rows, Hkvd, Dd)
-    Vp[perm] = Vc.view(Bd * nb, rows, Hkvd, Dd)
-    table = perm.view(Bd, nb).to(torch.int32)
-    qd = torch.randn(Bd, dc["Hq"], Dd, device=dev).to(torch.bfloat16)
-    pws = torch.empty(dca.dca_attn_decode_workspace(Bd, dc["Hq"], Dd, Tcap), dtype=torch.uint8,
-                      device=dev)
-    Opg = torch.empty_like(qd)
-    Lpg = torch.empty(Bd, dc["Hq"], dtype=torch.float32, device=dev)
+    if want("decode_paged"):
+        Bd, Tcap, Hkvd, Dd = Kc.shape
+        rows = 256
+        nb = Tcap // rows
+        gperm = torch.Generator().manual_seed(0)
+        perm = torch.randperm(Bd * nb, generator=gperm).to(dev)
+        Kp = torch.empty(Bd * nb, rows, Hkvd, Dd, dtype=Kc.dtype, device=dev)
+        Vp = torch.empty_like(Kp)
+        Kp[perm] = Kc.view(Bd * nb, rows, Hkvd, Dd)
+        Vp[perm] = Vc.view(Bd * nb, rows, Hkvd, Dd)
+        table = perm.view(Bd, nb).to(torch.int32)
+        qd = torch.randn(Bd, dc["Hq"], Dd, device=dev).to(torch.bfloat16)
+        pws = torch.empty(dca.dca_attn_decode_workspace(Bd, dc["Hq"], Dd, Tcap), dtype=torch.uint8,
+                          device=dev)
+        Opg = torch.empty_like(qd)
+        Lpg = torch.empty(Bd, dc["Hq"], dtype=torch.float32, device=dev)
 
-    def paged():
-        st = lib.dca_attn_decode_paged(P(qd.data_ptr()), P(Kp.data_ptr()), P(Vp.data_ptr()),
-                                       P(table.data_ptr()), nb, rows, Bd * nb,
-                                       P(t_dec.data_ptr()), P(Opg.data_ptr()), P(Lpg.data_ptr()),
-                                       Bd, dc["Hq"], Hkvd, Dd, dc["s"], dc["c"], dc["base"], 0.0,
-                                       P(pws.data_ptr()), pws.numel(), P(stream.cuda_stream))
-        if st != 0:
-            raise dca.DcaError(st, dca.dca_last_error_string())
-    ms = timed(paged, 10)
-    dbytes = W.decode_bytes(dc, t_dec.cpu().tolist())
-    out["decode_paged"] = {"value": dbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms": ms,
-                           "block_rows": rows, "launches_per_call": 2}
-    del Kp, Vp, pws
-
-    # decode-time append of one token per sequence (positions t_dec + 1 < Tcap)
-    Bd, Tcap, Hkvd, Dd = Kc.shape
-    kn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
-    vn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
-    t_app = torch.clamp(t_dec + 1, max=Tcap - 1).to(torch.int32)
-    Kc2, Vc2 = Kc.clone(), Vc.clone()  # the step's caches stay as they are
-
-    def append(strm):
-        for _ in range(100):
-            st = lib.dca_kv_append(P(kn.data_ptr()), P(vn.data_ptr()), P(Kc2.data_ptr()),
-                                   P(Vc2.data_ptr()), P(t_app.data_ptr()), Bd, Hkvd, Dd, Tcap,
-                                   dc["s"], dc["c"], dc["base"], P(strm.cuda_stream))
+        def paged():
+            st = lib.dca_attn_decode_paged(P(qd.data_ptr()), P(Kp.data_ptr()), P(Vp.data_ptr()),
+                                           P(table.data_ptr()), nb, rows, Bd * nb,
+                                           P(t_dec.data_ptr()), P(Opg.data_ptr()), P(Lpg.data_ptr()),
+                                           Bd, dc["Hq"], Hkvd, Dd, dc["s"], dc["c"], dc["base"], 0.0,
+                                           P(pws.data_ptr()), pws.numel(), P(stream.cuda_stream))
             if st != 0:
                 raise dca.DcaError(st, dca.dca_last_error_string())
-    ms_stream = timed(lambda: append(stream), 1) / 100
-    # the same 100 appends replayed from a CUDA graph (no host launch overhead)
-    side = torch.cuda.Stream(dev)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=side):
-        append(side)
-    ms_graph = timed(graph.replay, 1) / 100
-    del graph
-    nbytes = Bd * Hkvd * Dd * 2 * 4  # read k, v; write the two cache rows
-    out["kv_append"] = {"us_per_call": ms_graph * 1e3, "us_per_call_stream": ms_stream * 1e3,
-                        "bytes_per_call": nbytes, "timing": "100 appends in a CUDA graph",
-                        "bound": "launch latency (a few hundred KB per call)",
-                        "launches_per_call": 1}
-    del Kc2, Vc2
+        ms = timed(paged, 10)
+        dbytes = W.decode_bytes(dc, t_dec.cpu().tolist())
+        out["decode_paged"] = {"value": dbytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms": ms,
+                               "block_rows": rows, "launches_per_call": 2}
+        del Kp, Vp, pws
+
+    # decode-time append of one token per sequence (positions t_dec + 1 < Tcap)
+    if want("kv_append"):
+        Bd, Tcap, Hkvd, Dd = Kc.shape
+        kn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
+        vn = torch.randn(Bd, Hkvd, Dd, device=dev).to(torch.bfloat16)
+        t_app = torch.clamp(t_dec + 1, max=Tcap - 1).to(torch.int32)
+        Kc2, Vc2 = Kc.clone(), Vc.clone()  # the step's caches stay as they are
+
+        def append(strm):
+            for _ in range(100):
+                st = lib.dca_kv_append(P(kn.data_ptr()), P(vn.data_ptr()), P(Kc2.data_ptr()),
+                                       P(Vc2.data_ptr()), P(t_app.data_ptr()), Bd, Hkvd, Dd, Tcap,
+                                       dc["s"], dc["c"], dc["base"], P(strm.cuda_stream))
+                if st != 0:
+                    raise dca.DcaError(st, dca.dca_last_error_string())
+        ms_stream = timed(lambda: append(stream), 1) / 100
+        # the same 100 appends replayed from a CUDA graph (no host launch overhead)
+        side = torch.cuda.Stream(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            append(side)
+        ms_graph = timed(graph.replay, 1) / 100
+        del graph
+        nbytes = Bd * Hkvd * Dd * 2 * 4  # read k, v; write the two cache rows
+        out["kv_append"] = {"us_per_call": ms_graph * 1e3, "us_per_call_stream": ms_stream * 1e3,
+                            "bytes_per_call": nbytes, "timing": "100 appends in a CUDA graph",
+                            "bound": "launch latency (a few hundred KB per call)",
+                            "launches_per_call": 1}
+        del Kc2, Vc2
     return out
 
 
@@ -847,6 +868,9 @@ def main():
     ap.add_argument("--next-rows", action=argparse.BooleanOptionalAction, default=True,
                     help="also time chunked prefill, the 3-pass variant and KV append "
                          "(outside the timed step)")
+    ap.add_argument("--next-rows-select", default="",
+                    help="profiling runs: comma-separated names of the calls beyond the step "
+                         "to time (e.g. prefill_varlen_chunk); runs them with --only prefill too")
     ap.add_argument("--override-s", type=int, default=0,
                     help="profiling runs: chunk size s of the prefill workload (e.g. 3000, "
                          "whose tiles straddle chunk boundaries)")
