@@ -273,6 +273,38 @@ dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const v
                                            float scale, void* workspace, size_t ws_bytes,
                                            void* stream);
 
+/* Workspace bytes for dca_attn_prefill_varlen_chunk_mirror: the fp16 query
+ * rotations [3][T][Hq][D] and the attention's work order (B * ceil(T / 256)
+ * ints), each rounded up to 256 bytes.  Returns 0 for unsupported arguments. */
+size_t dca_attn_prefill_varlen_chunk_mirror_workspace(int B, int T, int Hq, int Hkv, int D);
+
+/* dca_attn_prefill_varlen_chunk with a caller-owned fp16 copy of the rotated
+ * keys, kept across calls, so that no call converts the cached prefix again.
+ * dca_attn_prefill_varlen_chunk rounds the cached bf16 keys 0 .. t0[b]-1 to
+ * fp16 (the S = Q K^T operand format) on every call, so a long prompt fed
+ * in many chunks moves its prefix again each time (traffic quadratic in the
+ * prompt length).  Here:
+ *   Kf16 [B][Tcap][Hkv][D] fp16, owned by the caller: rows 0 .. t0[b]-1 of
+ *     entry b must hold what earlier calls of this entry point wrote there
+ *     for sequence b (a sequence fed through it from its first chunk, t0 = 0);
+ *     this call writes the new keys' fp16 rotation to rows t0[b] .. t0[b]+n_b-1
+ *     (one rounding from the fp32 rotation, as in a one-shot prefill, so the
+ *     cached keys are as precise as the ones of dca_attn_prefill).
+ *   Everything else (arguments, Kcache / Vcache rows written, the value tail
+ *     zeroed to the next multiple of 128, offsets checked on the device,
+ *     results) as dca_attn_prefill_varlen_chunk.  Contiguous caches only.
+ * Source: as dca_attn_prefill_varlen_chunk (Guide, "Strategic
+ * Recommendations", item 1: a drop-in wrapper for chunked serving).
+ * D in {64, 128}.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+dca_status_t dca_attn_prefill_varlen_chunk_mirror(const void* Q, const void* K, const void* V,
+                                                  void* Kcache, void* Vcache, void* Kf16,
+                                                  void* O, float* LSE, const int* cu_seqlens,
+                                                  const int* t0, int B, int max_seqlen, int T,
+                                                  int max_kv, int Hq, int Hkv, int D, int Tcap,
+                                                  int s, int c, float base, float scale,
+                                                  void* workspace, size_t ws_bytes,
+                                                  void* stream);
+
 /* dca_attn_prefill_varlen_chunk over paged caches: Kpool, Vpool
  * [num_blocks][block_rows][Hkv][D] bf16; position p of sequence b lives in
  * row p % block_rows of block block_table[b][p / block_rows] (block_table

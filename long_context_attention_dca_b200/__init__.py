@@ -28,6 +28,7 @@ __all__ = [
     "dca_attn_prefill_varlen_workspace", "dca_attn_prefill_varlen",
     "dca_attn_prefill_varlen_chunk_workspace", "dca_attn_prefill_varlen_chunk",
     "dca_attn_prefill_varlen_chunk_paged",
+    "dca_attn_prefill_varlen_chunk_mirror_workspace", "dca_attn_prefill_varlen_chunk_mirror",
     "dca_selfextend_workspace", "dca_attn_prefill_selfextend",
     "dca_attn_prefill_host_workspace", "dca_attn_prefill_host",
     "dca_attn_decode_paged", "dca_kv_append_paged",
@@ -58,6 +59,10 @@ _SIGS = {
     "dca_attn_prefill_varlen_chunk_workspace": (_Z, [_I, _I, _I, _I, _I, _I]),
     "dca_attn_prefill_varlen_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
                                            _I, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
+    "dca_attn_prefill_varlen_chunk_mirror_workspace": (_Z, [_I, _I, _I, _I, _I]),
+    "dca_attn_prefill_varlen_chunk_mirror": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
+                                                  _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F,
+                                                  _P, _Z, _P]),
     "dca_attn_prefill_varlen_chunk_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P,
                                                  _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F,
                                                  _P, _Z, _P]),
@@ -289,6 +294,43 @@ def dca_attn_prefill_varlen_chunk(Q, K, V, Kcache, Vcache, cu_seqlens, t0, max_s
         base, scale, _ptr(ws), ws.numel(), _stream(Q)))
     return O, LSE
 
+
+
+def dca_attn_prefill_varlen_chunk_mirror_workspace(B: int, T: int, Hq: int, Hkv: int,
+                                                   D: int) -> int:
+    return lib().dca_attn_prefill_varlen_chunk_mirror_workspace(B, T, Hq, Hkv, D)
+
+
+def dca_attn_prefill_varlen_chunk_mirror(Q, K, V, Kcache, Vcache, Kf16, cu_seqlens, t0,
+                                         max_seqlen, max_kv, s, c, base=10000.0, scale=0.0,
+                                         workspace=None, O=None, LSE=None):
+    """As dca_attn_prefill_varlen_chunk, with Kf16 [B, Tcap, Hkv, D] fp16: the
+    caller's fp16 copy of the rotated keys, read for rows 0 .. t0[b]-1 and
+    extended by this call's new rows (see dca.h)."""
+    _need(Q, "Q", torch.bfloat16, 3)
+    _need(K, "K", torch.bfloat16, 3)
+    _need(V, "V", torch.bfloat16, 3)
+    _need(Kcache, "Kcache", torch.bfloat16, 4)
+    _need(Vcache, "Vcache", torch.bfloat16, 4)
+    _need(Kf16, "Kf16", torch.float16, 4)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    _need(t0, "t0", torch.int32, 1)
+    T, Hq, D = Q.shape
+    Hkv = K.shape[1]
+    B, Tcap = Kcache.shape[:2]
+    if tuple(Kf16.shape) != tuple(Kcache.shape):
+        raise DcaError(1, "Kf16 must have the shape of Kcache")
+    nbytes = dca_attn_prefill_varlen_chunk_mirror_workspace(B, T, Hq, Hkv, D)
+    ws = _workspace(nbytes, Q.device) if workspace is None else workspace
+    O = torch.empty_like(Q) if O is None else O
+    LSE = torch.empty((Hq, T), dtype=torch.float32, device=Q.device) if LSE is None else LSE
+    _need(O, "O", torch.bfloat16, 3)
+    _need(LSE, "LSE", torch.float32, 2)
+    _check(lib().dca_attn_prefill_varlen_chunk_mirror(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(Kcache), _ptr(Vcache), _ptr(Kf16), _ptr(O), _ptr(LSE),
+        _ptr(cu_seqlens), _ptr(t0), B, int(max_seqlen), T, int(max_kv), Hq, Hkv, D, Tcap, s, c,
+        base, scale, _ptr(ws), ws.numel(), _stream(Q)))
+    return O, LSE
 
 def dca_attn_prefill_varlen_chunk_paged(Q, K, V, Kpool, Vpool, block_table, cu_seqlens, t0,
                                         max_seqlen, max_kv, s, c, base=10000.0, scale=0.0,

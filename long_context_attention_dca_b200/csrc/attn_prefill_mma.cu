@@ -86,22 +86,6 @@ struct DcaRule {
   }
 };
 
-struct SelfExtendRule {
-  // pieces 0 neighbour (i - j < W), 1 grouped: query plane p with key plane p
-  static constexpr int kPieces = 2, kQPlanes = 2, kKPlanes = 2;
-  static constexpr bool kDca = false;
-  int W;
-  __device__ __forceinline__ int kplane(int p) const { return p; }
-  __device__ __forceinline__ void meets(int r0, int k0, bool (&pr)[3]) const {
-    // distances i - j in the tile span [r0 - k0 - (kBN - 1), r0 + 15 - k0]
-    pr[0] = max(r0 - k0 - (kBN - 1), 0) < W;
-    pr[1] = r0 + 15 - k0 >= W;
-    pr[2] = false;
-  }
-  __device__ __forceinline__ int row_key(int i) const { return i; }
-  __device__ __forceinline__ int piece(int rk, int j) const { return rk - j < W ? 0 : 1; }
-};
-
 // Query row r of this launch has absolute index q_off + r (0 for a whole-
 // sequence prefill; the chunk start for chunked prefill against a cache).
 // Keys 0 .. Lkv-1 are read from fp16 K and bf16 V rows of pitch k_rows and
@@ -382,19 +366,6 @@ cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, co
                           k_rows, v_rows, stream);
   return launch_mma<128>(Qrot, Kf16, V, O, LSE, B, Lq, Hq, Hkv, rule, scale, 7, nullptr, t0,
                          k_rows, v_rows, stream);
-}
-
-cudaError_t launch_prefill_attn_selfextend(const void* Qse, const void* Kse, const void* V,
-                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
-                                           int D, int W, float scale, cudaStream_t stream) {
-  using namespace mma_path;
-  if (L == 0 || B == 0 || Hq == 0) return cudaSuccess;
-  const SelfExtendRule rule{W};
-  if (D == 64)
-    return launch_mma<64>(Qse, Kse, V, O, LSE, B, L, Hq, Hkv, rule, scale, 3, nullptr, 0, L, L,
-                          stream);
-  return launch_mma<128>(Qse, Kse, V, O, LSE, B, L, Hq, Hkv, rule, scale, 3, nullptr, 0, L, L,
-                         stream);
 }
 
 // Combine the three single-piece passes: O = sum_p e^{LSE_p - LSE} O_p with

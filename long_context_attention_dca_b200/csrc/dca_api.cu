@@ -374,6 +374,11 @@ size_t dca_attn_prefill_varlen_chunk_workspace(int B, int T, int max_kv, int Hq,
          align256((size_t)B * varlen_pair_slots(T) * 4);
 }
 
+size_t dca_attn_prefill_varlen_chunk_mirror_workspace(int B, int T, int Hq, int Hkv, int D) {
+  if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (D != 64 && D != 128)) return 0;
+  return align256((size_t)3 * T * Hq * D * 2) + align256((size_t)B * varlen_pair_slots(T) * 4);
+}
+
 }  // extern "C"
 
 namespace {
@@ -447,6 +452,55 @@ dca_status_t dca_attn_prefill_varlen_chunk(const void* Q, const void* K, const v
                            base, scale, workspace, ws_bytes, stream, nullptr, 0, 0, 0);
 }
 
+dca_status_t dca_attn_prefill_varlen_chunk_mirror(
+    const void* Q, const void* K, const void* V, void* Kcache, void* Vcache, void* Kf16, void* O,
+    float* LSE, const int* cu_seqlens, const int* t0, int B, int max_seqlen, int T, int max_kv,
+    int Hq, int Hkv, int D, int Tcap, int s, int c, float base, float scale, void* workspace,
+    size_t ws_bytes, void* stream) {
+  const char* fn = "dca_attn_prefill_varlen_chunk_mirror";
+  dca_status_t st = check_heads(fn, B, max_seqlen, Hq, Hkv, D);
+  if (st == DCA_OK) st = check_chunking(fn, s, c, base);
+  if (st != DCA_OK) return st;
+  if (T < 0) return fail(DCA_ERR_INVALID_ARG, "%s: T=%d", fn, T);
+  if (max_seqlen > T) max_seqlen = T;
+  if (Tcap < 1 || max_kv < 1 || max_kv > Tcap)
+    return fail(DCA_ERR_INVALID_ARG, "%s: need 1 <= max_kv=%d <= Tcap=%d", fn, max_kv, Tcap);
+  if ((long long)B * max_seqlen == 0 || T == 0) return DCA_OK;
+  DCA_CHECK_PTR(Q);
+  DCA_CHECK_PTR(K);
+  DCA_CHECK_PTR(V);
+  DCA_CHECK_PTR(Kcache);
+  DCA_CHECK_PTR(Vcache);
+  DCA_CHECK_PTR(Kf16);
+  DCA_CHECK_PTR(O);
+  DCA_CHECK_PTR(LSE);
+  if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+      t0 == nullptr || (reinterpret_cast<uintptr_t>(t0) & 3u))
+    return fail(DCA_ERR_INVALID_ARG, "%s: cu_seqlens / t0 null or not 4-byte aligned", fn);
+  DCA_CHECK_PTR(workspace);
+  const size_t need = dca_attn_prefill_varlen_chunk_mirror_workspace(B, T, Hq, Hkv, D);
+  if (ws_bytes < need)
+    return fail(DCA_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", fn, ws_bytes, need);
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  // The new keys are rotated once: to bf16 in Kcache and, rounded once, to
+  // fp16 in the caller's mirror, at rows t0[b] .. t0[b]+n_b-1 of entry b.
+  // Earlier rows are read from the mirror as earlier calls left them: no key
+  // is converted, so a call moves bytes in proportion to its new rows (plus
+  // the attention's reads).
+  int* order = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                      align256((size_t)3 * T * Hq * D * 2));
+  cudaError_t e = launch_chunk_rope(Q, K, V, workspace, Kcache, Vcache, Kf16, 1, T, Hq, Hkv, D,
+                                    0, Tcap, Tcap, s, c, base, strm, cu_seqlens, B, t0);
+  if (e == cudaSuccess)
+    e = launch_value_tail_zero(Vcache, B, Tcap, max_kv, Hkv, D, t0, cu_seqlens, strm);
+  if (e == cudaSuccess)
+    e = launch_prefill_attn_sm100_gen(workspace, Kf16, Vcache, O, LSE, B, max_seqlen, Hq, Hkv, D,
+                                      s, sc, strm, 0, Tcap, Tcap, cu_seqlens, T, t0, max_kv,
+                                      nullptr, 0, 0, 0, order);
+  return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
+}
+
 dca_status_t dca_attn_prefill_varlen_chunk_paged(
     const void* Q, const void* K, const void* V, void* Kpool, void* Vpool,
     const int* block_table, int max_blocks, int block_rows, int num_blocks, void* O, float* LSE,
@@ -499,14 +553,9 @@ dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const voi
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_selfextend_rope(Q, K, workspace, kse, B, L, Hq, Hkv, D, G, W, base, strm);
-  if (e == cudaSuccess) {
-    if (auto_path(D, W) == DCA_PATH_TCGEN05)
-      e = launch_prefill_attn_sm100_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc,
-                                               strm);
-    else
-      e = launch_prefill_attn_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc,
-                                         strm);
-  }
+  if (e == cudaSuccess)
+    e = launch_prefill_attn_sm100_selfextend(workspace, kse, V, O, LSE, B, L, Hq, Hkv, D, W, sc,
+                                             strm);
   return e == cudaSuccess ? DCA_OK : cuda_fail(e, fn);
 }
 

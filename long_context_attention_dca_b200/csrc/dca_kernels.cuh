@@ -47,14 +47,11 @@ cudaError_t launch_prefill_attn_mma_chunk(const void* Qrot, const void* Kf16, co
                                           int v_rows, cudaStream_t stream);
 
 // SelfExtend (prior-art position map): Qse [2][B][L][Hq][D] and Kse
-// [2][B][L][Hkv][D] fp16 (neighbour, grouped rotations), then the general
-// kernel with the neighbour / grouped rule.
+// [2][B][L][Hkv][D] fp16 (neighbour, grouped rotations), read by the
+// per-row-interval tcgen05 kernel with the neighbour / grouped rule.
 cudaError_t launch_selfextend_rope(const void* Q, const void* K, void* Qse, void* Kse, int B,
                                    int L, int Hq, int Hkv, int D, int G, int W, float base,
                                    cudaStream_t stream);
-cudaError_t launch_prefill_attn_selfextend(const void* Qse, const void* Kse, const void* V,
-                                           void* O, float* LSE, int B, int L, int Hq, int Hkv,
-                                           int D, int W, float scale, cudaStream_t stream);
 
 // General prefill attention (warp MMA; any s, D in {64, 128}).  piece_mask
 // selects the pieces the softmax covers (1 intra, 2 successive, 4 inter; 7 =
@@ -111,6 +108,11 @@ cudaError_t launch_keys_to_f16(const void* Kcache, void* Kf16, int B, int rows, 
                                const int* t0s = nullptr, const int* cu_seqlens = nullptr,
                                void* Vcache = nullptr, const int* block_table = nullptr,
                                int max_blocks = 0, int block_rows = 0, int num_blocks = 0);
+
+// Zero value-cache rows e .. min(e rounded up to 128, kv_rows)-1 of every
+// sequence b of a packed chunk (e = t0[b] + its length; contiguous caches).
+cudaError_t launch_value_tail_zero(void* Vcache, int B, int Tcap, int kv_rows, int Hkv, int D,
+                                   const int* t0s, const int* cu_seqlens, cudaStream_t stream);
 
 // Decode-time append of one token per sequence into pre-rotated caches:
 // contiguous [B][Tcap][Hkv][D] (block_table null) or a paged pool

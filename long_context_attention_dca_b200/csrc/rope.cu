@@ -432,6 +432,31 @@ __global__ void __launch_bounds__(256) keys_to_f16_kernel(const uint4* __restric
   }
 }
 
+// Value rows e .. min(e rounded up to 128, kv_rows)-1 of each sequence b,
+// e = t0[b] + its chunk length, set to zero (contiguous caches [B][Tcap][H][D]):
+// rows the sequence does not have yet, read with zero weight by its last key
+// tile (zero keeps 0 * value finite).  One 16-byte group per thread over
+// (sequence, row after e, group); sequences whose span is invalid are left
+// alone (the RoPE kernel reports them).
+__global__ void __launch_bounds__(256) value_tail_zero_kernel(uint4* __restrict__ Vc, int B,
+                                                              int Tcap, int kv_rows,
+                                                              long long groups_per_row,
+                                                              const int* __restrict__ t0,
+                                                              const int* __restrict__ cu_seqlens) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long per_seq = 127 * groups_per_row;
+  if (gid >= (long long)B * per_seq) return;
+  const int seq = (int)(gid / per_seq);
+  const long long r = (gid % per_seq) / groups_per_row, g = gid % groups_per_row;
+  const long long off = __ldg(t0 + seq);
+  const long long n = (long long)__ldg(cu_seqlens + seq + 1) - __ldg(cu_seqlens + seq);
+  const long long e = off + n;
+  if (off < 0 || n < 0 || e > kv_rows) return;
+  const long long row = e + r;
+  if (row >= min((e + 127) / 128 * 128, (long long)kv_rows)) return;
+  Vc[((long long)seq * Tcap + row) * groups_per_row + g] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // SelfExtend rotations, fp16: query planes [2][B][L][Hq][D] at i (neighbour)
 // and floor(i/G) + W - floor(W/G) (grouped); key planes [2][B][L][Hkv][D] at
 // j and floor(j/G).  One thread per (row, head, 16-byte pair group).
@@ -594,6 +619,19 @@ cudaError_t launch_selfextend_rope(const void* Q, const void* K, void* Qse, void
   };
   if (D == 64) args(selfextend_rope_kernel<64>);
   else args(selfextend_rope_kernel<128>);
+  return cudaGetLastError();
+}
+}  // namespace dca
+
+namespace dca {
+cudaError_t launch_value_tail_zero(void* Vcache, int B, int Tcap, int kv_rows, int Hkv, int D,
+                                   const int* t0s, const int* cu_seqlens, cudaStream_t stream) {
+  using namespace rope_path;
+  const long long gpr = (long long)Hkv * D / 8;
+  const long long total = (long long)B * 127 * gpr;
+  if (total == 0) return cudaSuccess;
+  value_tail_zero_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
+      static_cast<uint4*>(Vcache), B, Tcap, kv_rows, gpr, t0s, cu_seqlens);
   return cudaGetLastError();
 }
 }  // namespace dca

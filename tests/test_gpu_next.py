@@ -423,6 +423,33 @@ def test_paged_decode_equals_contiguous_decode(block_rows):
     assert torch.equal(O1, O2) and torch.equal(L1, L2)
 
 
+
+@pytest.mark.parametrize("block_rows", [64, 256])
+def test_paged_decode_matches_oracle(block_rows):
+    # the paged call against the oracle directly, with the oracle reading the
+    # pool as stored: sequence b's position j is row j % P of pool block
+    # table[b][j // P] (gathered here on the CPU from the test's own pool)
+    dc = W.scaled(W.CONFIGS["decode_b16"], B=3, Tcap=4096, t_lo=100, t_hi=4096)
+    t, q, Kc, Vc = W.make_decode_inputs(dc, seed=4)
+    s, c = dc["s"], dc["c"]
+    Kp, table = _to_pool(Kc, block_rows, 5, 3)
+    Vp, _ = _to_pool(Vc, block_rows, 5, 3)
+    O, LSE = dca.dca_attn_decode_paged(q.cuda(), Kp.cuda(), Vp.cuda(), table.cuda(), t.cuda(),
+                                       s, c)
+    dca.dca_sync_status()
+    B, Tcap, Hkv, D = Kc.shape
+    idx = table.long()
+    Kg = Kp[idx].reshape(B, Tcap, Hkv, D)
+    Vg = Vp[idx].reshape(B, Tcap, Hkv, D)
+    heads = pu.sample_heads(dc["Hq"], dc["Hkv"]) + [21, 42]
+    O_ref, LSE_ref = orc.dca_decode(pu.F64View(q), pu.F64View(Kg), pu.F64View(Vg), t.numpy(),
+                                    s, c, heads=heads)
+    sel = np.ix_(range(B), heads)
+    err = np.abs(O.cpu().double().numpy()[sel] - O_ref[sel])
+    lse = np.abs(LSE.cpu().double().numpy()[sel] - LSE_ref[sel]) / np.maximum(
+        np.abs(LSE_ref[sel]), 1.0)
+    pu.assert_close(err.max(), err.mean(), lse.max(), f"paged decode P={block_rows}")
+
 def test_paged_append_then_decode_matches_contiguous():
     B, Hq, Hkv, D, T, s, c, rows = 2, 16, 2, 128, 1024, 256, 384, 128
     gen = torch.Generator().manual_seed(17)

@@ -356,6 +356,34 @@ def test_varlen_chunk_paged_equals_contiguous(case, block_rows):
     assert torch.isnan(Kp2[unused].float()).all() and torch.isnan(Vp2[unused].float()).all()
 
 
+
+@pytest.mark.parametrize("case", VARLEN_CHUNK_CASES[:2], ids=str)
+def test_varlen_chunk_paged_matches_oracle(case):
+    # the paged call against the oracle directly; the oracle reads each
+    # sequence's cached rows from the pool as stored, through its table row
+    lens, t0, Hq, Hkv, D, s, c, _ = case
+    block_rows = 128
+    max_kv = max(a + n for a, n in zip(t0, lens))
+    Tcap = (max_kv + block_rows - 1) // block_rows * block_rows
+    Q, K, V, Kc, Vc, cu = _chunk_inputs(lens, t0, Hq, Hkv, D, Tcap, seed=68)
+    B, nb = len(lens), Tcap // block_rows
+    num_blocks = B * nb + 2
+    perm = torch.randperm(num_blocks, generator=torch.Generator().manual_seed(69))[:B * nb]
+    Kp, Vp = _to_pool(Kc, block_rows, perm, num_blocks), _to_pool(Vc, block_rows, perm,
+                                                                   num_blocks)
+    table = perm.view(B, nb).to(torch.int32)
+    O, LSE = dca.dca_attn_prefill_varlen_chunk_paged(
+        Q.cuda(), K.cuda(), V.cuda(), Kp.cuda(), Vp.cuda(), table.cuda(), cu.cuda(),
+        torch.tensor(t0, dtype=torch.int32, device="cuda"), max(1, max(lens)), max_kv, s, c)
+    dca.dca_sync_status()
+    Kg = Kp[table.long()].reshape(B, Tcap, Hkv, D)
+    Vg = Vp[table.long()].reshape(B, Tcap, Hkv, D)
+    ref = orc.dca_prefill_varlen_chunk_rows(pu.F64View(Q), pu.F64View(K), pu.F64View(V),
+                                            cu.tolist(), t0, pu.F64View(Kg), pu.F64View(Vg),
+                                            s, c)
+    assert len(ref) == Hq * sum(lens)
+    _compare(O.cpu(), LSE.cpu(), ref, f"paged varlen chunk {case}")
+
 def test_varlen_chunk_paged_table_out_of_range_is_reported():
     lens, t0, Hq, Hkv, D, s, c = [100, 200], [300, 0], 2, 1, 128, 256, 384
     block_rows, Tcap = 128, 512
@@ -373,3 +401,66 @@ def test_varlen_chunk_paged_table_out_of_range_is_reported():
         dca.dca_sync_status()
     assert ei.value.status == 1
     dca.dca_sync_status()  # cleared; the context keeps working
+
+
+# ---------------------------------------------------------------------------
+# packed chunks with a caller-owned fp16 key mirror (no per-call conversion)
+# ---------------------------------------------------------------------------
+
+MIRROR_CASES = [
+    # full lengths, chunk boundaries per sequence (cumulative), Hq, Hkv, D, s, c
+    ([700, 1300, 257], [[0, 300, 301, 700], [0, 512, 1000, 1300], [0, 0, 256, 257]],
+     4, 2, 128, 256, 400),
+    ([900, 450], [[0, 100, 777, 900], [0, 449, 450, 450]], 2, 1, 64, 192, 256),
+]
+
+
+@pytest.mark.parametrize("case", MIRROR_CASES, ids=str)
+def test_varlen_chunk_mirror_chunks_equal_whole_prefill(case):
+    # each sequence is fed in three packed calls from an empty cache; every
+    # row must equal the row of a one-shot prefill over the whole sequence
+    # (the keys read back from the mirror were rounded once, to fp16, like a
+    # one-shot prefill's); caches start as NaN, so a row read before it is
+    # written shows
+    lens, bounds, Hq, Hkv, D, s, c = case
+    B, Tcap = len(lens), max(lens) + 128
+    gen = torch.Generator().manual_seed(70)
+    Qs = [torch.randn(n, Hq, D, generator=gen).to(torch.bfloat16) for n in lens]
+    Ks = [torch.randn(n, Hkv, D, generator=gen).to(torch.bfloat16) for n in lens]
+    Vs = [torch.randn(n, Hkv, D, generator=gen).to(torch.bfloat16) for n in lens]
+    Kc = torch.full((B, Tcap, Hkv, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Vc = torch.full_like(Kc, float("nan"))
+    Kf = torch.full((B, Tcap, Hkv, D), float("nan"), dtype=torch.float16, device="cuda")
+    ref = [orc.dca_prefill_rows(pu.F64View(Qs[b][None]), pu.F64View(Ks[b][None]),
+                                pu.F64View(Vs[b][None]), s, c) for b in range(B)]
+    for k in range(3):
+        t0 = [bounds[b][k] for b in range(B)]
+        ends = [bounds[b][k + 1] for b in range(B)]
+        n = [e - a for a, e in zip(t0, ends)]
+        cu = torch.zeros(B + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(n), 0).to(torch.int32)
+        pack = lambda X: torch.cat([X[b][t0[b]:ends[b]] for b in range(B)])
+        Q, K, V = pack(Qs), pack(Ks), pack(Vs)
+        if Q.shape[0] == 0:
+            continue
+        max_kv = max(ends)
+        O, LSE = dca.dca_attn_prefill_varlen_chunk_mirror(
+            Q.cuda(), K.cuda(), V.cuda(), Kc, Vc, Kf, cu.cuda(),
+            torch.tensor(t0, dtype=torch.int32, device="cuda"), max(1, max(n)), max_kv, s, c)
+        dca.dca_sync_status()
+        want = {}
+        for b in range(B):
+            for r in range(n[b]):
+                for h in range(Hq):
+                    want[(h, int(cu[b]) + r)] = ref[b][(0, h, t0[b] + r)]
+        _compare(O.cpu(), LSE.cpu(), want, f"mirror {case} call {k}")
+    # the caches hold every sequence's rows: values as given, keys rotated at
+    # j mod s (bf16 in the cache, fp16 in the mirror)
+    for b in range(B):
+        n = lens[b]
+        assert torch.equal(Vc[b, :n].cpu(), Vs[b])
+        ref_k = orc.rotate(Ks[b].double().numpy().transpose(1, 0, 2),
+                           orc.key_position(np.arange(n), s), 10000.0).transpose(1, 0, 2)
+        for cache, ulp in ((Kc, 2.0 ** -8), (Kf, 2.0 ** -11)):
+            err = np.abs(cache[b, :n].cpu().double().numpy() - ref_k)
+            assert (err <= np.abs(ref_k) * ulp + 1e-5).all(), (case, b)
