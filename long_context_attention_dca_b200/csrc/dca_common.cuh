@@ -103,6 +103,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// One lane of a converged warp, the same lane every time while all 32 are
+// active.  The MMA issuers run as whole warps so that their descriptors and
+// loop state are warp-uniform values; the elected lane issues the tcgen05
+// instructions and their commits (a commit tracks the MMAs of the thread
+// that issued them, so one lane must do both).
+__device__ __forceinline__ bool elect_one_lane() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// mbar_wait by every lane of a warp, with one answer for all of them.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, site));
+}
+
 // Where sequence b's rows sit in the prefill tensors.
 //   * Padded batch (cu_seqlens null): queries at tensor batch coordinate b,
 //     rows 0 .. L-1, at absolute indices q_off + r (q_off the call's chunk
