@@ -206,16 +206,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
       const uint64_t dk0 = smem_desc_sw128(sbase + kSmK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + kSmV, kBox, 1024);
       constexpr uint64_t kTileU = kTileBytes >> 4;
+      // Data readiness is checked ahead of the wait for P where it can be,
+      // so that once P is ready the MMAs follow without further waits.
+      int k_seen = -1, v_seen = -1;      // highest key / value tile seen to land
+      int q_seen[2] = {-1, -1};          // highest query load of tile A / B seen to land
+      auto phase_of = [&](int i) { return i >= b2 ? 2 : (i >= b1 ? 1 : 0); };
+      auto ensure_k = [&](int i) -> bool {
+        if (i <= k_seen) return true;
+        if (!warp_wait(bar(kKFull + (i & 1)), (i >> 1) & 1, abort_flag, 412)) return false;
+        k_seen = i;
+        return true;
+      };
+      auto ensure_v = [&](int i) -> bool {
+        if (i <= v_seen) return true;
+        if (!warp_wait(bar(kVFull + (i & 1)), (i >> 1) & 1, abort_flag, 414)) return false;
+        v_seen = i;
+        return true;
+      };
+      // the query rotation tile x uses at key tile i (load n = 2 * phase + x)
+      auto ensure_q = [&](int x, int i) -> bool {
+        const int n = 2 * phase_of(i) + x;
+        if (n <= (x ? q_seen[1] : q_seen[0])) return true;
+        const int slot = n >= 3 ? n - 3 : n;
+        if (!warp_wait(bar(kQFull + slot), n >= 3 ? 1u : 0u, abort_flag, 411)) return false;
+        if (x) q_seen[1] = n;
+        else q_seen[0] = n;
+        return true;
+      };
       auto issue_s = [&](int x, int i) -> bool {
-        const int p = i >= b2 ? 2 : (i >= b1 ? 1 : 0);
+        const int p = phase_of(i);
         const int n = 2 * p + x;              // Q load index: slot n % 3, use n / 3
         const int slot = n >= 3 ? n - 3 : n;
-        if ((i == 0 || i == b1 || i == b2) &&
-            !warp_wait(bar(kQFull + slot), n >= 3 ? 1u : 0u, abort_flag, 411))
-          return false;
-        const bool first_user = (x == 0) || (i >= nA);
-        if (first_user && !warp_wait(bar(kKFull + (i & 1)), (i >> 1) & 1, abort_flag, 412))
-          return false;
+        if (!ensure_q(x, i) || !ensure_k(i)) return false;
         tc_fence_after();
         const uint64_t dq = dq0 + (uint64_t)slot * kTileU;
         const uint64_t dk = dk0 + (uint64_t)(i & 1) * kTileU;
@@ -234,11 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         if (last_of_phase && leader) umma_commit(bar(kQEmpty + slot));
         return true;
       };
-      auto issue_pv = [&](int x, int i) -> bool {
+      // PV of tile x at key tile i; next_s is the key tile of the S MMA this
+      // tile issues right after it (-1: none), whose data is checked first
+      auto issue_pv = [&](int x, int i, int next_s) -> bool {
+        if (!ensure_v(i)) return false;
+        if (next_s >= 0 && !(ensure_q(x, next_s) && ensure_k(next_s))) return false;
         if (!warp_wait(bar(kPFull + x), i & 1, abort_flag, 413)) return false;
-        const bool first_user = (x == 0) || (i >= nA);
-        if (first_user && !warp_wait(bar(kVFull + (i & 1)), (i >> 1) & 1, abort_flag, 414))
-          return false;
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)(i & 1) * kTileU;
         const uint32_t pa = tmem + 128u * (uint32_t)x;
@@ -253,14 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
           umma_commit(bar(kVEmpty + (i & 1)));  // B is the last reader of V_i
         return true;
       };
-      bool ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0);
+      bool ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0, nA > 1 ? 1 : -1);
       for (int i = 1; i < nB && ok; ++i) {
         if (i < nA && !(ok = issue_s(0, i))) break;
-        if (!(ok = issue_pv(1, i - 1))) break;
+        if (!(ok = issue_pv(1, i - 1, i))) break;
         if (!(ok = issue_s(1, i))) break;
-        if (i < nA && !(ok = issue_pv(0, i))) break;
+        if (i < nA && !(ok = issue_pv(0, i, i + 1 < nA ? i + 1 : -1))) break;
       }
-      if (ok) issue_pv(1, nB - 1);
+      if (ok) issue_pv(1, nB - 1, -1);
       if (leader) umma_commit(bar(kMmaEnd));
       warp_wait(bar(kMmaEnd), 0, nullptr, 415);
     }
