@@ -18,9 +18,12 @@
 // Warps (384 threads, 3 warpgroups): 0-3 softmax A, 4-7 softmax B (row =
 // TMEM lane), 8 TMA producer, 9 TMEM allocator + UMMA issuer, 10-11 idle.
 // The issuer is the whole of warp 9 (warp-uniform descriptors and loop
-// state, one elected lane issuing the MMAs and their commits): against a
-// single-lane issuer, each key tile's MMAs reach the tensor core sooner
-// (clock64 trace: 4236 -> 4021 SM cycles per key tile on the 7B shape).
+// state, one elected lane issuing the MMAs and their commits).  The issuer
+// warp shares its SMSP with two softmax warps and runs its own
+// instructions slowly, so the path from "P is ready" to the next score MMA
+// holds nothing but MMAs and commits: each PV group is fused with the score
+// group the same tile issues next, and their data (value tile, key tile,
+// query slot) is checked before the wait for P.
 // Registers are rebalanced after set-up: the producer/issuer warpgroup drops
 // to 72 per thread, the softmax warpgroups rise to 216 (2*128*216 + 128*72 =
 // 384 * 168, the launch allotment).
@@ -256,16 +259,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         if (last_of_phase && leader) umma_commit(bar(kQEmpty + slot));
         return true;
       };
-      // PV of tile x at key tile i; next_s is the key tile of the S MMA this
-      // tile issues right after it (-1: none), whose data is checked first
-      auto issue_pv = [&](int x, int i, int next_s) -> bool {
+      // PV of tile x at key tile i, then (next_s >= 0) the score MMA of the
+      // same tile at key tile next_s.  Everything the two groups need is
+      // computed and checked before the wait for P, so that once P is ready
+      // only the MMAs and their commits run.
+      auto issue_pv_s = [&](int x, int i, int next_s) -> bool {
         if (!ensure_v(i)) return false;
         if (next_s >= 0 && !(ensure_q(x, next_s) && ensure_k(next_s))) return false;
-        if (!warp_wait(bar(kPFull + x), i & 1, abort_flag, 413)) return false;
-        tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)(i & 1) * kTileU;
         const uint32_t pa = tmem + 128u * (uint32_t)x;
         const uint32_t od = tmem + 256u + 128u * (uint32_t)x;
+        const int p = next_s >= 0 ? phase_of(next_s) : 0;
+        const int n = 2 * p + x;
+        const int slot = n >= 3 ? n - 3 : n;
+        const uint64_t dq = dq0 + (uint64_t)slot * kTileU;
+        const uint64_t dk = dk0 + (uint64_t)(next_s & 1) * kTileU;
+        const int next_begin = p == 0 ? b1 : (p == 1 ? b2 : kNever);
+        const bool last_of_phase =
+            next_begin != kNever ? (next_s == next_begin - 1) : (next_s == (x ? nB : nA) - 1);
+        if (!warp_wait(bar(kPFull + x), i & 1, abort_flag, 413)) return false;
+        tc_fence_after();
         if (leader) umma_ts(od, pa, dv, idesc_o, i > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < kTile / 16; ++kk)
@@ -274,16 +287,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
         if (leader) umma_commit(bar(kODone + x));
         if (x == 1 && leader)
           umma_commit(bar(kVEmpty + (i & 1)));  // B is the last reader of V_i
+        if (next_s < 0) return true;
+        const uint32_t d = tmem + 128u * (uint32_t)x;
+#pragma unroll
+        for (int kk = 0; kk < kHD / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+          if (leader) umma_ss(d, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        if (leader) umma_commit(bar(kSFull + x));
+        if (x == 1 && leader)
+          umma_commit(bar(kKEmpty + (next_s & 1)));  // B is the last reader of K_next_s
+        if (last_of_phase && leader) umma_commit(bar(kQEmpty + slot));
         return true;
       };
-      bool ok = issue_s(0, 0) && issue_s(1, 0) && issue_pv(0, 0, nA > 1 ? 1 : -1);
-      for (int i = 1; i < nB && ok; ++i) {
-        if (i < nA && !(ok = issue_s(0, i))) break;
-        if (!(ok = issue_pv(1, i - 1, i))) break;
-        if (!(ok = issue_s(1, i))) break;
-        if (i < nA && !(ok = issue_pv(0, i, i + 1 < nA ? i + 1 : -1))) break;
+      // order: S_A(0), S_B(0), then per key tile i: PV_A(i) + S_A(i+1),
+      // PV_B(i) + S_B(i+1) (the same sequence of MMAs as before)
+      bool ok = issue_s(0, 0) && issue_s(1, 0);
+      for (int i = 0; i < nB && ok; ++i) {
+        if (i < nA && !(ok = issue_pv_s(0, i, i + 1 < nA ? i + 1 : -1))) break;
+        if (!(ok = issue_pv_s(1, i, i + 1 < nB ? i + 1 : -1))) break;
       }
-      if (ok) issue_pv(1, nB - 1, -1);
       if (leader) umma_commit(bar(kMmaEnd));
       warp_wait(bar(kMmaEnd), 0, nullptr, 415);
     }
