@@ -216,6 +216,8 @@ def run_ours(args, rank, world, dev):
     pc = W.CONFIGS[args.workload]
     if args.override_s:  # profiling runs of the straddling-tile kernel
         pc = dict(pc, s=args.override_s)
+    if args.override_d:  # profiling runs of the D = 64 instantiation
+        pc = dict(pc, D=args.override_d)
     dc = W.CONFIGS[DECODE]
     Q, K, V = W.make_prefill_inputs(pc, device=dev)
     B, L, Hq, D = Q.shape
@@ -899,6 +901,9 @@ def main():
     ap.add_argument("--override-s", type=int, default=0,
                     help="profiling runs: chunk size s of the prefill workload (e.g. 3000, "
                          "whose tiles straddle chunk boundaries)")
+    ap.add_argument("--override-d", type=int, default=0, choices=[0, 64, 128],
+                    help="profiling runs: head dim of the prefill workload (64 runs the "
+                         "interval kernel's D = 64 instantiation)")
     ap.add_argument("--e2e-chunk", type=int, default=0,
                     help="rows per chunk of the host-buffer prefill in the e2e leg "
                          "(0: 8192 above 32k tokens, else 2048)")
