@@ -61,6 +61,26 @@ __device__ __forceinline__ bool f16x8_nonfinite(const uint4& v) {
   return f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) |
          f16x2_nonfinite(v.w);
 }
+// Range check by arithmetic: acc + w·0 over the fp16 pairs of a 16-byte
+// half-row pair (lo, hi).  w·0 is ±0 for a finite w and NaN for ±inf or NaN,
+// so the two accumulators (started at +0) stay +0 while every value is finite
+// and turn NaN at the first that is not: one f16x2 fma per word.
+__device__ __forceinline__ uint32_t f16x2_fma0(uint32_t w, uint32_t acc) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(0u), "r"(acc));
+  return r;
+}
+__device__ __forceinline__ void f16_range_acc(const uint4& lo, const uint4& hi, uint32_t& a0,
+                                              uint32_t& a1) {
+  a0 = f16x2_fma0(lo.x, a0);
+  a1 = f16x2_fma0(lo.y, a1);
+  a0 = f16x2_fma0(lo.z, a0);
+  a1 = f16x2_fma0(lo.w, a1);
+  a0 = f16x2_fma0(hi.x, a0);
+  a1 = f16x2_fma0(hi.y, a1);
+  a0 = f16x2_fma0(hi.z, a0);
+  a1 = f16x2_fma0(hi.w, a1);
+}
 
 // Device error sites of the fp16 range check (reported as a bad argument).
 constexpr int kSiteRopeF16Range = 106;
@@ -235,7 +255,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
   const int heads = Hq + (kChunk ? 2 : 1) * Hkv;  // [keys | (values) | queries]
   const bool write_kc = Kout != nullptr, write_v = Vc != nullptr;
   const int items = nrows * heads * kGroups;
-  bool bad = false;  // an fp16 output of a row of some sequence is not finite
+  uint32_t bad = 0u;  // nonzero: an fp16 output of a row of some sequence is not finite
 #pragma unroll 2
   for (int it = threadIdx.x; it < items; it += kRopeThreads) {
     const int g = it % kGroups;
@@ -276,7 +296,9 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
           *reinterpret_cast<uint4*>(Kc + dst + kHalf) = ohi;
         }
         rotate8<true>(lo, hi, cs, olo, ohi);
-        bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
+        uint32_t a0 = 0u, a1 = 0u;
+        f16_range_acc(olo, ohi, a0, a1);
+        if (live_s[r]) bad |= a0 | a1;
         const size_t hdst = (((size_t)seq * kh_rows + pos_s[r]) * Hkv + hh) * D + g * 8;
         *reinterpret_cast<uint4*>(Kh + hdst) = olo;
         *reinterpret_cast<uint4*>(Kh + hdst + kHalf) = ohi;
@@ -301,8 +323,10 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
     rotate8<true>(lo, hi, cs, olo, ohi);
     // each plane is checked: a rotation keeps a pair's norm, not its
     // largest component, so one angle can overflow where another does not
-    bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
+    uint32_t a0 = 0u, a1 = 0u;
+    f16_range_acc(olo, ohi, a0, a1);
     if (is_k) {
+      if (live_s[r]) bad |= a0 | a1;
       __half* Krot = static_cast<__half*>(Kout);
       *reinterpret_cast<uint4*>(Krot + off) = olo;
       *reinterpret_cast<uint4*>(Krot + off + kHalf) = ohi;
@@ -317,7 +341,7 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
       cs.s[e] = v.y;
     }
     rotate8<true>(lo, hi, cs, olo, ohi);  // inter plane (c - 1)
-    bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
+    f16_range_acc(olo, ohi, a0, a1);
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off) = olo;
     *reinterpret_cast<uint4*>(Qrot + 2 * plane + off + kHalf) = ohi;
     if (query_pos_for_piece(kSucc, im_s[r], s, c) != c - 1) {
@@ -328,12 +352,13 @@ __global__ void __launch_bounds__(kRopeThreads) prefill_rope_kernel(
         cs.s[e] = v.y;
       }
       rotate8<true>(lo, hi, cs, olo, ohi);
-      bad |= live_s[r] & (f16x8_nonfinite(olo) | f16x8_nonfinite(ohi));
+      f16_range_acc(olo, ohi, a0, a1);
     }
     *reinterpret_cast<uint4*>(Qrot + plane + off) = olo;  // successive plane
     *reinterpret_cast<uint4*>(Qrot + plane + off + kHalf) = ohi;
+    if (live_s[r]) bad |= a0 | a1;
   }
-  if (bad) report_error(kDevBadArg, kSiteRopeF16Range);
+  if ((bad & 0x7FFF7FFFu) != 0u) report_error(kDevBadArg, kSiteRopeF16Range);
 }
 
 // Decode-time append: rotate the new key of sequence b at t[b] mod s and
