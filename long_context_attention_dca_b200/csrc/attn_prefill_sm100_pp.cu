@@ -30,6 +30,8 @@
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // Shared memory: 3 rotating Q slots (the query rotation of each piece, loaded
 // in order of first use: A then B for each piece), K ring of 2, V ring of 2.
+// A pair whose rows all have i mod s >= c - s walks the inter and successive
+// key tiles as one piece (both query positions are c - 1).
 // The online softmax keeps running max / sum in fp32 (log2 domain); O is
 // rescaled in TMEM only when a warp's max grew by more than 2^8.
 // Every mbarrier wait is bounded; on expiry the CTA records an error, drains
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
     float* __restrict__ LSE, int B, int L, int Hq, int Hkv, int s, float scale_log2,
-    int pair_off, int group_units, const int* __restrict__ cu_seqlens, int T) {
+    int pair_off, int group_units, const int* __restrict__ cu_seqlens, int T, int w_merge) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -102,12 +104,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_attn_pp_kernel(
   const int tpc = s / kTile;
   // DCA pieces met by this query-tile pair, in walk order: phase p uses Qrot
   // plane n_ph - 1 - p (inter = 2, successive = 1, intra = 0) and starts at key
-  // tile 0, b1 or b2 (kNever when the phase does not exist).
+  // tile 0, b1 or b2 (kNever when the phase does not exist).  When every row
+  // of the pair has i mod s >= w (= c - s), its successive and inter query
+  // positions are both c - 1, and the successive plane (bit-identical to the
+  // inter plane for those rows) serves the inter key tiles too: the two
+  // pieces are walked as one phase, with one query load fewer per tile.
+  // (The pair lies in one chunk since s % 256 == 0; i mod s grows along it.)
   const int ci = q0 / s;
-  const int n_ph = ci >= 2 ? 3 : ci + 1;
+  const bool merged = ci >= 2 && q0 % s >= w_merge;
+  const int n_ph = merged ? 2 : (ci >= 2 ? 3 : ci + 1);
   constexpr int kNever = 0x7fffffff;
-  const int b1 = ci >= 2 ? (ci - 1) * tpc : (ci == 1 ? tpc : kNever);
-  const int b2 = ci >= 2 ? ci * tpc : kNever;
+  const int b1 = merged ? ci * tpc : (ci >= 2 ? (ci - 1) * tpc : (ci == 1 ? tpc : kNever));
+  const int b2 = !merged && ci >= 2 ? ci * tpc : kNever;
   const int nA = 2 * m + 1;  // key tiles 0 .. 2m   (diagonal of A)
   const int nB = 2 * m + 2;  // key tiles 0 .. 2m+1 (diagonal of B)
 
@@ -418,7 +426,7 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
                                          int q_off, int k_rows, int v_rows,
-                                         const int* cu_seqlens, int T) {
+                                         const int* cu_seqlens, int T, int c) {
   using namespace pp_path;
   if (D != kHD || s % (2 * kTile) != 0 || q_off % (2 * kTile) != 0) return cudaErrorInvalidValue;
   if (cu_seqlens != nullptr && (q_off != 0 || T < 1)) return cudaErrorInvalidValue;
@@ -460,7 +468,7 @@ cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, con
                                              B, L, Hq, Hkv, s, scale * 1.4426950408889634f,
                                              q_off / (2 * kTile),
                                              pair_group_units(B, Hkv, cu_seqlens ? L : Lkv, D),
-                                             cu_seqlens, T);
+                                             cu_seqlens, T, c > s ? c - s : 0x7fffffff);
   return cudaGetLastError();
 }
 

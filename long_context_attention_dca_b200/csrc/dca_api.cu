@@ -211,7 +211,8 @@ dca_status_t dca_prefill_attention(const void* V, void* O, float* LSE, int B, in
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (path == DCA_PATH_TCGEN05 && D == 128 && s % 256 == 0)
-    e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
+    e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm, 0,
+                                     0, 0, nullptr, 0, c);
   else if (path == DCA_PATH_TCGEN05)  // tiles or tile pairs straddle chunk boundaries
     e = launch_prefill_attn_sm100_gen(ws.qrot, ws.krot, V, O, LSE, B, L, Hq, Hkv, D, s, sc, strm);
   else
@@ -265,7 +266,7 @@ dca_status_t dca_attn_prefill_varlen(const void* Q, const void* K, const void* V
   if (e == cudaSuccess) {
     if (D == 128 && s % 256 == 0)
       e = launch_prefill_attn_sm100_pp(ws.qrot, ws.krot, V, O, LSE, B, max_seqlen, Hq, Hkv, D, s,
-                                       sc, strm, 0, 0, 0, cu_seqlens, T);
+                                       sc, strm, 0, 0, 0, cu_seqlens, T, c);
     else
       e = launch_prefill_attn_sm100_gen(ws.qrot, ws.krot, V, O, LSE, B, max_seqlen, Hq, Hkv, D, s,
                                         sc, strm, 0, 0, 0, cu_seqlens, T);
@@ -354,7 +355,7 @@ dca_status_t dca_attn_prefill_chunk(const void* Q, const void* K, const void* V,
   if (e != cudaSuccess) return cuda_fail(e, fn);
   if (auto_path(D, s) == DCA_PATH_TCGEN05 && D == 128 && s % 256 == 0 && t0 % 256 == 0)
     e = launch_prefill_attn_sm100_pp(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
-                                     strm, t0, t0 + Lq, Tcap);
+                                     strm, t0, t0 + Lq, Tcap, nullptr, 0, c);
   else if (auto_path(D, s) == DCA_PATH_TCGEN05)
     e = launch_prefill_attn_sm100_gen(workspace, kf16, Vcache, O, LSE, B, Lq, Hq, Hkv, D, s, sc,
                                       strm, t0, t0 + Lq, Tcap);

@@ -69,11 +69,15 @@ cudaError_t launch_merge3(const float* Op, const float* LSEp, void* O, float* LS
 // 0 .. q_off+L-1 held with k_rows / v_rows rows per sequence (0: q_off + L).
 // Packed form (cu_seqlens device [B+1], q_off 0): Qrot [3][T][Hq][D], Krot and
 // V [T][Hkv][D], O [T][Hq][D], LSE [Hq][T]; B sequences of at most L rows.
+// c > 0: the successive and inter pieces of a tile pair whose rows all have
+// i mod s >= c - s are walked as one (both query positions are c - 1, so the
+// successive plane, which the RoPE pass writes bit-identical to the inter
+// plane there, serves both); c = 0 keeps three pieces.
 cudaError_t launch_prefill_attn_sm100_pp(const void* Qrot, const void* Krot, const void* V,
                                          void* O, float* LSE, int B, int L, int Hq, int Hkv,
                                          int D, int s, float scale, cudaStream_t stream,
                                          int q_off = 0, int k_rows = 0, int v_rows = 0,
-                                         const int* cu_seqlens = nullptr, int T = 0);
+                                         const int* cu_seqlens = nullptr, int T = 0, int c = 0);
 // tcgen05 prefill attention for any chunk size (D = 64 or 128): per-row key
 // intervals per piece, straddling tiles visited once per piece they hold.
 // Same chunk and packed forms as the ping-pong variant (any q_off), and

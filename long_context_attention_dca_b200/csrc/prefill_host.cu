@@ -147,7 +147,7 @@ extern "C" dca_status_t dca_attn_prefill_host(const void* Q, const void* K, cons
     if (e == cudaSuccess) {
       if (pp)
         e = launch_prefill_attn_sm100_pp(w.qrot, w.kh, w.vd, w.oc[slot], w.lc[slot], B, Lq, Hq,
-                                         Hkv, D, s, sc, cs, a, L, L);
+                                         Hkv, D, s, sc, cs, a, L, L, nullptr, 0, c);
       else if (tc)
         e = launch_prefill_attn_sm100_gen(w.qrot, w.kh, w.vd, w.oc[slot], w.lc[slot], B, Lq, Hq,
                                           Hkv, D, s, sc, cs, a, L, L);

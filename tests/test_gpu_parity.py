@@ -145,6 +145,7 @@ SMALL = [  # (B, L, Hq, Hkv, D, s, c)
     (1, 1300, 2, 2, 128, 256, 4096),   # w > s
     (1, 129, 2, 2, 128, 256, 300),
     (1, 2200, 4, 1, 128, 512, 640),
+    (1, 2600, 4, 2, 128, 512, 768),    # pairs at i mod s = 256 >= w: inter + successive in one walk
     # D = 128, s not a multiple of 128: tiles straddle chunk boundaries
     (1, 1000, 2, 1, 128, 192, 256),
     (2, 777, 4, 2, 128, 100, 150),
