@@ -358,24 +358,31 @@ dca_status_t dca_attn_prefill_selfextend(const void* Q, const void* K, const voi
 
 /* Device workspace bytes for dca_attn_prefill_host with chunks of chunk_rows
  * rows: the whole sequence's rotated keys (fp16) and values, plus two
- * chunk-sized sets of staging and output buffers.  Returns 0 for unsupported
- * arguments. */
+ * chunk-sized sets of staging, query-rotation and output buffers (one set per
+ * compute stream).  Returns 0 for unsupported arguments. */
 size_t dca_attn_prefill_host_workspace(int B, int L, int Hq, int Hkv, int D, int chunk_rows);
 
 /* dca_attn_prefill with HOST buffers: Q, K, V are read from and O, LSE
  * written to host memory (same layouts as dca_attn_prefill), with the PCIe
- * copies overlapped with the attention.  The sequence is processed in chunks
- * of chunk_rows rows; chunk k is the chunked prefill of rows k*chunk_rows ..
- * against the keys before it (the index rule depends only on absolute
- * indices), so the results equal dca_attn_prefill's.  Copies of chunk k+1 in,
+ * copies overlapped with the attention and consecutive chunks' kernels on two
+ * compute streams (chunk k's attention needs only earlier chunks' keys and
+ * values, so it can start while chunk k-1's attention finishes).  The sequence is processed in chunks
+ * of at most chunk_rows rows; when chunk_rows is a multiple of 256 and at
+ * least 1024 the first chunks are shorter (chunk_rows/16 rounded down to a
+ * multiple of 256, at least 256, doubling up to chunk_rows), since the copy
+ * of the first rows is not hidden by any computation.  Each chunk is the
+ * chunked prefill of its rows against the keys before them (the index rule
+ * depends only on absolute indices), so the results equal
+ * dca_attn_prefill's.  Copies of chunk k+1 in,
  * the kernels of chunk k and the copies of chunk k-1's results out run
  * concurrently; this serves DCA as a drop-in wrapper on a host-fed pipeline
  * (Guide, "Strategic Recommendations", item 1).
  *   - Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister):
  *     with pageable memory the copies serialise.
- *   - Kernels run on `stream`; the call creates two copy streams and its
- *     events and releases them before returning (they are freed once the
- *     queued work is done), so it cannot be captured into a CUDA graph.
+ *   - Kernels run on `stream` and on a second compute stream; the call
+ *     creates that stream, two copy streams and its events and releases
+ *     them before returning (they are freed once the queued work is done),
+ *     so it cannot be captured into a CUDA graph.
  *     Work queued on `stream` after the call runs after the last copy out.
  *   - Kernels: tcgen05 (the two-tile kernel when D == 128, s % 256 == 0 and
  *     chunk_rows is a multiple of 256 or covers the sequence, the

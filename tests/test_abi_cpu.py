@@ -99,11 +99,12 @@ def test_workspace_queries(lib):
         up(3 * 2 * 100 * 8 * 128 * 2) + up(2 * 150 * 2 * 128 * 2))
     assert dca.dca_attn_prefill_chunk_workspace(2, 100, 8, 2, 128, -1) == 0
     # host prefill: whole-sequence fp16 keys and values + two chunk-sized sets
-    # of staging (Q, K), outputs (O, LSE) and one chunk's three query rotations
+    # of staging (Q, K), outputs (O, LSE) and three query rotations (one set
+    # per compute stream)
     B, L, Hq, Hkv, D, C = 2, 1000, 8, 2, 64, 300
     want = 2 * up(B * L * Hkv * D * 2) + 2 * (up(B * C * Hq * D * 2) + up(B * C * Hkv * D * 2) +
                                               up(B * C * Hq * D * 2) + up(B * Hq * C * 4)) + \
-        up(3 * B * C * Hq * D * 2)
+        2 * up(3 * B * C * Hq * D * 2)
     assert dca.dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, C) == want
     assert dca.dca_attn_prefill_host_workspace(B, L, Hq, Hkv, D, 0) == 0
     # SelfExtend: neighbour + grouped rotations of Q and K, fp16
