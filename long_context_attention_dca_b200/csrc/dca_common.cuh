@@ -235,7 +235,7 @@ __device__ __forceinline__ void reg_dealloc() {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled tensor copies; never with cluster multicast)
+// TMA (tiled tensor copies, each into the issuing CTA's own shared memory)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(desc) : "memory");
