@@ -100,8 +100,7 @@ extern "C" dca_status_t dca_attn_prefill_host(const void* Q, const void* K, cons
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf((float)D);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // chunk starts: short first chunks doubling up to C (C % 256 == 0, C >= 1024),
-  // else C rows each; every start but the first C-capped ones stays a
-  // multiple of 256 exactly when C is
+  // else C rows each; all starts are multiples of 256 when C is
   int first = C;
   if (C % 256 == 0 && C >= 1024) first = (C / 16) / 256 * 256 < 256 ? 256 : (C / 16) / 256 * 256;
   int n_chunks = 0;
